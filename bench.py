@@ -1,0 +1,481 @@
+"""Benchmark of the EntmaxKV support-aware paged α-entmax decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode token for every (sequence, KV head) unit of the
+workload: cache append + tail-page metadata, bounding-box page scores, top-k
+page selection, sparse α-entmax attention (scores over the selected K, τ,
+support-only V).  Inputs are resident in HBM; L2 is flushed (256 MiB write)
+between steps.  Prints one JSON line on rank 0.
+
+Workload (default): the clustered 128k-context decode — batch 4, 32 query /
+8 KV heads, d = 128, page size 16, bf16 cache, top-k k = 256, α = 1.5.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "entmax decode steps/s per (batch×KV-head) at 128k ctx; HBM GB/s vs roofline"
+UNIT = "(sequence×KV-head) decode steps/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of one score-kernel launch at the default workload, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of
+# the kernel's sources; stale entries read as null.
+SCORE_TRAFFIC = {}
+
+
+def kernel_hash(files=("score.cu", "common.cuh", "kernels.cuh")):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "sparse_kv_cache_kmax_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_timing(elapsed_s: float, units_done: int, group=None):
+    """Max elapsed time over ranks and total units over ranks (whole job)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return elapsed_s, units_done
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
+    u = torch.tensor([units_done], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), int(u.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        mhz, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if self.uuid and parts[1] != self.uuid:
+                    continue
+                try:
+                    mhz.append(float(parts[2]))
+                    mx.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[6:10]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- bytes
+def algorithmic_bytes(inp, eng, support_pages):
+    """Bytes one step must move: metadata rows, q, ub, selected K, V of
+    support pages, outputs, and the append (tail page + new rows + metadata)."""
+    wl = inp["workload"]
+    es = inp["k_pool"].element_size()
+    d, S, G = wl.head_dim, wl.page_size, wl.group
+    lens = inp["seq_lens"].tolist()
+    pages = [-(-L // S) for L in lens]
+    units_pages = sum(pages) * wl.num_kv_heads
+    meta = units_pages * 2 * d * es
+    q = wl.batch * wl.num_q_heads * d * es
+    ub = units_pages * 4
+    n_sel = eng.n_sel.to(torch.int64)
+    sel_tokens = int(n_sel.sum()) * S                     # full pages (tail rounding ignored)
+    selK = sel_tokens * d * es
+    supV = int(support_pages) * S * d * es
+    out = wl.batch * wl.num_q_heads * d * 4
+    append = wl.units * (S * d * es + 2 * d * es + 4 * d * es)
+    return {"meta": meta, "q": q, "ub": ub, "sel_k": selK, "support_v": supV, "out": out,
+            "append": append, "score_kernel": meta + q + ub,
+            "step": meta + q + selK + supV + out + append}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    from sparse_kv_cache_kmax_b200 import binding as Bd
+    from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    Bd.lib()                                   # fail loudly if the library is missing
+
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, seed=3000 + rank, device=dev, n_new=1)
+    q, k_new, v_new = inp["q"], inp["k_new"][0], inp["v_new"][0]
+    alpha, k = args.alpha, args.k or wl.topk
+    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
+                       policy="topk", k=k, alpha=alpha)
+    eng.build_meta()
+    cache, seqs, Hq = eng.cache, eng.seqs, wl.num_q_heads
+    scale = float(np.float32(wl.scale))
+    ub = torch.empty(wl.batch, wl.num_kv_heads, inp["max_pages"], device=dev)
+    dec_ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, cache, seqs, Hq, k), dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def stage_step(ev):
+        ev[0].record(stream)
+        Bd.ekv_append(cache, seqs, k_new, v_new, stream)
+        ev[1].record(stream)
+        Bd.ekv_score_pages(cache, seqs, q, scale, ub, stream)
+        ev[2].record(stream)
+        Bd.ekv_select_topk(seqs, wl.num_kv_heads, wl.page_size, ub, k, eng.sel, eng.n_sel, stream)
+        ev[3].record(stream)
+        Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws, stream=stream)
+        ev[4].record(stream)
+
+    def timed(step_fn, n_events, steps, warmup):
+        for _ in range(warmup):
+            flush.zero_()
+            step_fn([torch.cuda.Event(enable_timing=True) for _ in range(n_events)])
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            step_fn(evs[i])
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
+        return per                              # ms, [steps, stages]
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    with ClockSampler(uuid) as clk:
+        per = timed(stage_step, 5, args.steps, args.warmup)
+    stages = per.mean(axis=0)
+    step_ms = float(per.sum(axis=1).mean())
+    total_s = float(per.sum()) / 1e3
+    max_s, units_all = reduce_timing(total_s, wl.units * args.steps)
+    value = units_all / max_s
+    clocks = clk.summary()
+
+    # support statistics of the last step (untimed): pages whose V the step read
+    words = (k * wl.page_size + 31) // 32
+    bits = torch.zeros(wl.batch, Hq, words, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=dev)
+    Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws,
+                         support_count=cnt, support_bits=bits)
+    tok = ((bits.view(torch.int32).unsqueeze(-1) >> torch.arange(32, device=dev, dtype=torch.int32)) & 1)
+    tok = tok.view(wl.batch, wl.num_kv_heads, wl.group, -1).amax(dim=2)          # union over the group
+    page_sup = tok.view(wl.batch, wl.num_kv_heads, k, wl.page_size).amax(dim=-1)
+    support_pages = int(page_sup.sum())
+    nb = algorithmic_bytes(inp, eng, support_pages)
+
+    peak, peak_kind = hbm_peak()
+    score_ms = float(stages[1])
+    achieved = nb["score_kernel"] / (score_ms * 1e-3) / 1e9
+    h = kernel_hash()
+    traffic = SCORE_TRAFFIC.get(h)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: batch {wl.batch}, {wl.num_q_heads} q / {wl.num_kv_heads} KV heads, "
+                               f"d {wl.head_dim}, context {wl.context}, page size {wl.page_size}",
+                   "policy": "topk", "k": k, "alpha": alpha, "global_batch": wl.batch * world,
+                   "seq_len": wl.context, "parallelism": f"replicas x{world} (units sharded, no collective)",
+                   "l2": "flushed between steps (256 MiB write)"},
+        "steps_per_s": 1e3 / step_ms,
+        "stages_us": {"append": stages[0] * 1e3, "score": stages[1] * 1e3, "topk": stages[2] * 1e3,
+                      "decode": stages[3] * 1e3},
+        "roofline": {"bound": "hbm", "kernel": "score (bounding-box page scores)", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
+                     "algorithmic_bytes": nb["score_kernel"]},
+        "step_roofline": {"bytes": nb["step"], "achieved_gbs": nb["step"] / (step_ms * 1e-3) / 1e9,
+                          "frac": nb["step"] / (step_ms * 1e-3) / 1e9 / peak,
+                          "breakdown": {kk: v for kk, v in nb.items() if kk not in ("step", "score_kernel")}},
+        "support": {"mean_sel_pages": float(eng.n_sel.float().mean()), "support_pages_per_unit":
+                    support_pages / wl.units, "mean_support_tokens_per_head": float(cnt.float().mean())},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks,
+    }
+
+    if not args.quick:
+        result["gauss"] = bench_policy(args, wl, inp, "gauss", dev, flush)
+        result["full_cache"] = bench_policy(args, wl, inp, "full", dev, flush)
+        result["full_cache_dense_v"] = bench_policy(args, wl, inp, "full", dev, flush, dense_v=True)
+        result["e2e"] = bench_e2e(args, wl, inp, eng, dev, flush, world)
+    if rank == 0 and world == 1 and not args.quick:
+        result["cpu_baseline"] = cpu_baseline(wl, inp, k, alpha, budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def bench_policy(args, wl, inp, policy, dev, flush, dense_v=False):
+    """Whole-step timing (one ekv_decode_step call) of another policy."""
+    from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+
+    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
+                       policy=policy, k=wl.topk, delta=wl.delta if wl.delta is not None else 0.5,
+                       alpha=args.alpha, dense_v=dense_v)
+    eng.build_meta()
+    steps = max(3, min(args.steps, 200 if policy == "full" else args.steps))
+    for _ in range(args.warmup):
+        flush.zero_()
+        eng.step(inp["q"], inp["k_new"][0], inp["v_new"][0])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        eng.step(inp["q"], inp["k_new"][0], inp["v_new"][0])
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    res = {"ms_per_step": ms, "value": wl.units / (ms * 1e-3), "unit": UNIT, "steps": steps,
+           "mean_sel_pages": float(eng.n_sel.float().mean()) if policy != "full" else float(inp["max_pages"])}
+    if policy == "full":
+        es = inp["k_pool"].element_size()
+        kv = sum(int(L) for L in inp["seq_lens"].tolist()) * wl.num_kv_heads * wl.head_dim * es
+        res["k_bytes"] = kv
+        res["dense_v"] = bool(dense_v)
+    return res
+
+
+def bench_e2e(args, wl, inp, eng, dev, flush, world):
+    """Same step through the public one-call API with host buffers: pinned
+    H2D of q, k_new, v_new, the step, and D2H of the output, per step."""
+    q_h = inp["q"].cpu().pin_memory()
+    k_h = inp["k_new"][0].cpu().pin_memory()
+    v_h = inp["v_new"][0].cpu().pin_memory()
+    out_h = torch.empty(eng.out.shape, dtype=eng.out.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(inp["q"]), torch.empty_like(inp["k_new"][0]), torch.empty_like(inp["v_new"][0])
+    steps = max(3, min(args.steps, 500))
+
+    def one():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        eng.step(q_d, k_d, v_d)
+        out_h.copy_(eng.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        one()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(b) for a, b in ev) / 1e3
+    max_s, units_all = reduce_timing(total, wl.units * steps)
+    h2d = q_h.numel() * q_h.element_size() + 2 * k_h.numel() * k_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+    return {"value": units_all / max_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": total / steps * 1e3, "steps": steps}
+
+
+# ---------------------------------------------------------------- the oracle, timed
+def oracle_step_units(wl, host_units, k, alpha, budget_s):
+    """Run the oracle's decode step on host copies of some units until
+    budget_s of CPU time is spent; returns (unit-steps done, seconds)."""
+    import oracle as O
+
+    scale = float(np.float32(wl.scale))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for (kp, vp, n_valid, qg, meta) in host_units:
+            # append: refresh the tail page's metadata
+            last = len(n_valid) - 1
+            tail = O.page_metadata(kp[last:last + 1], n_valid[last:last + 1], wl.dtype)
+            for f in meta:
+                meta[f][last] = tail[f][0]
+            ub = O.bbox_upper_bound(qg, meta["kmax"], meta["kmin"], scale)
+            sel = O.select_topk(O.page_scores(ub), k)
+            Ks = np.concatenate([kp[p, : n_valid[p]] for p in sel])
+            Vs = np.concatenate([vp[p, : n_valid[p]] for p in sel])
+            O.entmax_attention(qg, Ks, Vs, scale, alpha)
+            done += 1
+            if time.perf_counter() - t0 >= budget_s:
+                return done, time.perf_counter() - t0
+
+
+def host_units_sample(wl, inp, n_units):
+    import oracle as O
+
+    units = []
+    for u in range(n_units):
+        b, h = divmod(u, wl.num_kv_heads)
+        L = int(inp["seq_lens"][b])
+        P = -(-L // wl.page_size)
+        ids = inp["page_table"][b, :P].long()
+        kp = inp["k_pool"][ids, h].double().cpu().numpy()
+        vp = inp["v_pool"][ids, h].double().cpu().numpy()
+        n_valid = np.minimum(wl.page_size, L - wl.page_size * np.arange(P))
+        qg = inp["q"][b, h * wl.group:(h + 1) * wl.group].double().cpu().numpy()
+        meta = O.page_metadata(kp, n_valid, wl.dtype)
+        units.append((kp, vp, n_valid, qg, meta))
+    return units
+
+
+def cpu_baseline(wl, inp, k, alpha, budget_s=15.0):
+    from threadpoolctl import threadpool_limits
+
+    units = host_units_sample(wl, inp, 2)
+    with threadpool_limits(1):
+        done, secs = oracle_step_units(wl, units, k, alpha, budget_s)
+    return {"value": done / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"float64 numpy oracle, 1 thread: {done} unit-steps (append + scores + top-k + "
+                      f"entmax attention) cycling over units 0-1 of {wl.name}, {secs:.1f} s"}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs, scaled_down
+
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    k = args.k or wl.topk
+    # inputs are drawn on the host here (the reference arm needs no GPU); the
+    # sampled units all live in sequence 0, so one sequence of the shape is drawn
+    inp = make_inputs(scaled_down(args.workload, batch=1), seed=3000, device="cpu")
+    units = host_units_sample(wl, inp, 2)
+    from threadpoolctl import threadpool_limits
+
+    # each step is a bounded sample of the workload: one unit-step of the
+    # oracle (append, scores, top-k, entmax attention), cycling over the units
+    import oracle as O  # noqa: F401  (the reference arm runs the oracle)
+
+    done, secs = 0, 0.0
+    with threadpool_limits(1):
+        for i in range(args.warmup + args.steps):
+            unit = [units[i % len(units)]]
+            d, s_ = oracle_step_units(wl, unit, k, args.alpha, 0.0)
+            if i >= args.warmup:
+                done += d
+                secs += s_
+    value = done / secs
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, done) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: batch {wl.batch}, {wl.num_q_heads} q / {wl.num_kv_heads} KV heads, "
+                               f"d {wl.head_dim}, context {wl.context}, page size {wl.page_size}",
+                   "policy": "topk", "k": k, "alpha": args.alpha, "global_batch": wl.batch,
+                   "seq_len": wl.context, "parallelism": "none (host oracle)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"float64 numpy oracle, 1 thread, one unit-step per step cycling "
+                                   f"over units 0-1 of {wl.name}: {done} unit-steps in {secs:.1f} s"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="clustered_128k")
+    p.add_argument("--alpha", type=float, default=1.5)
+    p.add_argument("--k", type=int, default=0)
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--quick", action="store_true", help="top-k step only (no other policies, e2e or CPU leg)")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+/*
+ * ekv.h — C ABI of the EntmaxKV support-aware paged α-entmax decode library
+ * (libekv.so, hand-written CUDA for sm_100a).
+ *
+ * Source of the method: "Résumé Technique : EntmaxKV – Décodage Conscient du
+ * Support pour l'Attention Entmax" (gist.science/fr/paper/2605.21649), cited
+ * below as [EntmaxKV] with the section that defines each operation.  The page
+ * states the problem (a paged KV cache, a decode query, per-page metadata, a
+ * top-k budget k or a margin Δ, α) and prints no formula and no API; the
+ * formulas used are stated beside each call.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Ownership   The caller owns every buffer.  All pointers named "device" point
+ *             to CUDA device memory; the library never allocates and keeps no
+ *             state between calls except the sticky device error word read by
+ *             ekv_get_error().
+ * Streams     `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *             default stream).  Every call only enqueues work on it and never
+ *             synchronises, except ekv_get_error().
+ * Errors      Host-side validation runs before any launch and returns
+ *             EKV_ERR_INVALID_ARG / EKV_ERR_UNSUPPORTED / EKV_ERR_WORKSPACE
+ *             without touching the device.  A failed launch returns
+ *             EKV_ERR_CUDA.  Data-dependent faults found on the device (a page
+ *             id outside the pool, a sequence length outside 1..max_pages·S, a
+ *             Gaussian selection larger than `cap`) never trap: the kernel skips
+ *             the access, clamps, and ORs a bit into the device error word.
+ * Dtypes      EKV_BF16 or EKV_F32 for the K/V pools, the metadata pools and
+ *             the query.  Scores, bounds, thresholds and outputs are fp32.
+ * Indices     Pages named in `sel` are *logical* page indices of the
+ *             sequence; page_table maps them to physical pages.
+ * Units       A unit is one (sequence b, KV head h) pair, u = b·Hkv + h.
+ *             Query head hq belongs to KV head hq / G with G = Hq / Hkv.
+ *
+ * Memory layouts (row-major, dense)
+ * ---------------------------------
+ *   k_pool, v_pool [num_phys_pages, Hkv, S, d]
+ *   box            [num_phys_pages, Hkv, 2, d]   row 0 = k_max, row 1 = k_min
+ *   mom            [num_phys_pages, Hkv, 2, d]   row 0 = mean,  row 1 = variance
+ *   page_table     [batch, max_pages] int32, seq_lens [batch] int32
+ *   q              [batch, Hq, d]
+ *   ub             [batch, Hkv, max_pages] fp32
+ *   sel            [batch, Hkv, cap] int32 (ascending), n_sel [batch, Hkv]
+ *   out            [batch, Hq, d] fp32
+ */
+#ifndef EKV_H
+#define EKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EKV_API __attribute__((visibility("default")))
+
+typedef enum {
+  EKV_OK = 0,
+  EKV_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, α ≤ 1, k < 1, ... */
+  EKV_ERR_UNSUPPORTED = 2, /* d ∉ {64,128}, S ∉ {16,32}, G ∉ {1,2,4,8,16}, β not integer */
+  EKV_ERR_WORKSPACE = 3,   /* ws too small or not 256-byte aligned */
+  EKV_ERR_CUDA = 4,        /* a kernel launch or CUDA runtime call failed */
+  EKV_ERR_TIMEOUT = 5      /* reserved: a bounded device wait gave up */
+} ekv_status;
+
+typedef enum { EKV_F32 = 0, EKV_BF16 = 1 } ekv_dtype;
+
+/* Bits of the sticky device error word (ekv_get_error). */
+#define EKV_EFLAG_BAD_PAGE 1u      /* page_table entry outside [0, num_phys_pages) */
+#define EKV_EFLAG_BAD_LEN 2u       /* seq_lens entry outside [1, max_pages·S] */
+#define EKV_EFLAG_SEL_OVERFLOW 4u  /* Gaussian policy kept more than cap pages */
+#define EKV_EFLAG_BAD_SEL 8u       /* sel entry outside [0, pages of the sequence) */
+
+/* The paged KV cache and its per-page metadata pools (all device memory). */
+typedef struct {
+  int32_t dtype;          /* ekv_dtype of k_pool, v_pool, box, mom and q */
+  int32_t head_dim;       /* d ∈ {64, 128} */
+  int32_t page_size;      /* S ∈ {16, 32} tokens per page */
+  int32_t num_kv_heads;   /* Hkv ≥ 1 */
+  int32_t num_phys_pages; /* pages in each pool */
+  void* k_pool;
+  void* v_pool;
+  void* box;
+  void* mom;
+} ekv_cache;
+
+/* The batch of sequences: page tables and lengths (device memory). */
+typedef struct {
+  const int32_t* page_table; /* [batch, max_pages] physical page of each logical page */
+  const int32_t* seq_lens;   /* [batch] tokens, including the one being decoded */
+  int32_t batch;
+  int32_t max_pages;
+} ekv_seqs;
+
+/*
+ * ekv_build_page_meta — [EntmaxKV] §2.A, "Bornes de Boîte Englobante" and
+ * "Statistiques Gaussiennes".  For every page p < ⌈L_b/S⌉ of every sequence
+ * and every KV head, over the n_p = min(S, L_b − p·S) valid tokens, writes
+ *   box: k_max_j, k_min_j (exact);
+ *   mom: μ_j = (1/n_p)Σ_t k_tj and the population variance
+ *        σ²_j = (1/n_p)Σ_t (k_tj − μ_j)²,
+ * both accumulated in float64 in token order and rounded once (nearest-even)
+ * to the cache dtype.  Used after prefill; reads all of K.
+ */
+EKV_API ekv_status ekv_build_page_meta(const ekv_cache* cache, const ekv_seqs* seqs, void* stream);
+
+/*
+ * ekv_append — the cache append of a decode step, fused with the metadata
+ * update of [EntmaxKV] §2.A.  k_new, v_new: device [batch, Hkv, d] in the cache
+ * dtype.  Writes token L_b − 1 of every sequence (seq_lens already counts it)
+ * into its page, then recomputes box/mom of that page over its valid tokens
+ * exactly as ekv_build_page_meta does.
+ */
+EKV_API ekv_status ekv_append(const ekv_cache* cache, const ekv_seqs* seqs, const void* k_new,
+                              const void* v_new, void* stream);
+
+/*
+ * ekv_score_pages — [EntmaxKV] §2.A, the bounding-box upper bound.  For query
+ * head h and page p: ub_{p,h} = scale·Σ_j max(q_hj·kmin_pj, q_hj·kmax_pj),
+ * an upper bound of every token score scale·q_h·k of the page.  The page
+ * score of a KV head is the max over the G query heads of its group:
+ * ub[b, kvh, p] for p < ⌈L_b/S⌉ (entries past that are not written).
+ * q: device [batch, Hq, d]; ub: device fp32 [batch, Hkv, max_pages].
+ */
+EKV_API ekv_status ekv_score_pages(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                   int32_t num_q_heads, float scale, float* ub, void* stream);
+
+/*
+ * ekv_select_topk — [EntmaxKV] §2.B.1, "Sélection de Pages Top-k": per unit,
+ * the k pages with the largest ub (ties to the lower logical index; all pages
+ * when ⌈L_b/S⌉ ≤ k), written ascending to sel[b, kvh, 0..n_sel) with
+ * n_sel = min(k, ⌈L_b/S⌉).  page_size S turns seq_lens into page counts.
+ * ub: device [batch, Hkv, max_pages] (ekv_score_pages); sel: device
+ * [batch, Hkv, k]; n_sel: [batch, Hkv].
+ */
+EKV_API ekv_status ekv_select_topk(const ekv_seqs* seqs, int32_t num_kv_heads, int32_t page_size,
+                                   const float* ub, int32_t k, int32_t* sel, int32_t* n_sel,
+                                   void* stream);
+
+/*
+ * ekv_select_gauss — [EntmaxKV] §2.A "Statistiques Gaussiennes" + §2.B.2,
+ * "Sélection Entmax Consciente de Gaussienne".  Per query head h: token scores
+ * of page p are modelled as N(m, s²) with m = scale·q_h·μ_p and
+ * s² = scale²·Σ_j q_hj² σ²_pj.  τ̂_h solves Σ_p n_p·E[(u − τ̂)_+^β] = 1 with
+ * u ~ N((α−1)m, (α−1)²s²), β = 1/(α−1) ∈ {1,2,3,4} (else EKV_ERR_UNSUPPORTED).
+ * Page p is kept when (α−1)·(m + s·√(2 ln n_p)) > τ̂_h − Δ for any head of the
+ * group; if none is, the single page with the largest margin.  sel (ascending)
+ * holds at most cap pages: a larger selection keeps its first cap pages and
+ * sets EKV_EFLAG_SEL_OVERFLOW.  tau_hat: device fp32 [batch, Hq] (nullable).
+ * ws: device scratch of ekv_workspace_bytes(EKV_OP_SELECT_GAUSS, ...) bytes.
+ */
+EKV_API ekv_status ekv_select_gauss(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                    int32_t num_q_heads, float scale, float alpha, float delta,
+                                    int32_t cap, int32_t* sel, int32_t* n_sel, float* tau_hat,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ekv_entmax_decode — [EntmaxKV] §2.C, "Attention Entmax Parcimonieuse".  Over
+ * the valid tokens T of the selected pages (sel == NULL: every page of the
+ * sequence, the full-cache decode), for every query head of the unit:
+ *   z_i = scale·q·k_i,  u_i = (α−1)·z_i,
+ *   τ solves Σ_{i∈T} [u_i − τ]_+^{1/(α−1)} = 1,  p_i = [u_i − τ]_+^{1/(α−1)},
+ *   out = Σ_i p_i·v_i,
+ * reading V only for pages that hold a token with p_i > 0 for some head of
+ * the group (dense_v ≠ 0 reads every selected V page instead).
+ * sel: device [batch, Hkv, cap] with n_sel entries per unit (ascending), or
+ * NULL with n_sel NULL; cap bounds n_sel (max_pages when sel is NULL).
+ * Outputs (device): out fp32 [batch, Hq, d]; nullable tau [batch, Hq],
+ * support_count [batch, Hq] int32, support_bits uint32
+ * [batch, Hq, ⌈cap·S/32⌉] (bit i of a row: token i of the selected-token list,
+ * page-major, is in the support).
+ * ws: ekv_workspace_bytes(EKV_OP_ENTMAX_DECODE, ...) bytes.
+ */
+EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                     int32_t num_q_heads, float scale, float alpha,
+                                     const int32_t* sel, const int32_t* n_sel, int32_t cap,
+                                     int32_t dense_v, float* out, float* tau,
+                                     int32_t* support_count, uint32_t* support_bits, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Selection policies of a whole decode step. */
+typedef enum { EKV_POLICY_TOPK = 0, EKV_POLICY_GAUSS = 1, EKV_POLICY_FULL = 2 } ekv_policy;
+
+typedef struct {
+  int32_t policy;  /* ekv_policy */
+  int32_t k;       /* top-k budget (EKV_POLICY_TOPK) */
+  float delta;     /* margin Δ (EKV_POLICY_GAUSS) */
+  int32_t cap;     /* pages a unit may select: k for top-k, ≤ max_pages otherwise */
+  float alpha;     /* α > 1 */
+  float scale;     /* score scale, usually 1/√d */
+  int32_t dense_v; /* 1: read V of every selected page */
+  int32_t append;  /* 1: run ekv_append(k_new, v_new) first */
+} ekv_step_params;
+
+/*
+ * ekv_decode_step — one whole decode step of [EntmaxKV] §2 in stream order:
+ * append (if params->append) → page scores + top-k, or the Gaussian policy,
+ * or every page → sparse α-entmax attention.  sel / n_sel receive the
+ * selection (device [batch, Hkv, cap] / [batch, Hkv]); out [batch, Hq, d].
+ * tau (nullable) receives [batch, Hq] thresholds.  ws: ekv_workspace_bytes(
+ * EKV_OP_DECODE_STEP, ...) bytes.
+ */
+EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
+                                   const ekv_step_params* params, const void* q,
+                                   int32_t num_q_heads, const void* k_new, const void* v_new,
+                                   int32_t* sel, int32_t* n_sel, float* out, float* tau, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+typedef enum {
+  EKV_OP_SELECT_GAUSS = 1,
+  EKV_OP_ENTMAX_DECODE = 2,
+  EKV_OP_DECODE_STEP = 3
+} ekv_op;
+
+/*
+ * ekv_workspace_bytes — device scratch an op needs, from the host-side sizes
+ * only (cache dims, batch, max_pages, Hq, cap; for EKV_OP_DECODE_STEP `cap` is
+ * params->cap).  Returns 0 when the sizes are invalid.
+ */
+EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv_seqs* seqs,
+                                   int32_t num_q_heads, int32_t cap);
+
+/* Reads the sticky device error word into *flags (EKV_EFLAG_* bits) and clears
+ * it.  Synchronises the device. */
+EKV_API ekv_status ekv_get_error(uint32_t* flags);
+
+/* Static description of a status code. */
+EKV_API const char* ekv_status_string(ekv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EKV_H */

@@ -1,0 +1,221 @@
+// Gaussian-aware entmax page selection — EntmaxKV summary page
+// (gist.science/fr/paper/2605.21649) §2.B, "Sélection Entmax Consciente de
+// Gaussienne": estimate the global α-entmax threshold τ̂ from per-page
+// Gaussian score statistics, then keep the pages whose estimated maximum
+// score clears τ̂ − Δ.
+//
+// τ̂ solves F(τ) = Σ_p n_p·E[(u_p − τ)_+^β] = 1 for u_p ~ N(μ_p, σ_p²) (in
+// threshold units u = (α−1)·score, β = 1/(α−1) an integer).  With
+// c = (τ − μ)/σ and J_k(c) = ∫_c^∞ (x − c)^k φ(x) dx,
+//   E[(u − τ)_+^β] = σ^β J_β(c),   dE/dτ = −β σ^(β−1) J_(β−1)(c),
+//   J_0 = Q(c),  J_1 = φ(c) − c·Q(c),  J_k = (k−1)·J_(k−2) − c·J_(k−1)
+// (integration by parts with xφ = −φ').  F is convex and decreasing, so
+// Newton's method started left of the root (Jensen's bound
+// τ_lo = max_p μ_p − n_p^(−1/β), where F ≥ 1) climbs monotonically to it and
+// never overshoots.  Pages with c > kPruneC at τ_lo contribute below
+// n·σ^β·J_β(kPruneC) and stay negligible for every later τ (c only grows), so
+// only the survivors are iterated, from shared memory.
+#include "kernels.cuh"
+
+namespace ekv {
+
+namespace {
+
+constexpr int kGaussThreads = 256;
+constexpr int kGaussCand = 3072;
+constexpr float kPruneC = 7.0f;
+
+__device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double tau, int beta,
+                                            double& F, double& dF) {
+  if (!(mu > -INFINITY)) return;
+  if (sg <= 0.f) {
+    const double w = static_cast<double>(mu) - tau;
+    if (w > 0.0) {
+      double wb1 = 1.0;
+      for (int k = 1; k < beta; ++k) wb1 *= w;
+      F += n * wb1 * w;
+      dF += n * beta * wb1;
+    }
+    return;
+  }
+  const float c = static_cast<float>((tau - static_cast<double>(mu)) / static_cast<double>(sg));
+  if (c > kPruneC) return;
+  const float Q = 0.5f * erfcf(c * 0.70710678118654752f);
+  const float phi = 0.39894228040143268f * expf(-0.5f * c * c);
+  float jm2 = Q, jm1 = phi - c * Q;  // J_0, J_1
+  float jb = jm1, jb1 = jm2;         // J_β, J_(β−1) for β = 1
+  for (int k = 2; k <= beta; ++k) {
+    const float jk = static_cast<float>(k - 1) * jm2 - c * jm1;
+    jb1 = jm1;
+    jb = jk;
+    jm2 = jm1;
+    jm1 = jk;
+  }
+  double sb1 = 1.0;
+  for (int k = 1; k < beta; ++k) sb1 *= sg;
+  F += static_cast<double>(n) * sb1 * sg * fmaxf(jb, 0.f);
+  dF += static_cast<double>(n) * beta * sb1 * fmaxf(jb1, 0.f);
+}
+
+__global__ void __launch_bounds__(kGaussThreads)
+    gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
+                     int Hkv, int G, int Hq, int chunks, int beta, float* __restrict__ tau_out) {
+  const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / Hkv, kvh = unit % Hkv;
+  const int tid = threadIdx.x;
+  int L;
+  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
+  __shared__ float c_mu[kGaussCand], c_sg[kGaussCand], c_n[kGaussCand];
+  __shared__ int s_count;
+  __shared__ float f_scratch[32];
+  __shared__ double d_scratch[32];
+
+  const int nch = (P + kStreamPagesPerCta - 1) / kStreamPagesPerCta;
+  float lo = -INFINITY;
+  for (int c = tid; c < nch; c += blockDim.x) lo = fmaxf(lo, ws.lo[static_cast<size_t>(row) * chunks + c]);
+  lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+  const size_t base = static_cast<size_t>(row) * max_pages;
+  if (P == 0 || !(lo > -INFINITY)) {
+    if (tid == 0) {
+      ws.tau_hat[row] = static_cast<double>(INFINITY);
+      if (tau_out) tau_out[static_cast<size_t>(b) * Hq + kvh * G + g] = INFINITY;
+    }
+    return;
+  }
+
+  if (tid == 0) s_count = 0;
+  __syncthreads();
+  for (int p = tid; p < P; p += blockDim.x) {
+    const float mu = ws.mu[base + p], sg = ws.sig[base + p];
+    if (mu > -INFINITY && mu + kPruneC * sg > lo) {
+      const int slot = atomicAdd(&s_count, 1);
+      if (slot < kGaussCand) {
+        c_mu[slot] = mu;
+        c_sg[slot] = sg;
+        c_n[slot] = static_cast<float>(min(S, L - p * S));
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = s_count;
+  const bool cached = nc <= kGaussCand;
+
+  double tau = static_cast<double>(lo);
+  for (int it = 0; it < 100; ++it) {
+    double F = 0.0, dF = 0.0;
+    if (cached) {
+      for (int i = tid; i < nc; i += blockDim.x) gauss_terms(c_mu[i], c_sg[i], c_n[i], tau, beta, F, dF);
+    } else {
+      for (int p = tid; p < P; p += blockDim.x)
+        gauss_terms(ws.mu[base + p], ws.sig[base + p], static_cast<float>(min(S, L - p * S)), tau,
+                    beta, F, dF);
+    }
+    F = block_reduce(F, d_scratch, [](double x, double y) { return x + y; });
+    dF = block_reduce(dF, d_scratch, [](double x, double y) { return x + y; });
+    const double step = (F - 1.0) / dF;
+    if (!(step > 0.0)) break;
+    tau += step;
+    if (step <= 1e-12 * fmax(1.0, fabs(tau))) break;
+  }
+  if (tid == 0) {
+    ws.tau_hat[row] = tau;
+    if (tau_out) tau_out[static_cast<size_t>(b) * Hq + kvh * G + g] = static_cast<float>(tau);
+  }
+}
+
+// Keep page p when (α−1)·ŝ_{p,h} > τ̂_h − Δ for some query head h of the unit;
+// compaction in ascending page order; fallback to the largest margin.
+__global__ void __launch_bounds__(kGaussThreads)
+    gauss_filter_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
+                        int Hkv, int G, double delta, int cap, int32_t* __restrict__ sel,
+                        int32_t* __restrict__ n_sel) {
+  const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
+  int L;
+  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
+  __shared__ double s_thr[16];
+  __shared__ int scan_scratch[32];
+  __shared__ double best_m[32];
+  __shared__ int best_i[32];
+  if (tid < G) s_thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
+  __syncthreads();
+  int32_t* out = sel + static_cast<size_t>(unit) * cap;
+  int carry = 0;
+  double my_best = -INFINITY;
+  int my_idx = 0x7fffffff;
+  for (int base = 0; base < P; base += blockDim.x) {
+    const int p = base + tid;
+    int keep = 0;
+    if (p < P) {
+      double mg = -INFINITY;
+      for (int g = 0; g < G; ++g) {
+        const double m = static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - s_thr[g];
+        mg = fmax(mg, m);
+      }
+      keep = mg > 0.0 ? 1 : 0;
+      if (mg > my_best) {
+        my_best = mg;
+        my_idx = p;
+      }
+    }
+    int total;
+    const int pos = block_exclusive_scan(keep, scan_scratch, &total) + carry;
+    if (keep && pos < cap) out[pos] = p;
+    carry += total;
+  }
+  if (carry > 0) {
+    if (tid == 0) {
+      n_sel[unit] = min(carry, cap);
+      if (carry > cap) raise_flag(EKV_EFLAG_SEL_OVERFLOW);
+    }
+    return;
+  }
+  // fallback: the single page with the largest margin, lowest index on ties
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int o = 16; o > 0; o >>= 1) {
+    const double om = __shfl_xor_sync(0xffffffffu, my_best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, my_idx, o);
+    if (om > my_best || (om == my_best && oi < my_idx)) {
+      my_best = om;
+      my_idx = oi;
+    }
+  }
+  if (lane == 0) {
+    best_m[warp] = my_best;
+    best_i[warp] = my_idx;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double bm = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+      if (best_m[w] > bm || (best_m[w] == bm && best_i[w] < bi)) {
+        bm = best_m[w];
+        bi = best_i[w];
+      }
+    }
+    if (P > 0 && bi < P) {
+      out[0] = bi;
+      n_sel[unit] = 1;
+    } else {
+      n_sel[unit] = 0;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, float alpha,
+                                float delta, int cap, const GaussWs& ws, int32_t* sel,
+                                int32_t* n_sel, float* tau_hat, cudaStream_t st) {
+  const int Hkv = c.num_kv_heads, G = Hq / Hkv, U = s.batch * Hkv;
+  const int beta = static_cast<int>(lrint(1.0 / (static_cast<double>(alpha) - 1.0)));
+  gauss_tau_kernel<<<U * G, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
+                                                    G, Hq, stream_chunks(s.max_pages), beta,
+                                                    tau_hat);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gauss_filter_kernel<<<U, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
+                                                   G, static_cast<double>(delta), cap, sel, n_sel);
+  return cudaGetLastError();
+}
+
+}  // namespace ekv

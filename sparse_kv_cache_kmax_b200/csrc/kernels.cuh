@@ -1,0 +1,59 @@
+// Launchers of libekv's kernels (internal to the library; the public C ABI is
+// include/ekv.h, implemented in api.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace ekv {
+
+// Pages handled by one CTA of the metadata-streaming kernels.
+constexpr int kStreamPagesPerCta = 64;
+// CTAs the split-over-pages decode kernels aim for (two per SM of a B200).
+constexpr int kDecodeTargetCtas = 296;
+
+struct DecodeWs {
+  float* zbuf;      // [U, G, cap·S] scores z of the selected tokens (−inf: no token)
+  float* pmax;      // [U, G, cap]   page maxima of z
+  float* cmax;      // [U, G, nsplit] split maxima of z
+  float* taus;      // [U, G]        thresholds τ (fp32)
+  float* part;      // [U, nsplit, G, d] partial outputs of the V pass
+  int* counter;     // [U]           finished V-pass splits
+};
+
+struct GaussWs {
+  float* mu;        // [U, G, max_pages] (α−1)·m
+  float* sig;       // [U, G, max_pages] (α−1)·s
+  float* hat;       // [U, G, max_pages] (α−1)·ŝ
+  float* lo;        // [U, G, chunks]    per-CTA lower brackets of τ̂
+  double* tau_hat;  // [U, G]
+};
+
+cudaError_t launch_build_meta(const ekv_cache& c, const ekv_seqs& s, cudaStream_t st);
+cudaError_t launch_append(const ekv_cache& c, const ekv_seqs& s, const void* k_new,
+                          const void* v_new, cudaStream_t st);
+cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq, float scale,
+                         float* ub, cudaStream_t st);
+cudaError_t launch_gauss_stats(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
+                               float scale, float alpha, const GaussWs& ws, cudaStream_t st);
+cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
+                        int32_t* sel, int32_t* n_sel, cudaStream_t st);
+cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, float alpha,
+                                float delta, int cap, const GaussWs& ws, int32_t* sel,
+                                int32_t* n_sel, float* tau_hat, cudaStream_t st);
+cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
+                          float scale, float alpha, const int32_t* sel, const int32_t* n_sel,
+                          int cap, int dense_v, float* out, float* tau, int32_t* support_count,
+                          uint32_t* support_bits, const DecodeWs& ws, int nsplit, cudaStream_t st);
+
+inline int stream_chunks(int max_pages) {
+  return (max_pages + kStreamPagesPerCta - 1) / kStreamPagesPerCta;
+}
+inline int decode_splits(int units, int cap) {
+  int ns = (kDecodeTargetCtas + units - 1) / units;
+  if (ns > cap) ns = cap;
+  if (ns < 1) ns = 1;
+  const int per = (cap + ns - 1) / ns;
+  return (cap + per - 1) / per;
+}
+
+}  // namespace ekv
