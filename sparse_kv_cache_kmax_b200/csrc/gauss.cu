@@ -14,7 +14,10 @@
 // τ_lo = max_p μ_p − n_p^(−1/β), where F ≥ 1) climbs monotonically to it and
 // never overshoots.  Pages with c > kPruneC at τ_lo contribute below
 // n·σ^β·J_β(kPruneC) and stay negligible for every later τ (c only grows), so
-// only the survivors are iterated, from shared memory.
+// only the survivors are iterated, from shared memory.  The recurrence
+// amplifies the rounding of Q and φ by about c^(2β)/β! for c > 0, so the fp32
+// iterations only approach the root; two final Newton steps evaluate every
+// term in float64.
 #include "kernels.cuh"
 
 namespace ekv {
@@ -25,6 +28,22 @@ constexpr int kGaussThreads = 256;
 constexpr int kGaussCand = 3072;
 constexpr float kPruneC = 7.0f;
 
+template <typename R>
+__device__ __forceinline__ void normal_tail(R c, R& Q, R& phi);
+template <>
+__device__ __forceinline__ void normal_tail<float>(float c, float& Q, float& phi) {
+  Q = 0.5f * erfcf(c * 0.70710678118654752f);
+  phi = 0.39894228040143268f * expf(-0.5f * c * c);
+}
+template <>
+__device__ __forceinline__ void normal_tail<double>(double c, double& Q, double& phi) {
+  Q = 0.5 * erfc(c * 0.70710678118654752);
+  phi = 0.39894228040143268 * exp(-0.5 * c * c);
+}
+
+// Adds page (μ, σ, n)'s n·E[(u−τ)_+^β] to F and n·β·E[(u−τ)_+^(β−1)] to dF,
+// evaluating the tail functions in precision R.
+template <typename R>
 __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double tau, int beta,
                                             double& F, double& dF) {
   if (!(mu > -INFINITY)) return;
@@ -38,14 +57,14 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
     }
     return;
   }
-  const float c = static_cast<float>((tau - static_cast<double>(mu)) / static_cast<double>(sg));
-  if (c > kPruneC) return;
-  const float Q = 0.5f * erfcf(c * 0.70710678118654752f);
-  const float phi = 0.39894228040143268f * expf(-0.5f * c * c);
-  float jm2 = Q, jm1 = phi - c * Q;  // J_0, J_1
-  float jb = jm1, jb1 = jm2;         // J_β, J_(β−1) for β = 1
+  const R c = static_cast<R>((tau - static_cast<double>(mu)) / static_cast<double>(sg));
+  if (c > static_cast<R>(kPruneC)) return;
+  R Q, phi;
+  normal_tail<R>(c, Q, phi);
+  R jm2 = Q, jm1 = phi - c * Q;  // J_0, J_1
+  R jb = jm1, jb1 = jm2;         // J_β, J_(β−1) for β = 1
   for (int k = 2; k <= beta; ++k) {
-    const float jk = static_cast<float>(k - 1) * jm2 - c * jm1;
+    const R jk = static_cast<R>(k - 1) * jm2 - c * jm1;
     jb1 = jm1;
     jb = jk;
     jm2 = jm1;
@@ -53,8 +72,8 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
   }
   double sb1 = 1.0;
   for (int k = 1; k < beta; ++k) sb1 *= sg;
-  F += static_cast<double>(n) * sb1 * sg * fmaxf(jb, 0.f);
-  dF += static_cast<double>(n) * beta * sb1 * fmaxf(jb1, 0.f);
+  F += static_cast<double>(n) * sb1 * sg * static_cast<double>(jb > R(0) ? jb : R(0));
+  dF += static_cast<double>(n) * beta * sb1 * static_cast<double>(jb1 > R(0) ? jb1 : R(0));
 }
 
 __global__ void __launch_bounds__(kGaussThreads)
@@ -99,22 +118,42 @@ __global__ void __launch_bounds__(kGaussThreads)
   const int nc = s_count;
   const bool cached = nc <= kGaussCand;
 
-  double tau = static_cast<double>(lo);
-  for (int it = 0; it < 100; ++it) {
-    double F = 0.0, dF = 0.0;
+  auto evaluate = [&](double t, bool exact, double& F, double& dF) {
+    F = 0.0;
+    dF = 0.0;
     if (cached) {
-      for (int i = tid; i < nc; i += blockDim.x) gauss_terms(c_mu[i], c_sg[i], c_n[i], tau, beta, F, dF);
+      for (int i = tid; i < nc; i += blockDim.x) {
+        if (exact)
+          gauss_terms<double>(c_mu[i], c_sg[i], c_n[i], t, beta, F, dF);
+        else
+          gauss_terms<float>(c_mu[i], c_sg[i], c_n[i], t, beta, F, dF);
+      }
     } else {
-      for (int p = tid; p < P; p += blockDim.x)
-        gauss_terms(ws.mu[base + p], ws.sig[base + p], static_cast<float>(min(S, L - p * S)), tau,
-                    beta, F, dF);
+      for (int p = tid; p < P; p += blockDim.x) {
+        const float n = static_cast<float>(min(S, L - p * S));
+        if (exact)
+          gauss_terms<double>(ws.mu[base + p], ws.sig[base + p], n, t, beta, F, dF);
+        else
+          gauss_terms<float>(ws.mu[base + p], ws.sig[base + p], n, t, beta, F, dF);
+      }
     }
     F = block_reduce(F, d_scratch, [](double x, double y) { return x + y; });
     dF = block_reduce(dF, d_scratch, [](double x, double y) { return x + y; });
+  };
+  double tau = static_cast<double>(lo);
+  for (int it = 0; it < 100; ++it) {  // fp32 terms: monotone approach from the left
+    double F, dF;
+    evaluate(tau, false, F, dF);
     const double step = (F - 1.0) / dF;
     if (!(step > 0.0)) break;
     tau += step;
-    if (step <= 1e-12 * fmax(1.0, fabs(tau))) break;
+    if (step <= 1e-7 * fmax(1.0, fabs(tau))) break;
+  }
+  for (int it = 0; it < 2; ++it) {    // float64 terms: quadratic polish (either side)
+    double F, dF;
+    evaluate(tau, true, F, dF);
+    if (!(dF > 0.0)) break;
+    tau += (F - 1.0) / dF;
   }
   if (tid == 0) {
     ws.tau_hat[row] = tau;
