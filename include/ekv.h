@@ -179,6 +179,33 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
                                      int32_t* support_count, uint32_t* support_bits, void* ws,
                                      size_t ws_bytes, void* stream);
 
+/* Bytes of the library-owned scratch array of ekv_entmax_decode_static_ws. */
+#define EKV_STATIC_WS_BYTES (16u << 20)
+
+/*
+ * ekv_entmax_decode_static_ws — ekv_entmax_decode without a caller workspace.
+ * The source page has no counterpart to this call: it exists for callers
+ * that cannot allocate device memory, such as a plugin inside a framework
+ * that owns the device memory pool and offers no scratch buffer, or a serving
+ * loop that must not call cudaMalloc once running.  Arguments and outputs are
+ * those of ekv_entmax_decode; the scratch comes from one static device array
+ * of EKV_STATIC_WS_BYTES bytes that every GPU loading the library holds until
+ * the process exits.  A configuration whose scratch
+ * (ekv_workspace_bytes(EKV_OP_ENTMAX_DECODE, ...)) exceeds that size returns
+ * EKV_ERR_WORKSPACE before any device work.  All calls on a device share the
+ * array: calls that overlap on the GPU race, so serialise them.  The array
+ * keeps the previous call's contents; the only part that must start at zero
+ * (the split counters) is reset by the call itself.  The first call on a
+ * device looks up the array's device address, so make it before any stream
+ * capture.  Allocates nothing.
+ */
+EKV_API ekv_status ekv_entmax_decode_static_ws(const ekv_cache* cache, const ekv_seqs* seqs,
+                                               const void* q, int32_t num_q_heads, float scale,
+                                               float alpha, const int32_t* sel,
+                                               const int32_t* n_sel, int32_t cap, int32_t dense_v,
+                                               float* out, float* tau, int32_t* support_count,
+                                               uint32_t* support_bits, void* stream);
+
 /* Selection policies of a whole decode step. */
 typedef enum { EKV_POLICY_TOPK = 0, EKV_POLICY_GAUSS = 1, EKV_POLICY_FULL = 2 } ekv_policy;
 
