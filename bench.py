@@ -5,7 +5,7 @@
 One step = one decode token for every (sequence, KV head) unit of the
 workload: cache append + tail-page metadata, bounding-box page scores, top-k
 page selection, sparse α-entmax attention (scores over the selected K, τ,
-support-only V).  Inputs are resident in HBM; L2 is flushed (256 MiB write)
+support-only V).  Inputs are resident in HBM; L2 is flushed (256 MiB read)
 between steps.  Prints one JSON line on rank 0.
 
 Workload (default): the clustered 128k-context decode — batch 4, 32 query /
@@ -14,6 +14,7 @@ Workload (default): the clustered 128k-context decode — batch 4, 32 query /
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -137,6 +138,18 @@ class ClockSampler:
                 "samples": len(mhz)}
 
 
+class L2Flush:
+    """Evicts the 126 MB L2 between timed steps by reading a 256 MiB buffer
+    (a read leaves clean lines, so the next step pays no write-back)."""
+
+    def __init__(self, dev):
+        self.buf = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def zero_(self):
+        torch.sum(self.buf, dim=0, out=self.sink)
+
+
 # ---------------------------------------------------------------- bytes
 def algorithmic_bytes(inp, eng, support_pages):
     """Bytes one step must move: metadata rows, q, ub, selected K, V of
@@ -189,7 +202,7 @@ def run_ours(args):
     scale = float(np.float32(wl.scale))
     ub = torch.empty(wl.batch, wl.num_kv_heads, inp["max_pages"], device=dev)
     dec_ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, cache, seqs, Hq, k), dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def stage_step(ev):
@@ -261,7 +274,7 @@ def run_ours(args):
                                f"d {wl.head_dim}, context {wl.context}, page size {wl.page_size}",
                    "policy": "topk", "k": k, "alpha": alpha, "global_batch": wl.batch * world,
                    "seq_len": wl.context, "parallelism": f"replicas x{world} (units sharded, no collective)",
-                   "l2": "flushed between steps (256 MiB write)"},
+                   "l2": "flushed between steps (256 MiB read)"},
         "steps_per_s": 1e3 / step_ms,
         "stages_us": {"append": stages[0] * 1e3, "score": stages[1] * 1e3, "topk": stages[2] * 1e3,
                       "decode": stages[3] * 1e3},
@@ -457,6 +470,91 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+# ---------------------------------------------------------------- kernel microbench
+def run_kernel(args):
+    """Launch one stage repeatedly on inputs of the workload's shape that only
+    hold what that stage reads (a few hundred MB): the case ncu captures."""
+    from sparse_kv_cache_kmax_b200 import binding as Bd
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    if args.shape:
+        bb, hq, hkv = (int(x) for x in args.shape.split(","))
+        wl = dataclasses.replace(wl, batch=bb, num_q_heads=hq, num_kv_heads=hkv)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(11)
+    B, Hkv, Hq, d, S = wl.batch, wl.num_kv_heads, wl.num_q_heads, wl.head_dim, wl.page_size
+    P = wl.max_pages
+    k = args.k or wl.topk
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    page_table = torch.arange(B * P, dtype=torch.int32, device=dev).view(B, P)
+    seq_lens = torch.full((B,), wl.context, dtype=torch.int32, device=dev)
+    q = torch.randn(B, Hq, d, generator=g, device=dev).to(dt)
+    scale = float(np.float32(wl.scale))
+    stream = torch.cuda.current_stream()
+    if args.kernel == "copy":
+        src = torch.empty(B * P * Hkv * 2 * d, dtype=dt, device=dev).normal_(generator=g)
+        dst = torch.empty_like(src)
+
+        def launch():
+            dst.copy_(src)
+        nbytes = 2 * src.numel() * src.element_size()
+    elif args.kernel in ("score", "gauss", "topk"):
+        kv = torch.empty(1, Hkv, S, d, dtype=dt, device=dev)          # never read by these stages
+        lo = torch.randn(B * P, Hkv, 1, d, generator=g, device=dev)
+        box = torch.cat([lo + 0.5, lo - 0.5], dim=2).to(dt).contiguous()
+        mom = torch.cat([lo, torch.rand(B * P, Hkv, 1, d, generator=g, device=dev)], dim=2).to(dt).contiguous()
+        cache = Bd.make_cache(kv, kv, box, mom)
+        cache.num_phys_pages = B * P
+        seqs = Bd.make_seqs(page_table, seq_lens)
+        ub = torch.randn(B, Hkv, P, generator=g, device=dev)
+        sel = torch.zeros(B, Hkv, max(k, P), dtype=torch.int32, device=dev)
+        n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
+        tau_hat = torch.zeros(B, Hq, device=dev)
+        gws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_GAUSS, cache, seqs, Hq, P), dev)
+
+        def launch():
+            if args.kernel == "score":
+                Bd.ekv_score_pages(cache, seqs, q, scale, ub, stream)
+            elif args.kernel == "topk":
+                Bd.ekv_select_topk(seqs, Hkv, S, ub, k, sel, n_sel, stream)
+            else:
+                Bd.ekv_select_gauss(cache, seqs, q, scale, args.alpha, wl.delta or 0.5, P, sel, n_sel, tau_hat,
+                                    gws, stream)
+        nbytes = B * P * Hkv * 2 * d * box.element_size()
+    else:  # decode: only the k selected pages of every unit exist in the pools
+        kpool = torch.randn(B * k, Hkv, S, d, generator=g, device=dev).to(dt)
+        vpool = torch.randn(B * k, Hkv, S, d, generator=g, device=dev).to(dt)
+        meta = torch.empty(1, Hkv, 2, d, dtype=dt, device=dev)
+        cache = Bd.make_cache(kpool, vpool, meta, meta)
+        pt = torch.zeros(B, P, dtype=torch.int32, device=dev)
+        pt[:, :k] = torch.arange(B * k, dtype=torch.int32, device=dev).view(B, k)
+        seqs = Bd.make_seqs(pt, seq_lens)
+        sel = torch.arange(k, dtype=torch.int32, device=dev).expand(B, Hkv, k).contiguous()
+        n_sel = torch.full((B, Hkv), k, dtype=torch.int32, device=dev)
+        out = torch.empty(B, Hq, d, device=dev)
+        ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, cache, seqs, Hq, k), dev)
+
+        def launch():
+            Bd.ekv_entmax_decode(cache, seqs, q, scale, args.alpha, sel, n_sel, k, out, ws, stream=stream)
+        nbytes = B * Hkv * k * S * d * kpool.element_size()
+    flush = L2Flush(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record()
+        launch()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in ev])) * 1e3
+    print(json.dumps({"kernel": args.kernel, "workload": wl.name, "us": us, "bytes": nbytes,
+                      "gbs": nbytes / (us * 1e-6) / 1e9}))
+
+
 def main(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -468,11 +566,17 @@ def main(argv=None):
     p.add_argument("--k", type=int, default=0)
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--quick", action="store_true", help="top-k step only (no other policies, e2e or CPU leg)")
+    p.add_argument("--kernel", choices=["score", "gauss", "topk", "decode", "copy"],
+                   help="time one stage alone on inputs holding only what it reads ('copy': a plain "
+                        "device copy of the stage's bytes, for reference)")
+    p.add_argument("--shape", default="", help="kernel mode: override 'batch,q_heads,kv_heads'")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.kernel:
+        run_kernel(args)
     else:
         run_ours(args)
 

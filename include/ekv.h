@@ -71,6 +71,7 @@ typedef enum { EKV_F32 = 0, EKV_BF16 = 1 } ekv_dtype;
 #define EKV_EFLAG_BAD_LEN 2u       /* seq_lens entry outside [1, max_pages·S] */
 #define EKV_EFLAG_SEL_OVERFLOW 4u  /* Gaussian policy kept more than cap pages */
 #define EKV_EFLAG_BAD_SEL 8u       /* sel entry outside [0, pages of the sequence) */
+#define EKV_EFLAG_TIMEOUT 16u      /* a bounded wait on an asynchronous copy gave up */
 
 /* The paged KV cache and its per-page metadata pools (all device memory). */
 typedef struct {

@@ -69,9 +69,7 @@ size_t gauss_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   const size_t G = static_cast<size_t>(Hq / c->num_kv_heads);
   const size_t rows = U * G * static_cast<size_t>(s->max_pages);
-  return 3 * a256(rows * sizeof(float)) +
-         a256(U * G * static_cast<size_t>(stream_chunks(s->max_pages)) * sizeof(float)) +
-         a256(U * G * sizeof(double));
+  return 3 * a256(rows * sizeof(float)) + a256(U * G * sizeof(double));
 }
 
 GaussWs carve_gauss(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq) {
@@ -82,7 +80,6 @@ GaussWs carve_gauss(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq) {
   w.mu = cv.take<float>(rows);
   w.sig = cv.take<float>(rows);
   w.hat = cv.take<float>(rows);
-  w.lo = cv.take<float>(U * G * static_cast<size_t>(stream_chunks(s->max_pages)));
   w.tau_hat = cv.take<double>(U * G);
   return w;
 }

@@ -78,7 +78,7 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
 
 __global__ void __launch_bounds__(kGaussThreads)
     gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
-                     int Hkv, int G, int Hq, int chunks, int beta, float* __restrict__ tau_out) {
+                     int Hkv, int G, int Hq, int beta, float* __restrict__ tau_out) {
   const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / Hkv, kvh = unit % Hkv;
   const int tid = threadIdx.x;
   int L;
@@ -88,11 +88,15 @@ __global__ void __launch_bounds__(kGaussThreads)
   __shared__ float f_scratch[32];
   __shared__ double d_scratch[32];
 
-  const int nch = (P + kStreamPagesPerCta - 1) / kStreamPagesPerCta;
-  float lo = -INFINITY;
-  for (int c = tid; c < nch; c += blockDim.x) lo = fmaxf(lo, ws.lo[static_cast<size_t>(row) * chunks + c]);
-  lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+  // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
   const size_t base = static_cast<size_t>(row) * max_pages;
+  const float inv_beta = 1.0f / static_cast<float>(beta);
+  float lo = -INFINITY;
+  for (int p = tid; p < P; p += blockDim.x) {
+    const float mu = ws.mu[base + p];
+    if (mu > -INFINITY) lo = fmaxf(lo, mu - powf(static_cast<float>(min(S, L - p * S)), -inv_beta));
+  }
+  lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
   if (P == 0 || !(lo > -INFINITY)) {
     if (tid == 0) {
       ws.tau_hat[row] = static_cast<double>(INFINITY);
@@ -248,8 +252,7 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
   const int Hkv = c.num_kv_heads, G = Hq / Hkv, U = s.batch * Hkv;
   const int beta = static_cast<int>(lrint(1.0 / (static_cast<double>(alpha) - 1.0)));
   gauss_tau_kernel<<<U * G, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
-                                                    G, Hq, stream_chunks(s.max_pages), beta,
-                                                    tau_hat);
+                                                    G, Hq, beta, tau_hat);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   gauss_filter_kernel<<<U, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,

@@ -6,8 +6,6 @@
 
 namespace ekv {
 
-// Pages handled by one CTA of the metadata-streaming kernels.
-constexpr int kStreamPagesPerCta = 64;
 // CTAs the split-over-pages decode kernels aim for (two per SM of a B200).
 constexpr int kDecodeTargetCtas = 296;
 
@@ -24,7 +22,6 @@ struct GaussWs {
   float* mu;        // [U, G, max_pages] (α−1)·m
   float* sig;       // [U, G, max_pages] (α−1)·s
   float* hat;       // [U, G, max_pages] (α−1)·ŝ
-  float* lo;        // [U, G, chunks]    per-CTA lower brackets of τ̂
   double* tau_hat;  // [U, G]
 };
 
@@ -45,9 +42,6 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
                           uint32_t* support_bits, const DecodeWs& ws, int nsplit, cudaStream_t st);
 
-inline int stream_chunks(int max_pages) {
-  return (max_pages + kStreamPagesPerCta - 1) / kStreamPagesPerCta;
-}
 inline int decode_splits(int units, int cap) {
   int ns = (kDecodeTargetCtas + units - 1) / units;
   if (ns > cap) ns = cap;
