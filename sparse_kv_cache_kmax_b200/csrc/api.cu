@@ -87,25 +87,29 @@ GaussWs carve_gauss(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq) {
 size_t decode_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   const size_t G = static_cast<size_t>(Hq / c->num_kv_heads);
-  const size_t ns = static_cast<size_t>(decode_splits(static_cast<int>(U), cap));
+  const size_t nqk = static_cast<size_t>(qk_splits(cap, c->page_size));
+  const size_t npv = static_cast<size_t>(pv_splits(static_cast<int>(U), cap));
   const size_t S = static_cast<size_t>(c->page_size), D = static_cast<size_t>(c->head_dim);
   return a256(U * G * cap * S * sizeof(float)) + a256(U * G * cap * sizeof(float)) +
-         a256(U * G * ns * sizeof(float)) + a256(U * G * sizeof(float)) +
-         a256(U * ns * G * D * sizeof(float)) + a256(U * sizeof(int));
+         a256(U * G * nqk * sizeof(float)) + a256(U * G * sizeof(float)) +
+         a256(U * npv * G * D * sizeof(float)) + a256(U * sizeof(int));
 }
 
 DecodeWs carve_decode(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   const size_t G = static_cast<size_t>(Hq / c->num_kv_heads);
-  const size_t ns = static_cast<size_t>(decode_splits(static_cast<int>(U), cap));
+  const int nqk = qk_splits(cap, c->page_size);
+  const int npv = pv_splits(static_cast<int>(U), cap);
   const size_t S = static_cast<size_t>(c->page_size), D = static_cast<size_t>(c->head_dim);
   DecodeWs w;
   w.zbuf = cv.take<float>(U * G * cap * S);
   w.pmax = cv.take<float>(U * G * cap);
-  w.cmax = cv.take<float>(U * G * ns);
+  w.cmax = cv.take<float>(U * G * static_cast<size_t>(nqk));
   w.taus = cv.take<float>(U * G);
-  w.part = cv.take<float>(U * ns * G * D);
+  w.part = cv.take<float>(U * static_cast<size_t>(npv) * G * D);
   w.counter = cv.take<int>(U);
+  w.nqk = nqk;
+  w.npv = npv;
   return w;
 }
 
@@ -217,10 +221,9 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
   EKV_TRY(check_ws(ws, ws_bytes, decode_ws_bytes(cache, seqs, num_q_heads, cap)));
   Carver cv{static_cast<char*>(ws)};
   const DecodeWs dw = carve_decode(cv, cache, seqs, num_q_heads, cap);
-  const int U = seqs->batch * cache->num_kv_heads;
   return cuda_status(launch_decode(*cache, *seqs, q, num_q_heads, scale, alpha, sel, n_sel, cap,
                                    dense_v, out, tau, support_count, support_bits, dw,
-                                   decode_splits(U, cap), static_cast<cudaStream_t>(stream)));
+                                   static_cast<cudaStream_t>(stream)));
 }
 
 EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
@@ -269,8 +272,7 @@ EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
     use_n = nullptr;
   }
   return cuda_status(launch_decode(*cache, *seqs, q, num_q_heads, p->scale, p->alpha, use_sel,
-                                   use_n, cap, p->dense_v, out, tau, nullptr, nullptr, dw,
-                                   decode_splits(static_cast<int>(U), cap), st));
+                                   use_n, cap, p->dense_v, out, tau, nullptr, nullptr, dw, st));
 }
 
 EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv_seqs* seqs,

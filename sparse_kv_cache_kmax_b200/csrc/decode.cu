@@ -4,18 +4,25 @@
 // tokens contain the α-entmax support, the output equals the full-cache one.
 //
 // Three kernels, all on the caller's stream:
-//  1. qk: split over selected pages.  K pages are staged in shared memory
-//     (16 B vector loads, padded rows), the G query heads of the unit share
-//     each tile, and z = scale·q·k lands in an L2-resident scratch together
-//     with per-page and per-split maxima.
-//  2. tau: one CTA per query head solves Σ_i [u_i − τ]_+^β = 1, u = (α−1)·z,
-//     by Newton's method from τ₀ = max(u) − 1 (the function is convex and
-//     decreasing, so iterates rise monotonically to the root), then for
-//     β ∈ {1, 2} re-solves in closed form on the support it found.
-//  3. pv: split over selected pages again; a page's V is read only when some
-//     head of the unit has a token with u > τ in it.  Splits write partial
-//     outputs and the last split of a unit (an atomic ticket, no waiting)
-//     adds them in split order, so results are deterministic.
+//  1. qk: z = scale·q·k for every valid token of every selected page and the
+//     G query heads of the unit.  A (page, KV head) K tile is one contiguous
+//     block of S rows; for bf16 each 16-token half is the A operand of a
+//     tensor-core MMA (m16n8k16) whose B operand is the group's queries, with
+//     rows loaded straight into fragment registers (the same k permutation
+//     as the page-score kernel).  Scores land in an L2-resident scratch with
+//     per-page and per-CTA maxima.
+//  2. tau: per query head, τ with Σ_i [u_i − τ]_+^β = 1, u = (α−1)·z,
+//     β = 1/(α−1).  f(τ) = Σ[u − τ]_+^β is convex and decreasing, so Newton's
+//     method started left of the root rises to it without overshooting.  The
+//     start comes from a 256-bin histogram of u over (max u − 1, max u]: if
+//     c values exceed an edge e then τ ≥ e − c^(−1/β) (c of them would give
+//     mass ≥ 1 at that τ), which lands within a bin of the root.  For β ∈ {1,2}
+//     the final τ is the closed form on the support found.
+//  3. pv: each CTA lists the selected pages of its run that hold support
+//     (some head has a token with u > τ) and its warps read only those V
+//     pages, one whole row per load instruction; CTA partials are added by
+//     the unit's last CTA (an atomic ticket, no waiting) in CTA order, so
+//     results are deterministic.
 #include "kernels.cuh"
 
 namespace ekv {
@@ -37,7 +44,7 @@ struct DecodeArgs {
   DecodeWs ws;
   float scale, am1, beta;
   int ibeta;  // β when it is 1 or 2, else 0
-  int Hkv, Hq, S, num_phys, max_pages, cap, nsplit, sps, tp, dense_v, words;
+  int Hkv, Hq, S, num_phys, max_pages, cap, spp_pv, dense_v, words;
 };
 
 __device__ __forceinline__ int unit_slots(const DecodeArgs& a, int unit, int P) {
@@ -67,23 +74,164 @@ __device__ __forceinline__ float pow_beta(float w, float beta, int ibeta) {
   return powf(w, beta);
 }
 
-// ------------------------------------------------------------------ 1. qk
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) qk_kernel(DecodeArgs a) {
-  constexpr int PAD = 16 / sizeof(T);
-  constexpr int RP = D + PAD;  // padded row pitch: rows start in different bank groups
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* q_s = reinterpret_cast<float*>(smem_raw);
-  T* ktile = reinterpret_cast<T*>(smem_raw + G * D * sizeof(float));
-  __shared__ int s_phys[8], s_nv[8];
-  __shared__ unsigned int cta_key[G];
+// ------------------------------------------------------------------ 1. qk (bf16 tensor cores)
+constexpr int kQkWarps = kQkTokensPerCta / 32;
 
+template <int D, int G>
+__global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) {
+  constexpr int KP = D / 32;          // 32-element chunks per K row
+  constexpr int NT = (G + 7) / 8;     // 8-head tiles of the B operand
+  __shared__ unsigned int cta_key[G];
   const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int tid = threadIdx.x, S = a.S, TP = a.tp;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int S = a.S;
   int L;
   const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
   const int n_slots = unit_slots(a, unit, P);
-  const int s0 = split * a.sps, s1 = min(s0 + a.sps, n_slots);
+  const int ppc = kQkTokensPerCta / S;  // pages per CTA
+  const int s_begin = split * ppc;
+  if (tid < G) cta_key[tid] = 0u;
+  if (split == 0 && tid == 0) a.ws.counter[unit] = 0;
+  __syncthreads();
+
+  // this warp's 32 token rows form two 16-row m-tiles of one or two pages
+  const int row0 = warp * 32;
+  int phys[2], nv[2], slot[2];
+  bool live[2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const int r = row0 + mt * 16;
+    slot[mt] = s_begin + r / S;
+    live[mt] = slot[mt] < n_slots;
+    phys[mt] = -1;
+    nv[mt] = 0;
+    if (live[mt]) phys[mt] = slot_page(a, unit, b, slot[mt], P, L, &nv[mt]);
+  }
+  // K rows straight into A fragments: rows g and g + 8 of each m-tile
+  uint4 va[2][KP], vb[2][KP];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const int tok0 = (row0 + mt * 16) % S;
+    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+    const bf16* kb = static_cast<const bf16*>(a.k_pool) +
+                     ((static_cast<size_t>(phys[mt] < 0 ? 0 : phys[mt]) * a.Hkv + kvh) * S + tok0) * D;
+    const uint4* row_lo = reinterpret_cast<const uint4*>(kb + g * D) + t;
+    const uint4* row_hi = reinterpret_cast<const uint4*>(kb + (g + 8) * D) + t;
+#pragma unroll
+    for (int c = 0; c < KP; ++c) {
+      va[mt][c] = ok_lo ? __ldcs(row_lo + 4 * c) : make_uint4(0, 0, 0, 0);
+      vb[mt][c] = ok_hi ? __ldcs(row_hi + 4 * c) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // B fragments: the group's queries under the same k permutation
+  uint32_t bfrag[2 * KP][NT][2];
+  {
+    const bf16* qb = static_cast<const bf16*>(a.q) + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G) * D;
+#pragma unroll
+    for (int ks = 0; ks < 2 * KP; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int col = nt * 8 + g;
+        const int k0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
+        if (col < G) {
+          const uint2 w = *reinterpret_cast<const uint2*>(qb + col * D + k0);
+          bfrag[ks][nt][0] = w.x;
+          bfrag[ks][nt][1] = w.y;
+        } else {
+          bfrag[ks][nt][0] = bfrag[ks][nt][1] = 0u;
+        }
+      }
+  }
+  const size_t zrow = static_cast<size_t>(a.cap) * S;
+  float pm[2][NT][2];  // page maxima per m-tile for heads 2t, 2t+1 of each tile
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int c = 0; c < KP; ++c) {
+      const uint32_t f0[4] = {va[mt][c].x, vb[mt][c].x, va[mt][c].y, vb[mt][c].y};
+      const uint32_t f1[4] = {va[mt][c].z, vb[mt][c].z, va[mt][c].w, vb[mt][c].w};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16(acc[nt], f0, bfrag[2 * c][nt][0], bfrag[2 * c][nt][1]);
+        mma_bf16(acc[nt], f1, bfrag[2 * c + 1][nt][0], bfrag[2 * c + 1][nt][1]);
+      }
+    }
+    const int tok0 = (row0 + mt * 16) % S;
+    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int hd = nt * 8 + 2 * t + e;
+        const float zl = ok_lo ? a.scale * acc[nt][e] : -INFINITY;
+        const float zh = ok_hi ? a.scale * acc[nt][2 + e] : -INFINITY;
+        if (live[mt] && hd < G) {
+          float* zr = a.ws.zbuf + (static_cast<size_t>(unit) * G + hd) * zrow + static_cast<size_t>(slot[mt]) * S + tok0;
+          zr[g] = zl;
+          zr[g + 8] = zh;
+        }
+        float m = fmaxf(zl, zh);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        pm[mt][nt][e] = m;
+      }
+  }
+  // page maxima: one page per m-tile (S = 16) or per warp (S = 32)
+  if (g == 0) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int hd = nt * 8 + 2 * t + e;
+        if (hd >= G) continue;
+        float* prow = a.ws.pmax + (static_cast<size_t>(unit) * G + hd) * a.cap;
+        if (S == 16) {
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            if (live[mt]) {
+              prow[slot[mt]] = pm[mt][nt][e];
+              if (pm[mt][nt][e] > -INFINITY) atomicMax(&cta_key[hd], float_key(pm[mt][nt][e]));
+            }
+        } else if (live[0]) {
+          const float m = fmaxf(pm[0][nt][e], pm[1][nt][e]);
+          prow[slot[0]] = m;
+          if (m > -INFINITY) atomicMax(&cta_key[hd], float_key(m));
+        }
+      }
+  }
+  __syncthreads();
+  if (tid < G) {
+    const unsigned int k = cta_key[tid];
+    a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
+  }
+}
+
+// ------------------------------------------------------------------ 1'. qk (CUDA cores, fp32 caches)
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(256) qk_cc_kernel(DecodeArgs a) {
+  constexpr int PAD = 16 / sizeof(T);
+  constexpr int RP = D + PAD;  // padded row pitch: rows start in different bank groups
+  constexpr int TP = 4;        // pages staged per round
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* q_s = reinterpret_cast<float*>(smem_raw);
+  T* ktile = reinterpret_cast<T*>(smem_raw + G * D * sizeof(float));
+  __shared__ int s_phys[TP], s_nv[TP];
+  __shared__ unsigned int cta_key[G];
+
+  const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int tid = threadIdx.x, S = a.S;
+  int L;
+  const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
+  const int n_slots = unit_slots(a, unit, P);
+  const int ppc = kQkTokensPerCta / S;
+  const int s0 = split * ppc, s1 = min(s0 + ppc, n_slots);
   if (split == 0 && tid == 0) a.ws.counter[unit] = 0;
 
   const T* qb = static_cast<const T*>(a.q) + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G) * D;
@@ -111,8 +259,7 @@ __global__ void __launch_bounds__(256) qk_kernel(DecodeArgs a) {
       }
     }
     __syncthreads();
-    // whole warps iterate (the page maxima below shuffle across S lanes)
-    const int items = (TP * G * S + 31) / 32 * 32;
+    const int items = (TP * G * S + 31) / 32 * 32;  // whole warps (page maxima shuffle across S lanes)
     for (int it = tid; it < items; it += blockDim.x) {
       const int tp = it / (G * S), g = (it / S) % G, t = it % S;
       float z = -INFINITY;
@@ -135,11 +282,11 @@ __global__ void __launch_bounds__(256) qk_kernel(DecodeArgs a) {
       }
       const size_t row = static_cast<size_t>(unit) * G + g;
       if (tp < np) a.ws.zbuf[row * zrow + static_cast<size_t>(base + tp) * S + t] = z;
-      float pm = z;
-      for (int o = S / 2; o > 0; o >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+      float pmx = z;
+      for (int o = S / 2; o > 0; o >>= 1) pmx = fmaxf(pmx, __shfl_xor_sync(0xffffffffu, pmx, o));
       if (t == 0 && tp < np) {
-        a.ws.pmax[row * a.cap + base + tp] = pm;
-        if (pm > -INFINITY) atomicMax(&cta_key[g], float_key(pm));
+        a.ws.pmax[row * a.cap + base + tp] = pmx;
+        if (pmx > -INFINITY) atomicMax(&cta_key[g], float_key(pmx));
       }
     }
     __syncthreads();
@@ -147,45 +294,97 @@ __global__ void __launch_bounds__(256) qk_kernel(DecodeArgs a) {
   __syncthreads();
   if (tid < G) {
     const unsigned int k = cta_key[tid];
-    a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.nsplit + split] = k == 0u ? -INFINITY : key_float(k);
+    a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
   }
 }
 
 // ------------------------------------------------------------------ 2. tau
-constexpr int kTauThreads = 512;
+constexpr int kTauThreads = 256;
+constexpr int kTauBins = 256;
+
+// Sums three doubles over the block; every thread gets the totals.
+__device__ __forceinline__ void block_sum3(double& x, double& y, double& z, double* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y += __shfl_xor_sync(0xffffffffu, y, o);
+    z += __shfl_xor_sync(0xffffffffu, z, o);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    scratch[3 * warp] = x;
+    scratch[3 * warp + 1] = y;
+    scratch[3 * warp + 2] = z;
+  }
+  __syncthreads();
+  x = y = z = 0.0;
+  for (int w = 0; w < nw; ++w) {
+    x += scratch[3 * w];
+    y += scratch[3 * w + 1];
+    z += scratch[3 * w + 2];
+  }
+}
 
 template <int VPT>
 __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
   const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / a.Hkv, kvh = unit % a.Hkv;
   const int tid = threadIdx.x, nt = blockDim.x;
   __shared__ float f_scratch[32];
-  __shared__ double d_scratch[32];
+  __shared__ double d_scratch[3 * 32];
   __shared__ int i_scratch[32];
+  __shared__ int hist[kTauBins];
   int L;
   const int P = seq_pages(a.seq_lens, b, a.S, a.max_pages, &L);
   const int n = unit_slots(a, unit, P) * a.S;
   const float* z = a.ws.zbuf + static_cast<size_t>(row) * a.cap * a.S;
   const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + g;
+  const float am1 = a.am1, beta = a.beta;
+  const int ib = a.ibeta;
 
   float m = -INFINITY;
-  for (int s = tid; s < a.nsplit; s += nt) m = fmaxf(m, a.ws.cmax[static_cast<size_t>(row) * a.nsplit + s]);
+  for (int s = tid; s < a.ws.nqk; s += nt) m = fmaxf(m, a.ws.cmax[static_cast<size_t>(row) * a.ws.nqk + s]);
   m = block_reduce(m, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+
+  float uv[VPT > 0 ? VPT : 1];
+#pragma unroll
+  for (int k = 0; k < (VPT > 0 ? VPT : 1); ++k) {
+    const int i = tid + k * nt;
+    uv[k] = (VPT > 0 && i < n) ? am1 * z[i] : -INFINITY;
+  }
+  // applies fn(u) to every value of the row
+  auto for_values = [&](auto fn) {
+    if constexpr (VPT > 0) {
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) fn(uv[k]);
+    } else {
+      for (int i = tid; i < n; i += nt) fn(am1 * z[i]);
+    }
+  };
 
   float tau_f = INFINITY;  // no token: no support, zero output
   if (n > 0 && m > -INFINITY) {
-    const float am1 = a.am1, beta = a.beta;
-    const int ib = a.ibeta;
-    float uv[VPT > 0 ? VPT : 1];
-#pragma unroll
-    for (int k = 0; k < (VPT > 0 ? VPT : 1); ++k) {
-      const int i = tid + k * nt;
-      uv[k] = (VPT > 0 && i < n) ? am1 * z[i] : -INFINITY;
+    const float um = am1 * m;
+    // lower bracket from the histogram of u over (um − 1, um]
+    for (int i = tid; i < kTauBins; i += nt) hist[i] = 0;
+    __syncthreads();
+    for_values([&](float u) {
+      if (u > um - 1.0f) atomicAdd(&hist[min(kTauBins - 1, static_cast<int>((um - u) * kTauBins))], 1);
+    });
+    __syncthreads();
+    float cand = um - 1.0f;
+    if (tid < kTauBins) {
+      int c = 0;  // values in bins 0..tid (u above the edge um − (tid+1)/bins, up to rounding)
+      for (int j = 0; j <= tid; ++j) c += hist[j];
+      if (c > 0)
+        cand = fmaxf(cand, um - static_cast<float>(tid + 1) / kTauBins - powf(static_cast<float>(c), -1.0f / beta));
     }
-    auto accumulate = [&](double t, double& f, double& df) {
-      f = 0.0;
-      df = 0.0;
-      auto term = [&](float u) {
-        const double w = static_cast<double>(u) - t;
+    cand = block_reduce(cand, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+    double tau = static_cast<double>(cand) - 1e-6 * (1.0 + fabs(static_cast<double>(um)));
+    for (int it = 0; it < 100; ++it) {
+      double f = 0.0, df = 0.0, unused = 0.0;
+      for_values([&](float u) {
+        const double w = static_cast<double>(u) - tau;
         if (w > 0.0) {
           if (ib == 1) {
             f += w;
@@ -199,20 +398,12 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
             df += wb1;
           }
         }
-      };
-      if (VPT > 0) {
-#pragma unroll
-        for (int k = 0; k < (VPT > 0 ? VPT : 1); ++k) term(uv[k]);
-      } else {
-        for (int i = tid; i < n; i += nt) term(am1 * z[i]);
+      });
+      block_sum3(f, df, unused, d_scratch);
+      if (it == 0 && f < 1.0) {  // bracket missed (rounding): restart from max u − 1
+        tau = static_cast<double>(um) - 1.0;
+        continue;
       }
-    };
-    double tau = static_cast<double>(am1 * m) - 1.0;
-    for (int it = 0; it < 200; ++it) {
-      double f, df;
-      accumulate(tau, f, df);
-      f = block_reduce(f, d_scratch, [](double x, double y) { return x + y; });
-      df = block_reduce(df, d_scratch, [](double x, double y) { return x + y; });
       const double step = (f - 1.0) / (static_cast<double>(beta) * df);
       if (!(step > 0.0)) break;
       tau += step;
@@ -223,22 +414,14 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
       // β = 2: τ = M − √(M² − Q + 1/k) with M, Q the mean and mean square
       for (int rep = 0; rep < 4; ++rep) {
         double c = 0.0, s1 = 0.0, s2 = 0.0;
-        auto add = [&](float u) {
+        for_values([&](float u) {
           if (static_cast<double>(u) > tau) {
             c += 1.0;
             s1 += u;
             s2 += static_cast<double>(u) * u;
           }
-        };
-        if (VPT > 0) {
-#pragma unroll
-          for (int k = 0; k < (VPT > 0 ? VPT : 1); ++k) add(uv[k]);
-        } else {
-          for (int i = tid; i < n; i += nt) add(am1 * z[i]);
-        }
-        c = block_reduce(c, d_scratch, [](double x, double y) { return x + y; });
-        s1 = block_reduce(s1, d_scratch, [](double x, double y) { return x + y; });
-        s2 = block_reduce(s2, d_scratch, [](double x, double y) { return x + y; });
+        });
+        block_sum3(c, s1, s2, d_scratch);
         if (c < 1.0) break;
         double t_new;
         if (ib == 1) {
@@ -259,17 +442,14 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
   const int words = a.words;
   for (int base = 0; base < (n + nt - 1) / nt * nt; base += nt) {
     const int i = base + tid;
-    const bool in = i < n && a.am1 * z[i] > tau_f;
+    const bool in = i < n && am1 * z[i] > tau_f;
     cnt += in ? 1 : 0;
     const unsigned int bal = __ballot_sync(0xffffffffu, in);
-    if (a.bits_out && (tid & 31) == 0 && (i >> 5) < words)
-      a.bits_out[orow * words + (i >> 5)] = bal;
+    if (a.bits_out && (tid & 31) == 0 && (i >> 5) < words) a.bits_out[orow * words + (i >> 5)] = bal;
   }
   cnt = block_reduce(cnt, i_scratch, [](int x, int y) { return x + y; });
-  if (a.bits_out) {
-    // clear words past the tokens of this unit
+  if (a.bits_out)
     for (int w = (n + 31) / 32 + tid; w < words; w += nt) a.bits_out[orow * words + w] = 0u;
-  }
   if (tid == 0) {
     a.ws.taus[row] = tau_f;
     if (a.tau_out) a.tau_out[orow] = tau_f;
@@ -278,169 +458,161 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
 }
 
 // ------------------------------------------------------------------ 3. pv
-constexpr int kPvPages = 4;
+constexpr int kPvWarps = 8;
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) pv_kernel(DecodeArgs a) {
-  constexpr int NPAIR = G * D / 2;
-  constexpr int IPT = (NPAIR + 255) / 256;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* vtile = reinterpret_cast<T*>(smem_raw);                                  // [kPvPages][S][D]
-  float* p_s = reinterpret_cast<float*>(smem_raw + kPvPages * a.S * D * sizeof(T));  // [kPvPages][G][S]
+__global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
+  constexpr int DPL = D / 32;  // output columns per lane
+  extern __shared__ __align__(16) float red[];  // [kPvWarps][G][D]
   __shared__ float s_tau[G];
-  __shared__ int s_list[256];
-  __shared__ int s_phys[kPvPages], s_nv[kPvPages], s_slot[kPvPages];
+  __shared__ int s_list[32 * kPvWarps];
   __shared__ int scan_scratch[32];
   __shared__ int s_last;
 
   const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int tid = threadIdx.x, S = a.S;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, S = a.S;
   int L;
   const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
   const int n_slots = unit_slots(a, unit, P);
-  const int s0 = split * a.sps, s1 = min(s0 + a.sps, n_slots);
+  const int s0 = split * a.spp_pv, s1 = min(s0 + a.spp_pv, n_slots);
   if (tid < G) s_tau[tid] = a.ws.taus[static_cast<size_t>(unit) * G + tid];
   __syncthreads();
 
-  float2 acc[IPT];
+  float acc[G][DPL];
 #pragma unroll
-  for (int k = 0; k < IPT; ++k) acc[k] = make_float2(0.f, 0.f);
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
   const size_t zrow = static_cast<size_t>(a.cap) * S;
 
-  for (int wbase = s0; wbase < s1; wbase += 256) {
-    const int slot = wbase + tid;
+  for (int w0 = s0; w0 < s1; w0 += blockDim.x) {
+    // the window's pages that hold support, in ascending order
+    const int slot = w0 + tid;
     int sup = 0;
     if (slot < s1) {
       if (a.dense_v) {
         sup = 1;
       } else {
-        for (int g = 0; g < G; ++g)
-          if (a.am1 * a.ws.pmax[(static_cast<size_t>(unit) * G + g) * a.cap + slot] > s_tau[g]) sup = 1;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          if (a.am1 * a.ws.pmax[(static_cast<size_t>(unit) * G + h) * a.cap + slot] > s_tau[h]) sup = 1;
       }
     }
     int nsup;
     const int pos = block_exclusive_scan(sup, scan_scratch, &nsup);
     if (sup) s_list[pos] = slot;
     __syncthreads();
-    for (int lb = 0; lb < nsup; lb += kPvPages) {
-      const int np = min(kPvPages, nsup - lb);
-      if (tid < np) {
-        int nv;
-        const int sl = s_list[lb + tid];
-        s_slot[tid] = sl;
-        s_phys[tid] = slot_page(a, unit, b, sl, P, L, &nv);
-        s_nv[tid] = s_phys[tid] >= 0 ? nv : 0;
-      }
-      __syncthreads();
-      constexpr int CPR = D * sizeof(T) / 16;
-      for (int i = tid; i < np * S * CPR; i += blockDim.x) {
-        const int tp = i / (S * CPR), r = (i / CPR) % S, c = i % CPR;
-        if (r < s_nv[tp]) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              static_cast<const T*>(a.v_pool) + ((static_cast<size_t>(s_phys[tp]) * a.Hkv + kvh) * S + r) * D) + c;
-          *reinterpret_cast<uint4*>(vtile + (tp * S + r) * D + c * (16 / sizeof(T))) = __ldcs(src);
-        }
-      }
-      for (int i = tid; i < np * G * S; i += blockDim.x) {
-        const int tp = i / (G * S), g = (i / S) % G, t = i % S;
-        float p = 0.f;
-        if (t < s_nv[tp]) {
-          const float u = a.am1 * a.ws.zbuf[(static_cast<size_t>(unit) * G + g) * zrow +
-                                            static_cast<size_t>(s_slot[tp]) * S + t];
-          const float w = u - s_tau[g];
-          if (w > 0.f) p = pow_beta(w, a.beta, a.ibeta);
-        }
-        p_s[(tp * G + g) * S + t] = p;
-      }
-      __syncthreads();
+    for (int e = warp; e < nsup; e += kPvWarps) {
+      const int sl = s_list[e];
+      int nv;
+      const int phys = slot_page(a, unit, b, sl, P, L, &nv);
+      if (phys < 0) continue;
+      // p of token `lane` for every head
+      float p[G];
 #pragma unroll
-      for (int k = 0; k < IPT; ++k) {
-        const int pair = tid + k * 256;
-        if (pair < NPAIR) {
-          const int g = pair / (D / 2), j = 2 * (pair % (D / 2));
-          for (int tp = 0; tp < np; ++tp) {
-            const int nv = s_nv[tp];
-            const float* pr = p_s + (tp * G + g) * S;
-            const T* vr = vtile + tp * S * D + j;
-            for (int t = 0; t < nv; ++t) {
-              const float p = pr[t];
-              float v0, v1;
-              if (sizeof(T) == 2) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(vr + t * D);
-                v0 = __uint_as_float(w << 16);
-                v1 = __uint_as_float(w & 0xffff0000u);
-              } else {
-                const float2 f = *reinterpret_cast<const float2*>(vr + t * D);
-                v0 = f.x;
-                v1 = f.y;
-              }
-              acc[k] = ffma2(make_float2(p, p), make_float2(v0, v1), acc[k]);
+      for (int h = 0; h < G; ++h) {
+        p[h] = 0.f;
+        if (lane < nv) {
+          const float w = a.am1 * a.ws.zbuf[(static_cast<size_t>(unit) * G + h) * zrow + static_cast<size_t>(sl) * S + lane] - s_tau[h];
+          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ibeta);
+        }
+      }
+      const T* vb = static_cast<const T*>(a.v_pool) + (static_cast<size_t>(phys) * a.Hkv + kvh) * S * D + lane * DPL;
+      for (int t0 = 0; t0 < nv; t0 += 8) {
+        float vv[8][DPL];
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+          const int t = t0 + tt;
+          if (t < nv) {
+            if constexpr (DPL == 4) {
+              load4(vb + static_cast<size_t>(t) * D, vv[tt]);
+            } else {
+              const T* src = vb + static_cast<size_t>(t) * D;
+              vv[tt][0] = to_f32(src[0]);
+              vv[tt][1] = to_f32(src[1]);
             }
+          } else {
+#pragma unroll
+            for (int e2 = 0; e2 < DPL; ++e2) vv[tt][e2] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float ph = __shfl_sync(0xffffffffu, p[h], (t0 + tt) & 31);
+#pragma unroll
+            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(ph, vv[tt][e2], acc[h][e2]);
           }
         }
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
 
-  // partial outputs, then the last split of the unit reduces them in order
-  float* part = a.ws.part + (static_cast<size_t>(unit) * a.nsplit + split) * G * D;
+  // CTA partial → workspace; the unit's last CTA adds the partials in order
 #pragma unroll
-  for (int k = 0; k < IPT; ++k) {
-    const int pair = tid + k * 256;
-    if (pair < NPAIR) *reinterpret_cast<float2*>(part + 2 * pair) = acc[k];
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) red[(warp * G + h) * D + lane * DPL + e] = acc[h][e];
+  __syncthreads();
+  float* part = a.ws.part + (static_cast<size_t>(unit) * a.ws.npv + split) * G * D;
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    float s = 0.f;
+    for (int w = 0; w < kPvWarps; ++w) s += red[w * G * D + i];
+    part[i] = s;
   }
   __syncthreads();
   if (tid == 0) {
     __threadfence();
     const int ticket = atomicAdd(&a.ws.counter[unit], 1);
-    s_last = ticket == a.nsplit - 1;
+    s_last = ticket == a.ws.npv - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const float* part0 = a.ws.part + static_cast<size_t>(unit) * a.nsplit * G * D;
-  for (int e = tid; e < G * D; e += blockDim.x) {
+  const float* part0 = a.ws.part + static_cast<size_t>(unit) * a.ws.npv * G * D;
+  for (int i = tid; i < G * D; i += blockDim.x) {
     float s = 0.f;
-    for (int sp = 0; sp < a.nsplit; ++sp) s += __ldcg(part0 + static_cast<size_t>(sp) * G * D + e);
-    const int g = e / D, j = e % D;
-    a.out[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + g) * D + j] = s;
+    for (int sp = 0; sp < a.ws.npv; ++sp) s += __ldcg(part0 + static_cast<size_t>(sp) * G * D + i);
+    const int h = i / D, j = i % D;
+    a.out[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h) * D + j] = s;
   }
   if (tid == 0) a.ws.counter[unit] = 0;
 }
 
 template <typename T, int D, int G>
 cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
-  constexpr int PAD = 16 / sizeof(T);
-  const size_t row_bytes = static_cast<size_t>(D + PAD) * sizeof(T);
-  const size_t q_bytes = static_cast<size_t>(G) * D * sizeof(float);
-  int tp = 256 / (G * a.S);
-  tp = tp < 1 ? 1 : (tp > 8 ? 8 : tp);
-  while (tp > 1 && q_bytes + static_cast<size_t>(tp) * a.S * row_bytes > 48 * 1024) tp >>= 1;
-  a.tp = tp;
-  const size_t qk_smem = q_bytes + static_cast<size_t>(tp) * a.S * row_bytes;
-  const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(U));
-  if (qk_smem > 48 * 1024)
-    cudaFuncSetAttribute(qk_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(qk_smem));
-  qk_kernel<T, D, G><<<grid, 256, qk_smem, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  const dim3 gq(static_cast<unsigned>(a.ws.nqk), static_cast<unsigned>(U));
+  if constexpr (sizeof(T) == 2) {
+    qk_mma_kernel<D, G><<<gq, 32 * kQkWarps, 0, st>>>(a);
+  } else {
+    const size_t smem = static_cast<size_t>(G) * D * sizeof(float) + 4 * static_cast<size_t>(a.S) * (D + 16 / sizeof(T)) * sizeof(T);
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(qk_cc_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    qk_cc_kernel<T, D, G><<<gq, 256, smem, st>>>(a);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_max = a.cap * a.S;
-  if (n_max <= 8 * kTauThreads)
-    tau_kernel<8><<<U * G, kTauThreads, 0, st>>>(a, G);
-  else if (n_max <= 32 * kTauThreads)
-    tau_kernel<32><<<U * G, kTauThreads, 0, st>>>(a, G);
+  if (n_max <= 16 * kTauThreads)
+    tau_kernel<16><<<U * G, kTauThreads, 0, st>>>(a, G);
+  else if (n_max <= 64 * kTauThreads)
+    tau_kernel<64><<<U * G, kTauThreads, 0, st>>>(a, G);
   else
     tau_kernel<0><<<U * G, kTauThreads, 0, st>>>(a, G);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t pv_smem = static_cast<size_t>(kPvPages) * a.S * D * sizeof(T) +
-                         static_cast<size_t>(kPvPages) * G * a.S * sizeof(float);
-  if (pv_smem > 48 * 1024)
-    cudaFuncSetAttribute(pv_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(pv_smem));
-  pv_kernel<T, D, G><<<grid, 256, pv_smem, st>>>(a);
+  const size_t pv_smem = static_cast<size_t>(kPvWarps) * G * D * sizeof(float);
+  if (pv_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(pv_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pv_smem));
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 gp(static_cast<unsigned>(a.ws.npv), static_cast<unsigned>(U));
+  pv_kernel<T, D, G><<<gp, 32 * kPvWarps, pv_smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -449,7 +621,7 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
 cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
                           float scale, float alpha, const int32_t* sel, const int32_t* n_sel,
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
-                          uint32_t* support_bits, const DecodeWs& ws, int nsplit, cudaStream_t st) {
+                          uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st) {
   DecodeArgs a{};
   a.k_pool = c.k_pool;
   a.v_pool = c.v_pool;
@@ -473,8 +645,7 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
   a.num_phys = c.num_phys_pages;
   a.max_pages = s.max_pages;
   a.cap = cap;
-  a.nsplit = nsplit;
-  a.sps = (cap + nsplit - 1) / nsplit;
+  a.spp_pv = (cap + ws.npv - 1) / ws.npv;
   a.dense_v = dense_v;
   a.words = (cap * c.page_size + 31) / 32;
   const int G = Hq / c.num_kv_heads, U = s.batch * c.num_kv_heads;

@@ -6,16 +6,20 @@
 
 namespace ekv {
 
-// CTAs the split-over-pages decode kernels aim for (two per SM of a B200).
-constexpr int kDecodeTargetCtas = 296;
+// Decode work split.  The score pass over the selected K takes 256 tokens per
+// CTA (8 warps × 32 tokens); the V pass aims for two CTAs per SM of a B200.
+constexpr int kQkTokensPerCta = 256;
+constexpr int kPvTargetCtas = 296;
+constexpr int kPvMaxSplits = 64;
 
 struct DecodeWs {
   float* zbuf;      // [U, G, cap·S] scores z of the selected tokens (−inf: no token)
   float* pmax;      // [U, G, cap]   page maxima of z
-  float* cmax;      // [U, G, nsplit] split maxima of z
+  float* cmax;      // [U, G, nqk]   maxima of z per score-pass CTA
   float* taus;      // [U, G]        thresholds τ (fp32)
-  float* part;      // [U, nsplit, G, d] partial outputs of the V pass
-  int* counter;     // [U]           finished V-pass splits
+  float* part;      // [U, npv, G, d] partial outputs of the V pass
+  int* counter;     // [U]           finished V-pass CTAs
+  int nqk, npv;     // score-pass and V-pass CTAs per unit
 };
 
 struct GaussWs {
@@ -40,10 +44,17 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
 cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
                           float scale, float alpha, const int32_t* sel, const int32_t* n_sel,
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
-                          uint32_t* support_bits, const DecodeWs& ws, int nsplit, cudaStream_t st);
+                          uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st);
 
-inline int decode_splits(int units, int cap) {
-  int ns = (kDecodeTargetCtas + units - 1) / units;
+// Score-pass CTAs per unit: cap pages of S tokens, 256 tokens per CTA.
+inline int qk_splits(int cap, int S) {
+  const int pages = kQkTokensPerCta / S;
+  return (cap + pages - 1) / pages;
+}
+// V-pass CTAs per unit (each scans an equal run of the selected pages).
+inline int pv_splits(int units, int cap) {
+  int ns = (kPvTargetCtas + units - 1) / units;
+  if (ns > kPvMaxSplits) ns = kPvMaxSplits;
   if (ns > cap) ns = cap;
   if (ns < 1) ns = 1;
   const int per = (cap + ns - 1) / ns;
