@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/ekv.h"
 
 namespace ekv {
@@ -16,6 +18,34 @@ using bf16 = __nv_bfloat16;
 extern __device__ unsigned int g_error_flags;
 
 __device__ __forceinline__ void raise_flag(unsigned int bit) { atomicOr(&g_error_flags, bit); }
+
+// ------------------------------------------------------------------ launches
+// Every kernel is launched with programmatic stream serialization: its CTAs
+// may be dispatched while the previous kernel on the stream drains.  Each
+// kernel therefore opens with grid_dep_enter(): it waits until the previous
+// kernel has completed and its memory is visible (griddepcontrol.wait; a
+// no-op when launched without the attribute), then lets the next kernel be
+// dispatched early.  No global memory is read or written before the wait.
+__device__ __forceinline__ void grid_dep_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ loads
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -225,6 +255,7 @@ __device__ __forceinline__ V block_reduce(V v, V* scratch, Op op) {
 }
 
 // Exclusive prefix sum of an int over the block; *total receives the sum.
+// Warp scans, then one warp scans the warp totals (blockDim.x ≤ 1024).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int x = v;
@@ -236,14 +267,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
   __syncthreads();
   if (lane == 31) scratch[warp] = x;
   __syncthreads();
-  int before = 0, all = 0;
-  for (int w = 0; w < nw; ++w) {
-    const int s = scratch[w];
-    if (w < warp) before += s;
-    all += s;
+  if (warp == 0) {
+    int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) scratch[lane] = w;  // inclusive warp-total prefix
   }
-  *total = all;
-  return before + x - v;
+  __syncthreads();
+  *total = scratch[nw - 1];
+  return (warp > 0 ? scratch[warp - 1] : 0) + x - v;
 }
 
 // ------------------------------------------------------------------ async copies

@@ -23,62 +23,18 @@
 //     pages, one whole row per load instruction; CTA partials are added by
 //     the unit's last CTA (an atomic ticket, no waiting) in CTA order, so
 //     results are deterministic.
-#include "kernels.cuh"
+#include "decode.cuh"
 
 namespace ekv {
 
 namespace {
-
-struct DecodeArgs {
-  const void* k_pool;
-  const void* v_pool;
-  const int32_t* page_table;
-  const int32_t* seq_lens;
-  const void* q;
-  const int32_t* sel;
-  const int32_t* n_sel;
-  float* out;
-  float* tau_out;
-  int32_t* count_out;
-  uint32_t* bits_out;
-  DecodeWs ws;
-  float scale, am1, beta;
-  int ibeta;  // β when it is 1 or 2, else 0
-  int Hkv, Hq, S, num_phys, max_pages, cap, spp_pv, dense_v, words;
-};
-
-__device__ __forceinline__ int unit_slots(const DecodeArgs& a, int unit, int P) {
-  if (a.sel == nullptr) return min(P, a.cap);
-  const int n = a.n_sel[unit];
-  return max(0, min(n, a.cap));
-}
-
-// Logical page of a selected slot → (physical page, valid tokens); −1 when bad.
-__device__ __forceinline__ int slot_page(const DecodeArgs& a, int unit, int b, int slot, int P,
-                                         int L, int* nv) {
-  const int lp = a.sel ? a.sel[static_cast<size_t>(unit) * a.cap + slot] : slot;
-  *nv = 0;
-  if (lp < 0 || lp >= P) {
-    raise_flag(EKV_EFLAG_BAD_SEL);
-    return -1;
-  }
-  const int phys = a.page_table[static_cast<size_t>(b) * a.max_pages + lp];
-  if (!phys_ok(phys, a.num_phys)) return -1;
-  *nv = min(a.S, L - lp * a.S);
-  return phys;
-}
-
-__device__ __forceinline__ float pow_beta(float w, float beta, int ibeta) {
-  if (ibeta == 1) return w;
-  if (ibeta == 2) return w * w;
-  return powf(w, beta);
-}
 
 // ------------------------------------------------------------------ 1. qk (bf16 tensor cores)
 constexpr int kQkWarps = kQkTokensPerCta / 32;
 
 template <int D, int G>
 __global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) {
+  grid_dep_enter();
   constexpr int KP = D / 32;          // 32-element chunks per K row
   constexpr int NT = (G + 7) / 8;     // 8-head tiles of the B operand
   __shared__ unsigned int cta_key[G];
@@ -127,40 +83,13 @@ __global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) 
   }
   // B fragments: the group's queries under the same k permutation
   uint32_t bfrag[2 * KP][NT][2];
-  {
-    const bf16* qb = static_cast<const bf16*>(a.q) + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G) * D;
-#pragma unroll
-    for (int ks = 0; ks < 2 * KP; ++ks)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int col = nt * 8 + g;
-        const int k0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
-        if (col < G) {
-          const uint2 w = *reinterpret_cast<const uint2*>(qb + col * D + k0);
-          bfrag[ks][nt][0] = w.x;
-          bfrag[ks][nt][1] = w.y;
-        } else {
-          bfrag[ks][nt][0] = bfrag[ks][nt][1] = 0u;
-        }
-      }
-  }
+  load_q_frags<D, G>(a, b, kvh, g, t, bfrag);
   const size_t zrow = static_cast<size_t>(a.cap) * S;
   float pm[2][NT][2];  // page maxima per m-tile for heads 2t, 2t+1 of each tile
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt) {
     float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-    for (int c = 0; c < KP; ++c) {
-      const uint32_t f0[4] = {va[mt][c].x, vb[mt][c].x, va[mt][c].y, vb[mt][c].y};
-      const uint32_t f1[4] = {va[mt][c].z, vb[mt][c].z, va[mt][c].w, vb[mt][c].w};
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_bf16(acc[nt], f0, bfrag[2 * c][nt][0], bfrag[2 * c][nt][1]);
-        mma_bf16(acc[nt], f1, bfrag[2 * c + 1][nt][0], bfrag[2 * c + 1][nt][1]);
-      }
-    }
+    score_mtile<D, G>(va[mt], vb[mt], bfrag, acc);
     const int tok0 = (row0 + mt * 16) % S;
     const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
     const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
@@ -216,6 +145,7 @@ __global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) 
 // ------------------------------------------------------------------ 1'. qk (CUDA cores, fp32 caches)
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) qk_cc_kernel(DecodeArgs a) {
+  grid_dep_enter();
   constexpr int PAD = 16 / sizeof(T);
   constexpr int RP = D + PAD;  // padded row pitch: rows start in different bank groups
   constexpr int TP = 4;        // pages staged per round
@@ -326,14 +256,19 @@ __device__ __forceinline__ void block_sum3(double& x, double& y, double& z, doub
   }
 }
 
+constexpr int kTauCand = 4096;
+
 template <int VPT>
 __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
+  grid_dep_enter();
   const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int tid = threadIdx.x, nt = blockDim.x;
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
   __shared__ float f_scratch[32];
   __shared__ double d_scratch[3 * 32];
   __shared__ int i_scratch[32];
   __shared__ int hist[kTauBins];
+  __shared__ float cand[kTauCand];
+  __shared__ double s_tau;
   int L;
   const int P = seq_pages(a.seq_lens, b, a.S, a.max_pages, &L);
   const int n = unit_slots(a, unit, P) * a.S;
@@ -352,7 +287,7 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
     const int i = tid + k * nt;
     uv[k] = (VPT > 0 && i < n) ? am1 * z[i] : -INFINITY;
   }
-  // applies fn(u) to every value of the row
+  // applies fn(u) to every value of the row (registers, or a pass over the scratch)
   auto for_values = [&](auto fn) {
     if constexpr (VPT > 0) {
 #pragma unroll
@@ -365,26 +300,40 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
   float tau_f = INFINITY;  // no token: no support, zero output
   if (n > 0 && m > -INFINITY) {
     const float um = am1 * m;
-    // lower bracket from the histogram of u over (um − 1, um]
+    // 1. lower bracket from the histogram of u over (um − 1, um]
     for (int i = tid; i < kTauBins; i += nt) hist[i] = 0;
     __syncthreads();
     for_values([&](float u) {
       if (u > um - 1.0f) atomicAdd(&hist[min(kTauBins - 1, static_cast<int>((um - u) * kTauBins))], 1);
     });
     __syncthreads();
-    float cand = um - 1.0f;
-    if (tid < kTauBins) {
-      int c = 0;  // values in bins 0..tid (u above the edge um − (tid+1)/bins, up to rounding)
-      for (int j = 0; j <= tid; ++j) c += hist[j];
-      if (c > 0)
-        cand = fmaxf(cand, um - static_cast<float>(tid + 1) / kTauBins - powf(static_cast<float>(c), -1.0f / beta));
+    float cb = um - 1.0f;
+    {
+      const int h = tid < kTauBins ? hist[tid] : 0;
+      int total;
+      const int c = block_exclusive_scan(h, i_scratch, &total) + h;  // values in bins 0..tid
+      if (tid < kTauBins && c > 0)
+        cb = fmaxf(cb, um - static_cast<float>(tid + 1) / kTauBins - powf(static_cast<float>(c), -1.0f / beta));
     }
-    cand = block_reduce(cand, f_scratch, [](float x, float y) { return fmaxf(x, y); });
-    double tau = static_cast<double>(cand) - 1e-6 * (1.0 + fabs(static_cast<double>(um)));
-    for (int it = 0; it < 100; ++it) {
-      double f = 0.0, df = 0.0, unused = 0.0;
+    cb = block_reduce(cb, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+    const double tau_lo = static_cast<double>(cb) - 1e-6 * (1.0 + fabs(static_cast<double>(um)));
+    // 2. τ only rises from tau_lo, so only values above it can ever count:
+    //    compact them (block-scan order, deterministic) and iterate on those
+    int mine = 0;
+    for_values([&](float u) { mine += static_cast<double>(u) > tau_lo ? 1 : 0; });
+    int nc;
+    int pos = block_exclusive_scan(mine, i_scratch, &nc);
+    const bool fits = nc <= kTauCand;
+    if (fits)
       for_values([&](float u) {
-        const double w = static_cast<double>(u) - tau;
+        if (static_cast<double>(u) > tau_lo) cand[pos++] = u;
+      });
+    __syncthreads();
+    auto sums = [&](double t, double& f, double& df, bool block) {
+      f = 0.0;
+      df = 0.0;
+      auto term = [&](float u) {
+        const double w = static_cast<double>(u) - t;
         if (w > 0.0) {
           if (ib == 1) {
             f += w;
@@ -398,43 +347,76 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
             df += wb1;
           }
         }
-      });
-      block_sum3(f, df, unused, d_scratch);
-      if (it == 0 && f < 1.0) {  // bracket missed (rounding): restart from max u − 1
-        tau = static_cast<double>(um) - 1.0;
-        continue;
+      };
+      if (fits) {
+        for (int i = block ? tid : lane; i < nc; i += block ? nt : 32) term(cand[i]);
+      } else {
+        for_values(term);
       }
-      const double step = (f - 1.0) / (static_cast<double>(beta) * df);
-      if (!(step > 0.0)) break;
-      tau += step;
-      if (step <= 1e-11 * fmax(1.0, fabs(tau))) break;
-    }
-    if (ib == 1 || ib == 2) {
-      // closed form on the support found: β = 1: τ = (Σu − 1)/k;
-      // β = 2: τ = M − √(M² − Q + 1/k) with M, Q the mean and mean square
-      for (int rep = 0; rep < 4; ++rep) {
-        double c = 0.0, s1 = 0.0, s2 = 0.0;
-        for_values([&](float u) {
-          if (static_cast<double>(u) > tau) {
-            c += 1.0;
-            s1 += u;
-            s2 += static_cast<double>(u) * u;
-          }
-        });
-        block_sum3(c, s1, s2, d_scratch);
-        if (c < 1.0) break;
-        double t_new;
-        if (ib == 1) {
-          t_new = (s1 - 1.0) / c;
-        } else {
-          const double M = s1 / c, Q = s2 / c;
-          t_new = M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
+      if (block) {
+        double unused = 0.0;
+        block_sum3(f, df, unused, d_scratch);
+      } else {
+        f = warp_sum(f);
+        df = warp_sum(df);
+      }
+    };
+    // one warp iterates when the candidates are few (no block barriers)
+    const bool solo = fits && nc <= 1024;
+    if (!solo || warp == 0) {
+      double tau = tau_lo;
+      for (int it = 0; it < 100; ++it) {
+        double f, df;
+        sums(tau, f, df, !solo);
+        if (it == 0 && f < 1.0) {  // bracket missed (rounding): restart from max u − 1
+          tau = static_cast<double>(um) - 1.0;
+          continue;
         }
-        if (t_new == tau) break;
-        tau = t_new;
+        const double step = (f - 1.0) / (static_cast<double>(beta) * df);
+        if (!(step > 0.0)) break;
+        tau += step;
+        if (step <= 1e-11 * fmax(1.0, fabs(tau))) break;
       }
+      if (ib == 1 || ib == 2) {
+        // closed form on the support found: β = 1: τ = (Σu − 1)/k;
+        // β = 2: τ = M − √(M² − Q + 1/k) with M, Q the mean and mean square
+        for (int rep = 0; rep < 4; ++rep) {
+          double c = 0.0, s1 = 0.0, s2 = 0.0;
+          auto add = [&](float u) {
+            if (static_cast<double>(u) > tau) {
+              c += 1.0;
+              s1 += u;
+              s2 += static_cast<double>(u) * u;
+            }
+          };
+          if (fits) {
+            for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : nt) add(cand[i]);
+          } else {
+            for_values(add);
+          }
+          if (solo) {
+            c = warp_sum(c);
+            s1 = warp_sum(s1);
+            s2 = warp_sum(s2);
+          } else {
+            block_sum3(c, s1, s2, d_scratch);
+          }
+          if (c < 1.0) break;
+          double t_new;
+          if (ib == 1) {
+            t_new = (s1 - 1.0) / c;
+          } else {
+            const double M = s1 / c, Q = s2 / c;
+            t_new = M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
+          }
+          if (t_new == tau) break;
+          tau = t_new;
+        }
+      }
+      if (tid == 0) s_tau = tau;
     }
-    tau_f = static_cast<float>(tau);
+    __syncthreads();
+    tau_f = static_cast<float>(s_tau);
   }
 
   // support of this head with the fp32 threshold every later stage uses
@@ -442,10 +424,18 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
   const int words = a.words;
   for (int base = 0; base < (n + nt - 1) / nt * nt; base += nt) {
     const int i = base + tid;
-    const bool in = i < n && am1 * z[i] > tau_f;
+    bool in = false;
+    if constexpr (VPT > 0) {
+      const int k = base / nt;
+#pragma unroll
+      for (int kk = 0; kk < VPT; ++kk)
+        if (kk == k) in = i < n && uv[kk] > tau_f;
+    } else {
+      in = i < n && am1 * z[i] > tau_f;
+    }
     cnt += in ? 1 : 0;
     const unsigned int bal = __ballot_sync(0xffffffffu, in);
-    if (a.bits_out && (tid & 31) == 0 && (i >> 5) < words) a.bits_out[orow * words + (i >> 5)] = bal;
+    if (a.bits_out && lane == 0 && (i >> 5) < words) a.bits_out[orow * words + (i >> 5)] = bal;
   }
   cnt = block_reduce(cnt, i_scratch, [](int x, int y) { return x + y; });
   if (a.bits_out)
@@ -462,10 +452,11 @@ constexpr int kPvWarps = 8;
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
+  grid_dep_enter();
   constexpr int DPL = D / 32;  // output columns per lane
   extern __shared__ __align__(16) float red[];  // [kPvWarps][G][D]
   __shared__ float s_tau[G];
-  __shared__ int s_list[32 * kPvWarps];
+  __shared__ int s_list[32 * kPvWarps], s_phys[32 * kPvWarps], s_nv[32 * kPvWarps];
   __shared__ int scan_scratch[32];
   __shared__ int s_last;
 
@@ -486,10 +477,12 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
   const size_t zrow = static_cast<size_t>(a.cap) * S;
 
   for (int w0 = s0; w0 < s1; w0 += blockDim.x) {
-    // the window's pages that hold support, in ascending order
+    // the window's pages that hold support, in ascending order; each thread
+    // resolves its slot's page id in the same pass as the support test
     const int slot = w0 + tid;
-    int sup = 0;
+    int sup = 0, phys = -1, nv = 0;
     if (slot < s1) {
+      phys = slot_page(a, unit, b, slot, P, L, &nv);
       if (a.dense_v) {
         sup = 1;
       } else {
@@ -497,33 +490,35 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
         for (int h = 0; h < G; ++h)
           if (a.am1 * a.ws.pmax[(static_cast<size_t>(unit) * G + h) * a.cap + slot] > s_tau[h]) sup = 1;
       }
+      if (phys < 0) sup = 0;
     }
     int nsup;
     const int pos = block_exclusive_scan(sup, scan_scratch, &nsup);
-    if (sup) s_list[pos] = slot;
+    if (sup) {
+      s_list[pos] = slot;
+      s_phys[pos] = phys;
+      s_nv[pos] = nv;
+    }
     __syncthreads();
     for (int e = warp; e < nsup; e += kPvWarps) {
-      const int sl = s_list[e];
-      int nv;
-      const int phys = slot_page(a, unit, b, sl, P, L, &nv);
-      if (phys < 0) continue;
-      // p of token `lane` for every head
+      const int sl = s_list[e], ph = s_phys[e], nvv = s_nv[e];
+      // V rows and p of token `lane` for every head are independent loads
+      const T* vb = static_cast<const T*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * S * D + lane * DPL;
       float p[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         p[h] = 0.f;
-        if (lane < nv) {
+        if (lane < nvv) {
           const float w = a.am1 * a.ws.zbuf[(static_cast<size_t>(unit) * G + h) * zrow + static_cast<size_t>(sl) * S + lane] - s_tau[h];
-          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ibeta);
+          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ipow);
         }
       }
-      const T* vb = static_cast<const T*>(a.v_pool) + (static_cast<size_t>(phys) * a.Hkv + kvh) * S * D + lane * DPL;
-      for (int t0 = 0; t0 < nv; t0 += 8) {
+      for (int t0 = 0; t0 < nvv; t0 += 8) {
         float vv[8][DPL];
 #pragma unroll
         for (int tt = 0; tt < 8; ++tt) {
           const int t = t0 + tt;
-          if (t < nv) {
+          if (t < nvv) {
             if constexpr (DPL == 4) {
               load4(vb + static_cast<size_t>(t) * D, vv[tt]);
             } else {
@@ -540,9 +535,9 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
         for (int tt = 0; tt < 8; ++tt) {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float ph = __shfl_sync(0xffffffffu, p[h], (t0 + tt) & 31);
+            const float ph_t = __shfl_sync(0xffffffffu, p[h], (t0 + tt) & 31);
 #pragma unroll
-            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(ph, vv[tt][e2], acc[h][e2]);
+            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(ph_t, vv[tt][e2], acc[h][e2]);
           }
         }
       }
@@ -586,24 +581,39 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
   cudaError_t e;
   const dim3 gq(static_cast<unsigned>(a.ws.nqk), static_cast<unsigned>(U));
   if constexpr (sizeof(T) == 2) {
-    qk_mma_kernel<D, G><<<gq, 32 * kQkWarps, 0, st>>>(a);
+    {
+    const cudaError_t le_ = launch_k(qk_mma_kernel<D, G>, gq, 32 * kQkWarps, 0, st, a);
+    if (le_ != cudaSuccess) return le_;
+  }
   } else {
     const size_t smem = static_cast<size_t>(G) * D * sizeof(float) + 4 * static_cast<size_t>(a.S) * (D + 16 / sizeof(T)) * sizeof(T);
     if (smem > 48 * 1024) {
       e = cudaFuncSetAttribute(qk_cc_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
     }
-    qk_cc_kernel<T, D, G><<<gq, 256, smem, st>>>(a);
+    {
+    const cudaError_t le_ = launch_k(qk_cc_kernel<T, D, G>, gq, 256, smem, st, a);
+    if (le_ != cudaSuccess) return le_;
+  }
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_max = a.cap * a.S;
   if (n_max <= 16 * kTauThreads)
-    tau_kernel<16><<<U * G, kTauThreads, 0, st>>>(a, G);
+    {
+    const cudaError_t le_ = launch_k(tau_kernel<16>, U * G, kTauThreads, 0, st, a, G);
+    if (le_ != cudaSuccess) return le_;
+  }
   else if (n_max <= 64 * kTauThreads)
-    tau_kernel<64><<<U * G, kTauThreads, 0, st>>>(a, G);
+    {
+    const cudaError_t le_ = launch_k(tau_kernel<64>, U * G, kTauThreads, 0, st, a, G);
+    if (le_ != cudaSuccess) return le_;
+  }
   else
-    tau_kernel<0><<<U * G, kTauThreads, 0, st>>>(a, G);
+    {
+    const cudaError_t le_ = launch_k(tau_kernel<0>, U * G, kTauThreads, 0, st, a, G);
+    if (le_ != cudaSuccess) return le_;
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t pv_smem = static_cast<size_t>(kPvWarps) * G * D * sizeof(float);
@@ -612,7 +622,10 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   const dim3 gp(static_cast<unsigned>(a.ws.npv), static_cast<unsigned>(U));
-  pv_kernel<T, D, G><<<gp, 32 * kPvWarps, pv_smem, st>>>(a);
+  {
+    const cudaError_t le_ = launch_k(pv_kernel<T, D, G>, gp, 32 * kPvWarps, pv_smem, st, a);
+    if (le_ != cudaSuccess) return le_;
+  }
   return cudaGetLastError();
 }
 
@@ -639,6 +652,10 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
   a.am1 = alpha - 1.0f;
   a.beta = static_cast<float>(1.0 / (static_cast<double>(alpha) - 1.0));
   a.ibeta = (alpha == 2.0f) ? 1 : (alpha == 1.5f ? 2 : 0);
+  {
+    const double bd = 1.0 / (static_cast<double>(alpha) - 1.0);
+    a.ipow = (bd == 1.0 || bd == 2.0 || bd == 3.0 || bd == 4.0) ? static_cast<int>(bd) : 0;
+  }
   a.Hkv = c.num_kv_heads;
   a.Hq = Hq;
   a.S = c.page_size;
@@ -651,11 +668,17 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
   const int G = Hq / c.num_kv_heads, U = s.batch * c.num_kv_heads;
 #define EKV_DEC_CASE(TT, DD, GG) \
   if (c.head_dim == DD && G == GG) return run_decode<TT, DD, GG>(a, U, st);
+#define EKV_DEC_BF16(DD, GG)                                                         \
+  if (c.head_dim == DD && G == GG) {                                                 \
+    if (U <= 65535 && fused_decode_fits<DD, GG>(U, cap, c.page_size))                \
+      return run_fused_decode<DD, GG>(a, U, st);                                     \
+    return run_decode<bf16, DD, GG>(a, U, st);                                       \
+  }
   if (c.dtype == EKV_BF16) {
-    EKV_DEC_CASE(bf16, 128, 1) EKV_DEC_CASE(bf16, 128, 2) EKV_DEC_CASE(bf16, 128, 4)
-    EKV_DEC_CASE(bf16, 128, 8) EKV_DEC_CASE(bf16, 128, 16)
-    EKV_DEC_CASE(bf16, 64, 1) EKV_DEC_CASE(bf16, 64, 2) EKV_DEC_CASE(bf16, 64, 4)
-    EKV_DEC_CASE(bf16, 64, 8) EKV_DEC_CASE(bf16, 64, 16)
+    EKV_DEC_BF16(128, 1) EKV_DEC_BF16(128, 2) EKV_DEC_BF16(128, 4)
+    EKV_DEC_BF16(128, 8) EKV_DEC_BF16(128, 16)
+    EKV_DEC_BF16(64, 1) EKV_DEC_BF16(64, 2) EKV_DEC_BF16(64, 4)
+    EKV_DEC_BF16(64, 8) EKV_DEC_BF16(64, 16)
   } else {
     EKV_DEC_CASE(float, 128, 1) EKV_DEC_CASE(float, 128, 2) EKV_DEC_CASE(float, 128, 4)
     EKV_DEC_CASE(float, 128, 8) EKV_DEC_CASE(float, 128, 16)
@@ -663,6 +686,7 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
     EKV_DEC_CASE(float, 64, 8) EKV_DEC_CASE(float, 64, 16)
   }
 #undef EKV_DEC_CASE
+#undef EKV_DEC_BF16
   return cudaErrorInvalidValue;
 }
 

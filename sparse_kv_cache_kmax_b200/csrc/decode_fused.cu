@@ -1,0 +1,743 @@
+// Sparse α-entmax decode over the selected pages, one thread-block cluster
+// per (sequence, KV head) — EntmaxKV summary page (gist.science/fr/paper/
+// 2605.21649) §2.C "Attention Entmax Parcimonieuse", with the support-only V
+// read that §2–§3 make exact.
+//
+// The unit's selected pages are split into C equal runs, one per CTA of the
+// cluster (C ≤ 16, chosen so that all units' clusters are resident at once).
+// Each CTA works in four phases separated by cluster barriers:
+//  1. K: every warp streams its own pages (page j of the run goes to warp
+//     j mod 16) through a private ring of shared-memory slots filled by 1-D
+//     bulk async copies (one copy = one contiguous S×d K tile), then scores
+//     them on tensor cores (m16n8k16, rows of the tile loaded from shared
+//     memory straight into A fragments).  Scores z and page maxima stay in
+//     shared memory.
+//  2. τ: query head h is solved by CTA h mod C, which gathers the head's
+//     scores of the whole unit from the cluster's shared memory (DSMEM) in
+//     token order and solves Σ[u − τ]_+^β = 1, u = (α−1)·z, β = 1/(α−1):
+//     a histogram bracket over (max u − 1, max u], Newton's method from the
+//     left on the values above the bracket, and for β ∈ {1,2} the closed form
+//     on the support found.  τ goes to every CTA of the cluster.
+//  3. V: each CTA lists the pages of its run holding a support token
+//     (some head has a page maximum above τ) and its warps read only those V
+//     rows; p = [u − τ]_+^β comes from the scores in shared memory.  The
+//     support bits and counts of the run's tokens are written alongside.
+//  4. The CTA partial outputs are summed across the cluster in rank order,
+//     CTA r owning a 1/C slice of the unit's G×d outputs.
+// Every sum has a fixed order, so results are deterministic.
+#include <cooperative_groups.h>
+
+#include <mutex>
+#include <vector>
+
+#include "decode.cuh"
+
+namespace ekv {
+
+namespace {
+
+namespace cg = cooperative_groups;
+
+constexpr int kFWarps = 16;
+constexpr int kFThreads = 32 * kFWarps;
+constexpr int kFMaxCluster = 16;
+constexpr int kFMaxSpw = 8;                   // ring slots per warp
+constexpr int kTauBinsF = 256;
+
+struct FusedGeom {
+  int C;          // CTAs per unit (cluster size)
+  int spc;        // selected slots per CTA
+  int zpitch;     // floats per head row of the score array (spc·S + 4)
+  int spw;        // ring slots per warp
+  int tile_bytes; // bytes of one S×d K or V tile
+  int off_ints, off_pm, off_zs, off_out, off_ring;  // byte offsets in dynamic shared memory
+  int smem;       // dynamic shared memory bytes
+};
+
+struct TauShared {
+  float f[2][kFWarps];   // fp32 partials, double-buffered: one barrier per reduction
+  float f2[2][kFWarps];
+  double d[3][kFWarps];  // fp64 partials
+  int i[32];
+  int hist[kTauBinsF];
+  float m;
+  double tau;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, unsigned int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Pairwise sum of the 16 per-warp partials (a fixed tree, so every thread
+// computes the same value).
+template <typename V>
+__device__ __forceinline__ V tree16(const V* p) {
+  const V a0 = (p[0] + p[1]) + (p[2] + p[3]), a1 = (p[4] + p[5]) + (p[6] + p[7]);
+  const V a2 = (p[8] + p[9]) + (p[10] + p[11]), a3 = (p[12] + p[13]) + (p[14] + p[15]);
+  return (a0 + a1) + (a2 + a3);
+}
+static_assert(kFWarps == 16, "tree16 sums one partial per warp");
+
+// w^(β−1) for w > 0 in the precision of w.
+template <typename V>
+__device__ __forceinline__ V pow_bm1(V w, V beta, int ipow) {
+  switch (ipow) {
+    case 1: return V(1);
+    case 2: return w;
+    case 3: return w * w;
+    case 4: return w * w * w;
+    default:
+      if constexpr (sizeof(V) == 8) return pow(w, beta - 1.0);
+      else return powf(w, beta - 1.0f);
+  }
+}
+
+// f(t) = Σ(u − t)_+^β − 1 and f'(t)/(−β) = Σ(u − t)_+^(β−1) over the
+// candidates, by one warp (solo) or by the CTA (one barrier, parity `par`).
+template <typename V>
+__device__ __forceinline__ void f_df(const float* cand, int nc, V t, V beta, int ipow, bool solo,
+                                     TauShared& sh, int par, V& f, V& df) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  V a = V(0), b = V(0);
+  for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
+    const V w = static_cast<V>(cand[i]) - t;
+    if (w > V(0)) {
+      const V wb1 = pow_bm1<V>(w, beta, ipow);
+      a += wb1 * w;
+      b += wb1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if (!solo) {
+    if constexpr (sizeof(V) == 4) {
+      if (lane == 0) {
+        sh.f[par][warp] = a;
+        sh.f2[par][warp] = b;
+      }
+      __syncthreads();
+      a = tree16(sh.f[par]);
+      b = tree16(sh.f2[par]);
+    } else {
+      if (lane == 0) {
+        sh.d[par][warp] = a;
+        sh.d[2][warp] = b;
+      }
+      __syncthreads();
+      a = tree16(sh.d[par]);
+      b = tree16(sh.d[2]);
+    }
+  }
+  f = a - V(1);
+  df = b;
+}
+
+// τ of one query head: Σ_i [u_i − τ]_+^β = 1, u_i = (α−1)·z_i, over the n
+// scores z[0..n) in shared memory (m = their maximum, finite); the whole CTA
+// calls it with sh.hist zeroed.  cand: shared scratch of n floats.
+//  1. Bracket: a histogram of u over (max u − 1, max u]; c values above an
+//     edge e force τ ≥ e − c^(−1/β).
+//  2. The values above the bracket are compacted in scan order.
+//  3. Newton's method from the left in fp32 (f is convex and decreasing),
+//     then float64: for β ∈ {1,2} the closed form on the support found
+//     (β = 1: τ = (Σu − 1)/k; β = 2: τ = M − √(M² − Q + 1/k) with M, Q the
+//     support's mean and mean square), repeated until the support is stable;
+//     otherwise one float64 Newton step.
+// Returns the fp32 τ every later step uses.
+__device__ float cta_solve_tau(const float* z, int n, float m, float* cand, float am1, float beta,
+                               int ib, int ipow, TauShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float um = am1 * m;
+  for (int i = tid; i < n; i += kFThreads) {
+    const float u = am1 * z[i];
+    if (u > um - 1.0f) atomicAdd(&sh.hist[min(kTauBinsF - 1, static_cast<int>((um - u) * kTauBinsF))], 1);
+  }
+  __syncthreads();
+  float cb = um - 1.0f;
+  {
+    const int h = tid < kTauBinsF ? sh.hist[tid] : 0;
+    int total;
+    const int c = block_exclusive_scan(h, sh.i, &total) + h;
+    if (tid < kTauBinsF && c > 0)
+      cb = fmaxf(cb, um - static_cast<float>(tid + 1) / kTauBinsF - powf(static_cast<float>(c), -1.0f / beta));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cb = fmaxf(cb, __shfl_xor_sync(0xffffffffu, cb, o));
+  if (lane == 0) sh.f[0][warp] = cb;
+  __syncthreads();
+  cb = sh.f[0][0];
+#pragma unroll
+  for (int w = 1; w < kFWarps; ++w) cb = fmaxf(cb, sh.f[0][w]);
+  const double tau_lo = static_cast<double>(cb) - 1e-6 * (1.0 + fabs(static_cast<double>(um)));
+  int mine = 0;
+  for (int i = tid; i < n; i += kFThreads) mine += static_cast<double>(am1 * z[i]) > tau_lo ? 1 : 0;
+  int nc;
+  int pos = block_exclusive_scan(mine, sh.i, &nc);
+  for (int i = tid; i < n; i += kFThreads) {
+    const float u = am1 * z[i];
+    if (static_cast<double>(u) > tau_lo) cand[pos++] = u;
+  }
+  __syncthreads();
+  const bool solo = nc <= 1024;
+  if (!solo || warp == 0) {
+    // fp32 Newton from the left
+    float t = static_cast<float>(tau_lo);
+    if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
+    int par = 1;
+    for (int it = 0; it < 64; ++it) {
+      float f, df;
+      par ^= 1;
+      f_df<float>(cand, nc, t, beta, ipow, solo, sh, par, f, df);
+      if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
+        t = um - 1.0f;
+        continue;
+      }
+      const float step = f / (beta * df);
+      if (!(step > 0.0f)) break;
+      t += step;
+      if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+    }
+    // float64 finish
+    double tau = t;
+    if (ib == 1 || ib == 2) {
+      for (int rep = 0; rep < 4; ++rep) {
+        double c = 0.0, s1 = 0.0, s2 = 0.0;
+        for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
+          const double u = cand[i];
+          if (u > tau) {
+            c += 1.0;
+            s1 += u;
+            s2 += u * u;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+          s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        }
+        if (!solo) {
+          if (lane == 0) {
+            sh.d[0][warp] = c;
+            sh.d[1][warp] = s1;
+            sh.d[2][warp] = s2;
+          }
+          __syncthreads();
+          c = tree16(sh.d[0]);
+          s1 = tree16(sh.d[1]);
+          s2 = tree16(sh.d[2]);
+          __syncthreads();
+        }
+        if (c < 1.0) break;
+        double t_new;
+        if (ib == 1) {
+          t_new = (s1 - 1.0) / c;
+        } else {
+          const double M = s1 / c, Q = s2 / c;
+          t_new = M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
+        }
+        if (t_new == tau) break;
+        tau = t_new;
+      }
+    } else {
+      double f, df;
+      f_df<double>(cand, nc, tau, static_cast<double>(beta), ipow, solo, sh, 0, f, df);
+      if (df > 0.0) tau += f / (static_cast<double>(beta) * df);
+    }
+    if (tid == 0) sh.tau = tau;
+  }
+  __syncthreads();
+  return static_cast<float>(sh.tau);
+}
+
+// Four (D = 128) or two (D = 64) consecutive bf16 of a V row as fp32.
+template <int DPL>
+__device__ __forceinline__ void load_v(const bf16* p, float (&v)[DPL]) {
+  if constexpr (DPL == 4) {
+    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(w.x << 16);
+    v[1] = __uint_as_float(w.x & 0xffff0000u);
+    v[2] = __uint_as_float(w.y << 16);
+    v[3] = __uint_as_float(w.y & 0xffff0000u);
+  } else {
+    const uint32_t w = __ldcs(reinterpret_cast<const unsigned int*>(p));
+    v[0] = __uint_as_float(w << 16);
+    v[1] = __uint_as_float(w & 0xffff0000u);
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a, FusedGeom f) {
+  constexpr int KP = D / 32, NT = (G + 7) / 8, DPL = D / 32;
+  constexpr int VCH = G >= 8 ? 8 : 16;  // V rows in flight per warp
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint64_t bars[kFWarps * kFMaxSpw];
+  __shared__ TauShared tsh;
+  __shared__ float s_tau[G];
+  __shared__ float s_mloc[G];
+  __shared__ int scan_scratch[32];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int C = f.C;
+  const int unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  const int S = a.S, spc = f.spc, zp = f.zpitch, spw = f.spw;
+  int* phys_s = reinterpret_cast<int*>(smem + f.off_ints);  // [spc]
+  int* nv_s = phys_s + spc;                                  // [spc]
+  int* list_s = nv_s + spc;                                  // [spc]
+  float* pm = reinterpret_cast<float*>(smem + f.off_pm);     // [G][spc] page maxima of z
+  float* zs = reinterpret_cast<float*>(smem + f.off_zs);     // [G][zpitch] scores z
+  float* out_s = reinterpret_cast<float*>(smem + f.off_out); // [G][D] CTA partial output
+  unsigned char* ring = smem + f.off_ring;
+
+  if (tid == 0) {
+    for (int s = 0; s < kFWarps * spw; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dep_enter();
+  int L;
+  const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
+  const int n_slots = unit_slots(a, unit, P);
+  const int s0 = rank * spc;
+  const int np = max(0, min(spc, n_slots - s0));
+
+  // ---------------------------------------------------------------- 1. K
+  // Warp w owns pages w, w+16, ... of the run: its lanes resolve them, and
+  // the lanes of its first spw pages start their copies at once.
+  const int cnt_w = warp < np ? (np - warp + kFWarps - 1) / kFWarps : 0;
+  const size_t tile_elems = static_cast<size_t>(S) * D;
+  auto issue = [&](int i, int ph) {  // page i of this warp into its slot
+    uint64_t* bar = &bars[warp * spw + i % spw];
+    if (ph < 0) {
+      mbar_arrive(bar);  // nothing to copy: complete the phase
+      return;
+    }
+    mbar_arrive_expect_tx(bar, static_cast<unsigned int>(f.tile_bytes));
+    const bf16* src = static_cast<const bf16*>(a.k_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems;
+    bulk_g2s(ring + static_cast<size_t>(warp * spw + i % spw) * f.tile_bytes, src,
+             static_cast<unsigned int>(f.tile_bytes), bar);
+  };
+  for (int i = lane; i < cnt_w; i += 32) {
+    const int j = warp + i * kFWarps;
+    int nv;
+    const int ph = slot_page(a, unit, b, s0 + j, P, L, &nv);
+    phys_s[j] = ph;
+    nv_s[j] = nv;
+    if (i < spw) issue(i, ph);
+  }
+  __syncwarp();
+  uint32_t bfrag[2 * KP][NT][2];
+  load_q_frags<D, G>(a, b, kvh, g, t, bfrag);
+
+  for (int i = 0; i < cnt_w; ++i) {
+    const int j = warp + i * kFWarps, sl = warp * spw + i % spw;
+    const unsigned int parity = static_cast<unsigned int>(i / spw) & 1u;
+    if (!mbar_wait(&bars[sl], parity)) mbar_wait(&bars[sl], parity);  // second bounded wait: no copy left in flight
+    const unsigned char* tile = ring + static_cast<size_t>(sl) * f.tile_bytes;
+    const int nv = phys_s[j] < 0 ? 0 : nv_s[j];
+    float pmx[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) pmx[nt][0] = pmx[nt][1] = -INFINITY;
+    for (int mt = 0; mt < S / 16; ++mt) {
+      const int tok0 = mt * 16;
+      const uint4* rlo = reinterpret_cast<const uint4*>(tile + static_cast<size_t>(tok0 + g) * D * 2) + t;
+      const uint4* rhi = reinterpret_cast<const uint4*>(tile + static_cast<size_t>(tok0 + g + 8) * D * 2) + t;
+      uint4 va[KP], vb[KP];
+#pragma unroll
+      for (int c = 0; c < KP; ++c) {
+        va[c] = rlo[4 * c];
+        vb[c] = rhi[4 * c];
+      }
+      float acc[NT][4];
+      score_mtile<D, G>(va, vb, bfrag, acc);
+      const bool ok_lo = tok0 + g < nv, ok_hi = tok0 + g + 8 < nv;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hd = nt * 8 + 2 * t + e;
+          const float zl = ok_lo ? a.scale * acc[nt][e] : -INFINITY;
+          const float zh = ok_hi ? a.scale * acc[nt][2 + e] : -INFINITY;
+          if (hd < G) {
+            float* zr = zs + hd * zp + j * S + tok0;
+            zr[g] = zl;
+            zr[g + 8] = zh;
+          }
+          float m = fmaxf(zl, zh);
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+          pmx[nt][e] = fmaxf(pmx[nt][e], m);
+        }
+    }
+    if (g == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hd = nt * 8 + 2 * t + e;
+          if (hd < G) pm[hd * spc + j] = pmx[nt][e];
+        }
+    }
+    __syncwarp();
+    if (lane == 0 && i + spw < cnt_w) {
+      fence_proxy_async_smem();  // the slot's reads come before the copy that refills it
+      issue(i + spw, phys_s[warp + (i + spw) * kFWarps]);
+    }
+  }
+  __syncthreads();
+  // V tiles of the pages that can hold support (a page maximum within 1 of
+  // this run's maximum, in u) start moving to L2 while τ is solved
+  if (!a.dense_v) {
+    for (int h = warp; h < G; h += kFWarps) {
+      float m = -INFINITY;
+      for (int j = lane; j < np; j += 32) m = fmaxf(m, pm[h * spc + j]);
+      m = warp_max(m);
+      if (lane == 0) s_mloc[h] = m;
+    }
+    __syncthreads();
+  }
+  for (int j = tid; j < np; j += kFThreads) {
+    const int ph = phys_s[j];
+    if (ph < 0) continue;
+    bool cand = a.dense_v != 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      if (!cand && pm[h * spc + j] > -INFINITY && a.am1 * pm[h * spc + j] > a.am1 * s_mloc[h] - 1.0f) cand = true;
+    if (cand)
+      prefetch_l2_bulk(static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems,
+                       static_cast<unsigned int>(f.tile_bytes));
+  }
+  cluster.sync();
+
+  // ---------------------------------------------------------------- 2. τ
+  // Head h is solved by CTA h mod C on the unit's scores gathered in token
+  // order; the solver also writes the head's support bits and count.
+  const int tpc = spc * S;
+  const int n_tok = n_slots * S;
+  float* zh = reinterpret_cast<float*>(ring);
+  float* cand = zh + ((n_tok + 31) & ~31);
+  const size_t words = static_cast<size_t>(a.words);
+  for (int h = rank; h < G; h += C) {
+    const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h;
+    for (int i = tid; i < kTauBinsF; i += kFThreads) tsh.hist[i] = 0;
+    float m = -INFINITY;
+    for (int i = 4 * tid; i < n_tok; i += 4 * kFThreads) {
+      const int r = i / tpc;
+      const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(zs, r) + h * zp + (i - r * tpc));
+      *reinterpret_cast<float4*>(zh + i) = v;
+      m = fmaxf(fmaxf(m, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+    }
+    m = warp_max(m);
+    if (lane == 0) tsh.f[0][warp] = m;
+    __syncthreads();
+    m = tsh.f[0][0];
+#pragma unroll
+    for (int w = 1; w < kFWarps; ++w) m = fmaxf(m, tsh.f[0][w]);
+    float tau = INFINITY;  // no finite score: no support, zero output
+    if (m > -INFINITY) tau = cta_solve_tau(zh, n_tok, m, cand, a.am1, a.beta, a.ibeta, a.ipow, tsh);
+    if (tid < C) cluster.map_shared_rank(s_tau, tid)[h] = tau;
+    if (tid == 0 && a.tau_out) a.tau_out[orow] = tau;
+    int cnt = 0;
+    for (int base = 0; base < n_tok; base += kFThreads) {
+      const int i = base + tid;
+      const bool in = i < n_tok && a.am1 * zh[i] > tau;
+      cnt += in ? 1 : 0;
+      const unsigned int bal = __ballot_sync(0xffffffffu, in);
+      if (a.bits_out && lane == 0 && i < n_tok) a.bits_out[orow * words + i / 32] = bal;
+    }
+    if (a.bits_out)
+      for (int w = (n_tok + 31) / 32 + tid; w < a.words; w += kFThreads) a.bits_out[orow * words + w] = 0u;
+    cnt = warp_sum(cnt);
+    __syncthreads();  // tsh.i and zh are free again after this
+    if (lane == 0) tsh.i[warp] = cnt;
+    __syncthreads();
+    if (tid == 0 && a.count_out) {
+      int c = 0;
+      for (int w = 0; w < kFWarps; ++w) c += tsh.i[w];
+      a.count_out[orow] = c;
+    }
+  }
+  cluster.sync();
+
+  // ---------------------------------------------------------------- 3. V
+  int nsup = 0;
+  for (int w0 = 0; w0 < np; w0 += kFThreads) {
+    const int j = w0 + tid;
+    int sup = 0;
+    if (j < np && phys_s[j] >= 0) {
+      if (a.dense_v) {
+        sup = 1;
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          if (a.am1 * pm[h * spc + j] > s_tau[h]) sup = 1;
+      }
+    }
+    int tot;
+    const int pos = block_exclusive_scan(sup, scan_scratch, &tot);
+    if (sup) list_s[nsup + pos] = j;
+    nsup += tot;
+  }
+  __syncthreads();
+
+  float acc[G][DPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+  for (int e = warp; e < nsup; e += kFWarps) {
+    const int j = list_s[e], ph = phys_s[j], nvv = nv_s[j];
+    const bf16* vrow = static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems + lane * DPL;
+    for (int t0 = 0; t0 < nvv; t0 += 32) {
+      float p[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        p[h] = 0.f;
+        if (t0 + lane < nvv) {
+          const float w = a.am1 * zs[h * zp + j * S + t0 + lane] - s_tau[h];
+          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ipow);
+        }
+      }
+      const int nt32 = min(32, nvv - t0);
+      for (int t1 = 0; t1 < nt32; t1 += VCH) {
+        float vv[VCH][DPL];
+#pragma unroll
+        for (int tt = 0; tt < VCH; ++tt) {
+          if (t1 + tt < nt32) {
+            load_v<DPL>(vrow + static_cast<size_t>(t0 + t1 + tt) * D, vv[tt]);
+          } else {
+#pragma unroll
+            for (int e2 = 0; e2 < DPL; ++e2) vv[tt][e2] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int tt = 0; tt < VCH; ++tt) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pt = __shfl_sync(0xffffffffu, p[h], (t1 + tt) & 31);
+#pragma unroll
+            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(pt, vv[tt][e2], acc[h][e2]);
+          }
+        }
+      }
+    }
+  }
+  // warp partials → CTA partial (warp order)
+  float* red = reinterpret_cast<float*>(ring);  // [kFWarps][G][D]
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) red[(warp * G + h) * D + lane * DPL + e] = acc[h][e];
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kFThreads) {
+    float pw[kFWarps];
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) pw[w] = red[w * G * D + i];
+    out_s[i] = tree16(pw);
+  }
+  cluster.sync();
+
+  // ---------------------------------------------------------------- 4. cluster sum
+  const int GD = G * D, chunk = (GD + C - 1) / C;
+  const int i_end = min(GD, (rank + 1) * chunk);
+  for (int i = rank * chunk + tid; i < i_end; i += kFThreads) {
+    float s = 0.f;
+    for (int r = 0; r < C; ++r) s += cluster.map_shared_rank(out_s, r)[i];
+    const int h = i / D, d = i - h * D;
+    a.out[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h) * D + d] = s;
+  }
+  cluster.sync();  // no CTA leaves while another still reads its shared memory
+}
+
+// ------------------------------------------------------------------ host side
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+struct DeviceLimits {
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+DeviceLimits device_limits() {
+  static std::mutex mu;
+  static std::vector<DeviceLimits> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  DeviceLimits& l = cache[dev];
+  if (l.sms == 0) {
+    cudaDeviceGetAttribute(&l.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&l.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  }
+  return l;
+}
+
+// Geometry for C CTAs per unit; smem = 0 when it does not fit.
+template <int D, int G>
+FusedGeom plan(int C, int cap, int S, int smem_limit) {
+  FusedGeom f{};
+  f.C = C;
+  f.spc = (cap + C - 1) / C;
+  const int step = S >= 32 ? 1 : 32 / S;  // each CTA's tokens start on a 32-token word
+  f.spc = round_up(f.spc, step);
+  f.zpitch = f.spc * S + 4;
+  f.tile_bytes = S * D * 2;
+  int off = 0;
+  f.off_ints = off;
+  off += round_up(3 * f.spc * 4, 128);
+  f.off_pm = off;
+  off += round_up(G * f.spc * 4, 128);
+  f.off_zs = off;
+  off += round_up(G * f.zpitch * 4, 128);
+  f.off_out = off;
+  off += round_up(G * D * 4, 128);
+  f.off_ring = off;
+  const int n_tok_max = cap * S;
+  const int ring_min = std::max(2 * round_up(n_tok_max, 32) * 4, kFWarps * G * D * 4);
+  const int pages_per_warp = (f.spc + kFWarps - 1) / kFWarps;
+  const int avail = smem_limit - off;
+  int spw = std::min(std::min(pages_per_warp, kFMaxSpw), avail / (kFWarps * f.tile_bytes));
+  if (spw < 1) return FusedGeom{};
+  f.spw = spw;
+  const int ring = std::max(kFWarps * spw * f.tile_bytes, ring_min);
+  if (off + ring > smem_limit) return FusedGeom{};
+  f.smem = off + ring;
+  return f;
+}
+
+template <int D, int G>
+int max_active_clusters(int C, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(C), 1);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fused_decode_kernel<D, G>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int D, int G>
+cudaError_t prepare_kernel(int smem_limit) {
+  static std::mutex mu;
+  static std::vector<char> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (static_cast<int>(done.size()) <= dev) done.resize(dev + 1, 0);
+  if (done[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_limit);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fused_decode_kernel<D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  done[dev] = 1;
+  return cudaSuccess;
+}
+
+// Chosen geometry per (device, units, cap, S): the largest cluster whose
+// clusters for all units are resident together, else one CTA per unit.
+template <int D, int G>
+FusedGeom choose(int units, int cap, int S) {
+  struct Entry {
+    int dev, units, cap, S;
+    FusedGeom f;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> memo;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : memo)
+      if (e.dev == dev && e.units == units && e.cap == cap && e.S == S) return e.f;
+  }
+  const DeviceLimits lim = device_limits();
+  cudaFuncAttributes fa{};
+  FusedGeom best{};
+  const bool have_attr = cudaFuncGetAttributes(&fa, fused_decode_kernel<D, G>) == cudaSuccess;
+  const int smem_limit = lim.smem_optin - static_cast<int>(fa.sharedSizeBytes);
+  if (have_attr && prepare_kernel<D, G>(smem_limit) == cudaSuccess) {
+    for (int C = kFMaxCluster; C >= 1; C >>= 1) {
+      if (C > 1 && (cap + C - 1) / C < 2) continue;
+      const FusedGeom f = plan<D, G>(C, cap, S, smem_limit);
+      if (f.smem == 0) continue;
+      if (C == 1) {
+        best = f;
+        break;
+      }
+      if (max_active_clusters<D, G>(C, f.smem) >= units) {
+        best = f;
+        break;
+      }
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  memo.push_back(Entry{dev, units, cap, S, best});
+  return best;
+}
+
+}  // namespace
+
+template <int D, int G>
+bool fused_decode_fits(int units, int cap, int S) {
+  if (S % 16 != 0 || cap < 1) return false;
+  return choose<D, G>(units, cap, S).smem > 0;
+}
+
+template <int D, int G>
+cudaError_t run_fused_decode(DecodeArgs& a, int units, cudaStream_t st) {
+  const FusedGeom f = choose<D, G>(units, a.cap, a.S);
+  if (f.smem == 0) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(f.C), static_cast<unsigned>(units));
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(f.smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(f.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_decode_kernel<D, G>, a, f);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+#define EKV_FUSED_INST(DD, GG)                                            \
+  template bool fused_decode_fits<DD, GG>(int, int, int);                 \
+  template cudaError_t run_fused_decode<DD, GG>(DecodeArgs&, int, cudaStream_t);
+EKV_FUSED_INST(128, 1)
+EKV_FUSED_INST(128, 2)
+EKV_FUSED_INST(128, 4)
+EKV_FUSED_INST(128, 8)
+EKV_FUSED_INST(128, 16)
+EKV_FUSED_INST(64, 1)
+EKV_FUSED_INST(64, 2)
+EKV_FUSED_INST(64, 4)
+EKV_FUSED_INST(64, 8)
+EKV_FUSED_INST(64, 16)
+#undef EKV_FUSED_INST
+
+}  // namespace ekv

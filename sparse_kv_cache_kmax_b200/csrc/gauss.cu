@@ -79,6 +79,7 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
 __global__ void __launch_bounds__(kGaussThreads)
     gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
                      int Hkv, int G, int Hq, int beta, float* __restrict__ tau_out) {
+  grid_dep_enter();
   const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / Hkv, kvh = unit % Hkv;
   const int tid = threadIdx.x;
   int L;
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kGaussThreads)
     gauss_filter_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
                         int Hkv, int G, double delta, int cap, int32_t* __restrict__ sel,
                         int32_t* __restrict__ n_sel) {
+  grid_dep_enter();
   const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
@@ -251,12 +253,18 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
                                 int32_t* n_sel, float* tau_hat, cudaStream_t st) {
   const int Hkv = c.num_kv_heads, G = Hq / Hkv, U = s.batch * Hkv;
   const int beta = static_cast<int>(lrint(1.0 / (static_cast<double>(alpha) - 1.0)));
-  gauss_tau_kernel<<<U * G, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
+  {
+    const cudaError_t le_ = launch_k(gauss_tau_kernel, U * G, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
                                                     G, Hq, beta, tau_hat);
+    if (le_ != cudaSuccess) return le_;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gauss_filter_kernel<<<U, kGaussThreads, 0, st>>>(ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
+  {
+    const cudaError_t le_ = launch_k(gauss_filter_kernel, U, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
                                                    G, static_cast<double>(delta), cap, sel, n_sel);
+    if (le_ != cudaSuccess) return le_;
+  }
   return cudaGetLastError();
 }
 

@@ -54,43 +54,49 @@ struct Pair<float> {
   }
 };
 
-// Metadata of one coordinate pair over tokens 0..n-1 of a page.  When
-// `inject` ≥ 0, token `inject` takes the values (xa, xb) instead of the pool.
+// Metadata of one coordinate pair over tokens 0..n-1 of a page (n ≤ 32).
+// When `inject` ≥ 0, token `inject` takes the values (xa, xb) instead of the
+// pool.  The page's values are loaded first as one batch of independent loads.
 template <typename T>
 __device__ void page_pair_meta(const T* page_k, int D, int n, int j, int inject, float xa,
                                float xb, T* box_row, T* mom_row) {
+  float va[32], vb[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    va[t] = vb[t] = 0.f;
+    if (t < n) {
+      if (t == inject) {
+        va[t] = xa;
+        vb[t] = xb;
+      } else {
+        Pair<T>::load(page_k + static_cast<size_t>(t) * D + j, va[t], vb[t]);
+      }
+    }
+  }
   float mx0 = -INFINITY, mx1 = -INFINITY, mn0 = INFINITY, mn1 = INFINITY;
   double s0 = 0.0, s1 = 0.0;
-  for (int t = 0; t < n; ++t) {
-    float a, b;
-    if (t == inject) {
-      a = xa;
-      b = xb;
-    } else {
-      Pair<T>::load(page_k + static_cast<size_t>(t) * D + j, a, b);
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    if (t < n) {
+      mx0 = fmaxf(mx0, va[t]);
+      mx1 = fmaxf(mx1, vb[t]);
+      mn0 = fminf(mn0, va[t]);
+      mn1 = fminf(mn1, vb[t]);
+      s0 = __dadd_rn(s0, static_cast<double>(va[t]));
+      s1 = __dadd_rn(s1, static_cast<double>(vb[t]));
     }
-    mx0 = fmaxf(mx0, a);
-    mx1 = fmaxf(mx1, b);
-    mn0 = fminf(mn0, a);
-    mn1 = fminf(mn1, b);
-    s0 = __dadd_rn(s0, static_cast<double>(a));
-    s1 = __dadd_rn(s1, static_cast<double>(b));
   }
   const double dn = static_cast<double>(n);
   const double m0 = __ddiv_rn(s0, dn), m1 = __ddiv_rn(s1, dn);
   double v0 = 0.0, v1 = 0.0;
-  for (int t = 0; t < n; ++t) {
-    float a, b;
-    if (t == inject) {
-      a = xa;
-      b = xb;
-    } else {
-      Pair<T>::load(page_k + static_cast<size_t>(t) * D + j, a, b);
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    if (t < n) {
+      const double d0 = __dsub_rn(static_cast<double>(va[t]), m0);
+      const double d1 = __dsub_rn(static_cast<double>(vb[t]), m1);
+      v0 = __dadd_rn(v0, __dmul_rn(d0, d0));
+      v1 = __dadd_rn(v1, __dmul_rn(d1, d1));
     }
-    const double d0 = __dsub_rn(static_cast<double>(a), m0);
-    const double d1 = __dsub_rn(static_cast<double>(b), m1);
-    v0 = __dadd_rn(v0, __dmul_rn(d0, d0));
-    v1 = __dadd_rn(v1, __dmul_rn(d1, d1));
   }
   Pair<T>::store_exact(box_row + j, mx0, mx1);           // k_max row
   Pair<T>::store_exact(box_row + D + j, mn0, mn1);       // k_min row
@@ -104,6 +110,7 @@ __global__ void build_meta_kernel(const T* __restrict__ k_pool, T* __restrict__ 
                                   T* __restrict__ mom, const int32_t* __restrict__ page_table,
                                   const int32_t* __restrict__ seq_lens, int D, int S, int Hkv,
                                   int num_phys, int max_pages) {
+  grid_dep_enter();
   const int b = blockIdx.y;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
@@ -126,6 +133,7 @@ __global__ void append_kernel(T* __restrict__ k_pool, T* __restrict__ v_pool, T*
                               const int32_t* __restrict__ seq_lens, const T* __restrict__ k_new,
                               const T* __restrict__ v_new, int D, int S, int Hkv, int num_phys,
                               int max_pages) {
+  grid_dep_enter();
   const int b = blockIdx.x;
   int L;
   seq_pages(seq_lens, b, S, max_pages, &L);
@@ -152,15 +160,21 @@ cudaError_t launch_build_meta(const ekv_cache& c, const ekv_seqs& s, cudaStream_
   const dim3 grid(static_cast<unsigned>(min(s.max_pages, 4096)), static_cast<unsigned>(s.batch),
                   static_cast<unsigned>(c.num_kv_heads));
   if (c.dtype == EKV_BF16)
-    build_meta_kernel<bf16><<<grid, threads, 0, st>>>(
+    {
+    const cudaError_t le_ = launch_k(build_meta_kernel<bf16>, grid, threads, 0, st, 
         static_cast<const bf16*>(c.k_pool), static_cast<bf16*>(c.box), static_cast<bf16*>(c.mom),
         s.page_table, s.seq_lens, c.head_dim, c.page_size, c.num_kv_heads, c.num_phys_pages,
         s.max_pages);
+    if (le_ != cudaSuccess) return le_;
+  }
   else
-    build_meta_kernel<float><<<grid, threads, 0, st>>>(
+    {
+    const cudaError_t le_ = launch_k(build_meta_kernel<float>, grid, threads, 0, st, 
         static_cast<const float*>(c.k_pool), static_cast<float*>(c.box),
         static_cast<float*>(c.mom), s.page_table, s.seq_lens, c.head_dim, c.page_size,
         c.num_kv_heads, c.num_phys_pages, s.max_pages);
+    if (le_ != cudaSuccess) return le_;
+  }
   return cudaGetLastError();
 }
 
@@ -169,17 +183,23 @@ cudaError_t launch_append(const ekv_cache& c, const ekv_seqs& s, const void* k_n
   const int threads = c.head_dim / 2;
   const dim3 grid(static_cast<unsigned>(s.batch), static_cast<unsigned>(c.num_kv_heads));
   if (c.dtype == EKV_BF16)
-    append_kernel<bf16><<<grid, threads, 0, st>>>(
+    {
+    const cudaError_t le_ = launch_k(append_kernel<bf16>, grid, threads, 0, st, 
         static_cast<bf16*>(c.k_pool), static_cast<bf16*>(c.v_pool), static_cast<bf16*>(c.box),
         static_cast<bf16*>(c.mom), s.page_table, s.seq_lens, static_cast<const bf16*>(k_new),
         static_cast<const bf16*>(v_new), c.head_dim, c.page_size, c.num_kv_heads,
         c.num_phys_pages, s.max_pages);
+    if (le_ != cudaSuccess) return le_;
+  }
   else
-    append_kernel<float><<<grid, threads, 0, st>>>(
+    {
+    const cudaError_t le_ = launch_k(append_kernel<float>, grid, threads, 0, st, 
         static_cast<float*>(c.k_pool), static_cast<float*>(c.v_pool), static_cast<float*>(c.box),
         static_cast<float*>(c.mom), s.page_table, s.seq_lens, static_cast<const float*>(k_new),
         static_cast<const float*>(v_new), c.head_dim, c.page_size, c.num_kv_heads,
         c.num_phys_pages, s.max_pages);
+    if (le_ != cudaSuccess) return le_;
+  }
   return cudaGetLastError();
 }
 

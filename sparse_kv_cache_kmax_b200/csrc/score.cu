@@ -108,6 +108,7 @@ struct StageRows {
 
 template <typename T, int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) meta_stream_kernel(StreamArgs a) {
+  grid_dep_enter();
   constexpr int ROW = 2 * D * static_cast<int>(sizeof(T));  // bytes per metadata row
   constexpr int ROWP = ROW + 16;                             // padded pitch in shared memory
   constexpr bool MMA = UseMma<T, G, GAUSS>::value;
@@ -448,6 +449,7 @@ struct DirectOcc {
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::value)
     meta_direct_kernel(StreamArgs a) {
+  grid_dep_enter();
   constexpr int KP = 2 * D / 32;              // 32-element chunks per row
   constexpr int NT = Cols<G, GAUSS>::tiles;   // 8-column tiles of the B operand
   constexpr int ROW = 2 * D * 2;              // bytes per metadata row
@@ -641,8 +643,9 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
                                                  static_cast<int>(smem));
       if (e != cudaSuccess) return e;
     }
-    meta_direct_kernel<D, G, GAUSS>
-        <<<sm_count() * DirectOcc<D, G, GAUSS>::value, 32 * kDirectWarps, smem, st>>>(a);
+    const cudaError_t le_ = launch_k(meta_direct_kernel<D, G, GAUSS>, sm_count() * DirectOcc<D, G, GAUSS>::value,
+                                     32 * kDirectWarps, smem, st, a);
+    if (le_ != cudaSuccess) return le_;
     return cudaGetLastError();
   }
   constexpr int ROWP = 2 * D * static_cast<int>(sizeof(T)) + 16;
@@ -654,7 +657,10 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(meta_stream_kernel<T, D, G, GAUSS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  meta_stream_kernel<T, D, G, GAUSS><<<sm_count() * kCtasPerSm, kStreamThreads, smem, st>>>(a);
+  {
+    const cudaError_t le_ = launch_k(meta_stream_kernel<T, D, G, GAUSS>, sm_count() * kCtasPerSm, kStreamThreads, smem, st, a);
+    if (le_ != cudaSuccess) return le_;
+  }
   return cudaGetLastError();
 }
 

@@ -1,0 +1,123 @@
+"""GPU edge cases: single-token and ragged sequences, budgets that cover the
+whole sequence, and data errors (bad page ids, lengths, selections, a full
+Gaussian selection buffer) that the kernels turn into error flags."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sparse_kv_cache_kmax_b200 import binding as B
+from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+from sparse_kv_cache_kmax_b200.workloads import scaled_down
+
+from gpu_helpers import OUT_TOL, Gpu, gen, np64, oracle_unit, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_outputs(inp, eng, policy, k=None):
+    wl = inp["workload"]
+    G = wl.group
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            if policy == "full":
+                orc = oracle_unit(inp, b, h, policy="all")
+            else:
+                got = eng.sel[b, h, : int(eng.n_sel[b, h])].cpu().numpy()
+                orc = oracle_unit(inp, b, h, sel=got)
+            err = row_rel_err(np64(eng.out[b, h * G:(h + 1) * G]), orc["o"])
+            assert np.all(err <= OUT_TOL[wl.dtype]), (b, h, err.max())
+
+
+@pytest.mark.parametrize("lens", [[1, 17, 33], [16, 15, 1]])
+def test_tiny_and_ragged_sequences(lens):
+    wl = scaled_down("gqa_32k", batch=3, context=64)
+    inp = gen(wl, 21)
+    inp["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    for policy in ("topk", "full", "gauss"):
+        eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"],
+                           wl.num_q_heads, policy=policy, k=2, delta=0.5, alpha=1.5)
+        eng.build_meta()
+        eng.step(inp["q"])
+        torch.cuda.synchronize()
+        assert B.ekv_get_error() == 0
+        if policy == "topk":
+            P = [-(-L // wl.page_size) for L in lens]
+            assert eng.n_sel[:, 0].tolist() == [min(2, p) for p in P]
+        _check_outputs(inp, eng, policy)
+
+
+def test_budget_covering_every_page_selects_all():
+    wl = scaled_down("clustered_128k", batch=2, context=200)
+    inp = gen(wl, 22)
+    gpu = Gpu(inp)
+    gpu.build_meta()
+    sel, n = gpu.topk(gpu.score(), 64)
+    torch.cuda.synchronize()
+    P = -(-200 // wl.page_size)
+    assert torch.all(n == P)
+    assert torch.equal(sel[:, :, :P].cpu(), torch.arange(P, dtype=torch.int32).expand(2, wl.num_kv_heads, P))
+
+
+def test_bad_page_id_and_length_raise_flags_without_faulting():
+    wl = scaled_down("gqa_32k", batch=2, context=300)
+    inp = gen(wl, 23)
+    assert B.ekv_get_error() == 0
+    pt = inp["page_table"].clone()
+    pt[0, 3] = inp["num_phys"] + 5            # outside the pool: skipped by every kernel
+    lens = inp["seq_lens"].clone()
+    lens[1] = wl.max_pages * wl.page_size + 100  # longer than the page table: clamped
+    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], pt, lens, wl.num_q_heads, policy="topk", k=8)
+    eng.build_meta()
+    eng.step(inp["q"])
+    torch.cuda.synchronize()
+    flags = B.ekv_get_error()
+    assert flags & B.EKV_EFLAG_BAD_PAGE and flags & B.EKV_EFLAG_BAD_LEN
+    assert torch.isfinite(eng.out).all()
+    assert B.ekv_get_error() == 0                # reading clears the word
+
+
+def test_bad_selection_entries_raise_flag():
+    wl = scaled_down("gqa_32k", batch=1, context=300)
+    inp = gen(wl, 24)
+    gpu = Gpu(inp)
+    gpu.build_meta()
+    sel = torch.zeros(1, wl.num_kv_heads, 4, dtype=torch.int32, device="cuda")
+    sel[0, :, 1] = 10_000                         # past the sequence's pages
+    n = torch.full((1, wl.num_kv_heads), 4, dtype=torch.int32, device="cuda")
+    out, tau, cnt, bits = gpu.decode(1.5, sel, n, 4)
+    torch.cuda.synchronize()
+    assert B.ekv_get_error() & B.EKV_EFLAG_BAD_SEL
+    assert torch.isfinite(out).all()
+
+
+def test_gauss_selection_overflow_is_flagged_and_truncated():
+    wl = scaled_down("clustered_128k", batch=1, context=800)
+    inp = gen(wl, 25)
+    gpu = Gpu(inp)
+    gpu.build_meta()
+    sel, n, tau_hat = gpu.gauss(1.25, 1e6, cap=4)  # Δ huge: every page passes
+    torch.cuda.synchronize()
+    assert B.ekv_get_error() & B.EKV_EFLAG_SEL_OVERFLOW
+    assert torch.all(n == 4)
+    assert torch.equal(sel[0, :, :4].cpu(), torch.arange(4, dtype=torch.int32).expand(wl.num_kv_heads, 4))
+
+
+def test_fp32_cache_full_size_tiny_config():
+    """The tiny fp32 configuration at its full size (4096 tokens, 256 pages)."""
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS
+
+    wl = WORKLOADS["tiny_fp32"]
+    inp = gen(wl, 26)
+    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], 1,
+                       policy="topk", k=wl.topk, alpha=1.5)
+    eng.build_meta()
+    eng.step(inp["q"])
+    torch.cuda.synchronize()
+    orc = oracle_unit(inp, 0, 0, policy="topk", k=wl.topk)
+    got = eng.sel[0, 0, : int(eng.n_sel[0, 0])].cpu().numpy()
+    from gpu_helpers import assert_sel_matches, topk_tie_band
+    assert_sel_matches(got, orc["sel"], topk_tie_band(orc["score"], wl.topk), "tiny")
+    if not np.array_equal(got, orc["sel"]):
+        orc = oracle_unit(inp, 0, 0, sel=got)
+    assert row_rel_err(np64(eng.out[0]), orc["o"]).max() <= OUT_TOL["f32"]
