@@ -512,9 +512,9 @@ def run_kernel(args):
         nbytes = 2 * src.numel() * src.element_size()
     elif args.kernel in ("score", "gauss", "topk"):
         kv = torch.empty(1, Hkv, S, d, dtype=dt, device=dev)          # never read by these stages
-        lo = torch.randn(B * P, Hkv, 1, d, generator=g, device=dev)
+        lo = torch.randn(Hkv, B * P, 1, d, generator=g, device=dev)           # head-major [Hkv, pages, 2, d]
         box = torch.cat([lo + 0.5, lo - 0.5], dim=2).to(dt).contiguous()
-        mom = torch.cat([lo, torch.rand(B * P, Hkv, 1, d, generator=g, device=dev)], dim=2).to(dt).contiguous()
+        mom = torch.cat([lo, torch.rand(Hkv, B * P, 1, d, generator=g, device=dev)], dim=2).to(dt).contiguous()
         cache = Bd.make_cache(kv, kv, box, mom)
         cache.num_phys_pages = B * P
         seqs = Bd.make_seqs(page_table, seq_lens)

@@ -35,8 +35,10 @@
  * Memory layouts (row-major, dense)
  * ---------------------------------
  *   k_pool, v_pool [num_phys_pages, Hkv, S, d]
- *   box            [num_phys_pages, Hkv, 2, d]   row 0 = k_max, row 1 = k_min
- *   mom            [num_phys_pages, Hkv, 2, d]   row 0 = mean,  row 1 = variance
+ *   box            [Hkv, num_phys_pages, 2, d]   row 0 = k_max, row 1 = k_min
+ *   mom            [Hkv, num_phys_pages, 2, d]   row 0 = mean,  row 1 = variance
+ *                  (head-major: one head's rows of consecutive physical pages
+ *                  are adjacent, so scoring a sequence reads them in order)
  *   page_table     [batch, max_pages] int32, seq_lens [batch] int32
  *   q              [batch, Hq, d]
  *   ub             [batch, Hkv, max_pages] fp32

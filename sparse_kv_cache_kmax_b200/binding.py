@@ -130,9 +130,10 @@ _DTYPES = {torch.float32: EKV_F32, torch.bfloat16: EKV_BF16}
 
 def make_cache(k_pool, v_pool, box=None, mom=None) -> Cache:
     """Describe a paged cache.  k_pool, v_pool: [num_phys, Hkv, S, d];
-    box, mom: [num_phys, Hkv, 2, d] of the same dtype (allocated here if None)."""
+    box, mom: [Hkv, num_phys, 2, d] (head-major) of the same dtype (allocated
+    here if None)."""
     if box is None:
-        box = torch.empty(k_pool.shape[0], k_pool.shape[1], 2, k_pool.shape[3], dtype=k_pool.dtype,
+        box = torch.empty(k_pool.shape[1], k_pool.shape[0], 2, k_pool.shape[3], dtype=k_pool.dtype,
                           device=k_pool.device)
     if mom is None:
         mom = torch.empty_like(box)

@@ -260,11 +260,12 @@ EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
   const int32_t* use_sel = sel;
   const int32_t* use_n = n_sel;
   if (p->policy == EKV_POLICY_TOPK) {
-    EKV_TRY(cuda_status(launch_score(*cache, *seqs, q, num_q_heads, p->scale, ub, st)));
+    EKV_TRY(cuda_status(launch_score(*cache, *seqs, q, num_q_heads, p->scale, ub, st, p->append ? 1 : 0)));
     EKV_TRY(cuda_status(launch_topk(*seqs, cache->num_kv_heads, cache->page_size, ub, p->k, cap,
                                     sel, n_sel, st)));
   } else if (p->policy == EKV_POLICY_GAUSS) {
-    EKV_TRY(cuda_status(launch_gauss_stats(*cache, *seqs, q, num_q_heads, p->scale, p->alpha, gw, st)));
+    EKV_TRY(cuda_status(launch_gauss_stats(*cache, *seqs, q, num_q_heads, p->scale, p->alpha, gw, st,
+                                           p->append ? 1 : 0)));
     EKV_TRY(cuda_status(launch_gauss_select(*cache, *seqs, num_q_heads, p->alpha, p->delta, cap, gw,
                                             sel, n_sel, nullptr, st)));
   } else {

@@ -329,6 +329,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned in
       : "memory");
 }
 
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// its later async-proxy ones (a bulk copy into a slot that was read).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Sequence geometry with device-side checks (no trap: clamp and flag).
 __device__ __forceinline__ int seq_pages(const int32_t* seq_lens, int b, int S, int max_pages,
                                          int* len_out) {

@@ -5,25 +5,26 @@
 //
 // The unit's selected pages are split into C equal runs, one per CTA of the
 // cluster (C ≤ 16, chosen so that all units' clusters are resident at once).
-// Each CTA works in four phases separated by cluster barriers:
+// Each CTA works in three phases separated by cluster barriers:
 //  1. K: every warp streams its own pages (page j of the run goes to warp
 //     j mod 16) through a private ring of shared-memory slots filled by 1-D
-//     bulk async copies (one copy = one contiguous S×d K tile), then scores
+//     bulk async copies (one copy = one contiguous S×d K tile) and scores
 //     them on tensor cores (m16n8k16, rows of the tile loaded from shared
 //     memory straight into A fragments).  Scores z and page maxima stay in
-//     shared memory.
-//  2. τ: query head h is solved by CTA h mod C, which gathers the head's
-//     scores of the whole unit from the cluster's shared memory (DSMEM) in
-//     token order and solves Σ[u − τ]_+^β = 1, u = (α−1)·z, β = 1/(α−1):
-//     a histogram bracket over (max u − 1, max u], Newton's method from the
-//     left on the values above the bracket, and for β ∈ {1,2} the closed form
-//     on the support found.  τ goes to every CTA of the cluster.
-//  3. V: each CTA lists the pages of its run holding a support token
-//     (some head has a page maximum above τ) and its warps read only those V
-//     rows; p = [u − τ]_+^β comes from the scores in shared memory.  The
-//     support bits and counts of the run's tokens are written alongside.
-//  4. The CTA partial outputs are summed across the cluster in rank order,
-//     CTA r owning a 1/C slice of the unit's G×d outputs.
+//     shared memory.  The CTA then pushes its per-head maxima to the CTAs
+//     that solve those heads and starts bulk copies of the V tiles of the
+//     pages that can hold support (a page maximum within 1 of the run's
+//     maximum, in u = (α−1)·z units: τ ≥ max u − 1).
+//  2. τ: query head h is solved by CTA h mod C on the head's scores of the
+//     whole unit, gathered from the cluster's shared memory (DSMEM) in token
+//     order: Σ[u − τ]_+^β = 1, β = 1/(α−1) (see cta_solve_tau).  The solver
+//     writes the head's support bits and count and sends τ to every CTA.
+//  3. V: each CTA lists the pages of its run holding a support token (some
+//     head's page maximum above τ) and its warps read only those V tiles,
+//     from shared memory when staged, else from global memory; p = [u − τ]^β
+//     comes from the scores in shared memory.  CTA r owns a 1/C slice of the
+//     unit's G×d outputs: every CTA pushes its partial of that slice to CTA
+//     r, which sums the C partials in rank order.
 // Every sum has a fixed order, so results are deterministic.
 #include <cooperative_groups.h>
 
@@ -41,16 +42,22 @@ namespace cg = cooperative_groups;
 constexpr int kFWarps = 16;
 constexpr int kFThreads = 32 * kFWarps;
 constexpr int kFMaxCluster = 16;
-constexpr int kFMaxSpw = 8;                   // ring slots per warp
+constexpr int kFMaxSpw = 8;       // K ring slots per warp
+constexpr int kFMaxVSlots = 64;   // staged V tiles per CTA
+constexpr int kFMaxHeads = 16;    // query heads per KV head (G)
 constexpr int kTauBinsF = 256;
+constexpr int kPairwiseMax = 256; // candidates for the pairwise support test
 
 struct FusedGeom {
   int C;          // CTAs per unit (cluster size)
   int spc;        // selected slots per CTA
   int zpitch;     // floats per head row of the score array (spc·S + 4)
-  int spw;        // ring slots per warp
+  int spw;        // K ring slots per warp
   int tile_bytes; // bytes of one S×d K or V tile
-  int off_ints, off_pm, off_zs, off_out, off_ring;  // byte offsets in dynamic shared memory
+  int chunk;      // outputs owned per CTA: ceil(G·d / C)
+  int off_ints, off_pm, off_zs, off_inbox, off_ring;  // byte offsets in dynamic shared memory
+  int off_v;      // V staging area, from the start of the ring
+  int nvslots;    // staged V tiles
   int smem;       // dynamic shared memory bytes
 };
 
@@ -58,17 +65,13 @@ struct TauShared {
   float f[2][kFWarps];   // fp32 partials, double-buffered: one barrier per reduction
   float f2[2][kFWarps];
   double d[3][kFWarps];  // fp64 partials
-  int i[32];
+  int i[kFWarps];
   int hist[kTauBinsF];
-  float m;
   double tau;
 };
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, unsigned int bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // Pairwise sum of the 16 per-warp partials (a fixed tree, so every thread
@@ -95,8 +98,8 @@ __device__ __forceinline__ V pow_bm1(V w, V beta, int ipow) {
   }
 }
 
-// f(t) = Σ(u − t)_+^β − 1 and f'(t)/(−β) = Σ(u − t)_+^(β−1) over the
-// candidates, by one warp (solo) or by the CTA (one barrier, parity `par`).
+// f(t) − 1 = Σ(u − t)_+^β − 1 and Σ(u − t)_+^(β−1) over the candidates, by
+// one warp (solo) or by the CTA (one barrier, buffer parity `par`).
 template <typename V>
 __device__ __forceinline__ void f_df(const float* cand, int nc, V t, V beta, int ipow, bool solo,
                                      TauShared& sh, int par, V& f, V& df) {
@@ -126,89 +129,156 @@ __device__ __forceinline__ void f_df(const float* cand, int nc, V t, V beta, int
       b = tree16(sh.f2[par]);
     } else {
       if (lane == 0) {
-        sh.d[par][warp] = a;
-        sh.d[2][warp] = b;
+        sh.d[0][warp] = a;
+        sh.d[1][warp] = b;
       }
       __syncthreads();
-      a = tree16(sh.d[par]);
-      b = tree16(sh.d[2]);
+      a = tree16(sh.d[0]);
+      b = tree16(sh.d[1]);
+      __syncthreads();
     }
   }
   f = a - V(1);
   df = b;
 }
 
-// τ of one query head: Σ_i [u_i − τ]_+^β = 1, u_i = (α−1)·z_i, over the n
-// scores z[0..n) in shared memory (m = their maximum, finite); the whole CTA
-// calls it with sh.hist zeroed.  cand: shared scratch of n floats.
-//  1. Bracket: a histogram of u over (max u − 1, max u]; c values above an
-//     edge e force τ ≥ e − c^(−1/β).
-//  2. The values above the bracket are compacted in scan order.
-//  3. Newton's method from the left in fp32 (f is convex and decreasing),
-//     then float64: for β ∈ {1,2} the closed form on the support found
-//     (β = 1: τ = (Σu − 1)/k; β = 2: τ = M − √(M² − Q + 1/k) with M, Q the
-//     support's mean and mean square), repeated until the support is stable;
-//     otherwise one float64 Newton step.
-// Returns the fp32 τ every later step uses.
-__device__ float cta_solve_tau(const float* z, int n, float m, float* cand, float am1, float beta,
-                               int ib, int ipow, TauShared& sh) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float um = am1 * m;
-  for (int i = tid; i < n; i += kFThreads) {
-    const float u = am1 * z[i];
-    if (u > um - 1.0f) atomicAdd(&sh.hist[min(kTauBinsF - 1, static_cast<int>((um - u) * kTauBinsF))], 1);
+// Sums of (c, s1, s2) over the CTA (fp64, fixed tree); every thread gets them.
+__device__ __forceinline__ void cta_sum3(double& c, double& s1, double& s2, TauShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  if (lane == 0) {
+    sh.d[0][warp] = c;
+    sh.d[1][warp] = s1;
+    sh.d[2][warp] = s2;
   }
   __syncthreads();
+  c = tree16(sh.d[0]);
+  s1 = tree16(sh.d[1]);
+  s2 = tree16(sh.d[2]);
+  __syncthreads();
+}
+
+// Closed-form τ on a support of c values with sums s1 = Σu, s2 = Σu²:
+// β = 1: τ = (s1 − 1)/c;  β = 2: τ = M − √(M² − Q + 1/c), M = s1/c, Q = s2/c.
+__device__ __forceinline__ double closed_tau(int ipow, double c, double s1, double s2) {
+  if (ipow == 1) return (s1 - 1.0) / c;
+  const double M = s1 / c, Q = s2 / c;
+  return M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
+}
+
+// τ of one query head: Σ_i [u_i − τ]_+^β = 1, u_i = (α−1)·z_i, over the n
+// scores z[0..n) in shared memory whose histogram over (um − 1, um] (um =
+// (α−1)·max z, 256 bins from the top) is in sh.hist.  The whole CTA calls it;
+// it leaves sh.hist zeroed.  cand: shared scratch of n floats.
+//  1. Bracket: c values above an edge e force τ ≥ e − c^(−1/β) (c of them
+//     would already carry mass ≥ 1); the best edge gives τ_lo.
+//  2. The values above τ_lo are compacted (warp order, then scan order).
+//  3. For β ∈ {1,2} and few candidates: u_j is in the support iff
+//     f(u_j) = Σ_i (u_i − u_j)_+^β < 1 (f decreases, f(τ) = 1), tested for
+//     every candidate at once; τ is the float64 closed form on that support,
+//     kept if the support it implies is the same, else refined by repeating
+//     the closed form on {u > τ}.  Otherwise Newton's method from the left in
+//     fp32 (f is convex and decreasing) and a float64 finish: the closed form
+//     for β ∈ {1,2}, one float64 Newton step otherwise.
+// Returns the fp32 τ every later step uses.
+__device__ float cta_solve_tau(const float* z, int n, float um, float* cand, float am1, float beta,
+                               int ipow, TauShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // 1. bracket, computed by every warp from the histogram (no barrier)
   float cb = um - 1.0f;
   {
-    const int h = tid < kTauBinsF ? sh.hist[tid] : 0;
-    int total;
-    const int c = block_exclusive_scan(h, sh.i, &total) + h;
-    if (tid < kTauBinsF && c > 0)
-      cb = fmaxf(cb, um - static_cast<float>(tid + 1) / kTauBinsF - powf(static_cast<float>(c), -1.0f / beta));
-  }
+    constexpr int kPer = kTauBinsF / 32;
+    int cnt[kPer], tot = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cb = fmaxf(cb, __shfl_xor_sync(0xffffffffu, cb, o));
-  if (lane == 0) sh.f[0][warp] = cb;
-  __syncthreads();
-  cb = sh.f[0][0];
-#pragma unroll
-  for (int w = 1; w < kFWarps; ++w) cb = fmaxf(cb, sh.f[0][w]);
-  const double tau_lo = static_cast<double>(cb) - 1e-6 * (1.0 + fabs(static_cast<double>(um)));
-  int mine = 0;
-  for (int i = tid; i < n; i += kFThreads) mine += static_cast<double>(am1 * z[i]) > tau_lo ? 1 : 0;
-  int nc;
-  int pos = block_exclusive_scan(mine, sh.i, &nc);
-  for (int i = tid; i < n; i += kFThreads) {
-    const float u = am1 * z[i];
-    if (static_cast<double>(u) > tau_lo) cand[pos++] = u;
-  }
-  __syncthreads();
-  const bool solo = nc <= 1024;
-  if (!solo || warp == 0) {
-    // fp32 Newton from the left
-    float t = static_cast<float>(tau_lo);
-    if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
-    int par = 1;
-    for (int it = 0; it < 64; ++it) {
-      float f, df;
-      par ^= 1;
-      f_df<float>(cand, nc, t, beta, ipow, solo, sh, par, f, df);
-      if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
-        t = um - 1.0f;
-        continue;
-      }
-      const float step = f / (beta * df);
-      if (!(step > 0.0f)) break;
-      t += step;
-      if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+    for (int k = 0; k < kPer; ++k) {
+      tot += sh.hist[lane * kPer + k];
+      cnt[k] = tot;
     }
-    // float64 finish
-    double tau = t;
-    if (ib == 1 || ib == 2) {
-      for (int rep = 0; rep < 4; ++rep) {
-        double c = 0.0, s1 = 0.0, s2 = 0.0;
-        for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int before = incl - tot;
+    // c^(−1/β) without libm: exact-enough reciprocals for β ∈ {1,2}, fast
+    // exp2/log2 otherwise; the slack below keeps τ_lo a lower bound
+#pragma unroll 1
+    for (int k = 0; k < kPer; ++k) {
+      const int c = before + cnt[k];
+      if (c > 0) {
+        const float fc = static_cast<float>(c);
+        const float r = ipow == 1 ? 1.0f / fc : (ipow == 2 ? rsqrtf(fc) : exp2f(-__log2f(fc) / beta));
+        cb = fmaxf(cb, um - static_cast<float>(lane * kPer + k + 1) / kTauBinsF - r);
+      }
+    }
+    cb = warp_max(cb);
+  }
+  const double tau_lo = static_cast<double>(cb) - 4e-6 * (1.0 + fabs(static_cast<double>(um)));
+  // 2. compaction: warp w takes elements k·512 + 32w + lane; order (w, k, lane)
+  int nc;
+  {
+    int mine = 0;
+    for (int base = 0; base < n; base += kFThreads) {
+      const int i = base + tid;
+      const bool in = i < n && static_cast<double>(am1 * z[i]) > tau_lo;
+      mine += __popc(__ballot_sync(0xffffffffu, in));
+    }
+    if (lane == 0) sh.i[warp] = mine;
+    __syncthreads();
+    int pos = 0;
+    nc = 0;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) {
+      const int c = sh.i[w];
+      pos += w < warp ? c : 0;
+      nc += c;
+    }
+    for (int base = 0; base < n; base += kFThreads) {
+      const int i = base + tid;
+      const float u = i < n ? am1 * z[i] : -INFINITY;
+      const bool in = i < n && static_cast<double>(u) > tau_lo;
+      const unsigned int bal = __ballot_sync(0xffffffffu, in);
+      if (in) cand[pos + __popc(bal & ((1u << lane) - 1u))] = u;
+      pos += __popc(bal);
+    }
+    for (int i = tid; i < kTauBinsF; i += kFThreads) sh.hist[i] = 0;  // ready for the next head
+    __syncthreads();
+  }
+  // 3. τ
+  double tau;
+  const bool closed = ipow == 1 || ipow == 2;
+  if (closed && nc <= kPairwiseMax) {
+    bool in = false;
+    float ut = 0.f;
+    double c = 0.0, s1 = 0.0, s2 = 0.0;
+    if (tid < nc) {
+      ut = cand[tid];
+      float fs = 0.f;
+#pragma unroll 4
+      for (int i = 0; i < nc; ++i) {
+        const float w = cand[i] - ut;
+        if (w > 0.f) fs = fmaf(ipow == 1 ? 1.0f : w, w, fs);
+      }
+      in = fs < 1.0f;
+      if (in) {
+        c = 1.0;
+        s1 = ut;
+        s2 = static_cast<double>(ut) * ut;
+      }
+    }
+    cta_sum3(c, s1, s2, sh);
+    tau = closed_tau(ipow, c, s1, s2);
+    const bool bad = tid < nc && (in != (static_cast<double>(ut) > tau));
+    if (__syncthreads_or(bad)) {
+      for (int rep = 0; rep < 8; ++rep) {
+        c = s1 = s2 = 0.0;
+        for (int i = tid; i < nc; i += kFThreads) {
           const double u = cand[i];
           if (u > tau) {
             c += 1.0;
@@ -216,71 +286,81 @@ __device__ float cta_solve_tau(const float* z, int n, float m, float* cand, floa
             s2 += u * u;
           }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          c += __shfl_xor_sync(0xffffffffu, c, o);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-          s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-        }
-        if (!solo) {
-          if (lane == 0) {
-            sh.d[0][warp] = c;
-            sh.d[1][warp] = s1;
-            sh.d[2][warp] = s2;
-          }
-          __syncthreads();
-          c = tree16(sh.d[0]);
-          s1 = tree16(sh.d[1]);
-          s2 = tree16(sh.d[2]);
-          __syncthreads();
-        }
+        cta_sum3(c, s1, s2, sh);
         if (c < 1.0) break;
-        double t_new;
-        if (ib == 1) {
-          t_new = (s1 - 1.0) / c;
-        } else {
-          const double M = s1 / c, Q = s2 / c;
-          t_new = M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
-        }
+        const double t_new = closed_tau(ipow, c, s1, s2);
         if (t_new == tau) break;
         tau = t_new;
       }
-    } else {
-      double f, df;
-      f_df<double>(cand, nc, tau, static_cast<double>(beta), ipow, solo, sh, 0, f, df);
-      if (df > 0.0) tau += f / (static_cast<double>(beta) * df);
     }
-    if (tid == 0) sh.tau = tau;
-  }
-  __syncthreads();
-  return static_cast<float>(sh.tau);
-}
-
-// Four (D = 128) or two (D = 64) consecutive bf16 of a V row as fp32.
-template <int DPL>
-__device__ __forceinline__ void load_v(const bf16* p, float (&v)[DPL]) {
-  if constexpr (DPL == 4) {
-    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(p));
-    v[0] = __uint_as_float(w.x << 16);
-    v[1] = __uint_as_float(w.x & 0xffff0000u);
-    v[2] = __uint_as_float(w.y << 16);
-    v[3] = __uint_as_float(w.y & 0xffff0000u);
   } else {
-    const uint32_t w = __ldcs(reinterpret_cast<const unsigned int*>(p));
-    v[0] = __uint_as_float(w << 16);
-    v[1] = __uint_as_float(w & 0xffff0000u);
+    const bool solo = nc <= 1024;
+    if (!solo || warp == 0) {
+      float t = static_cast<float>(tau_lo);
+      if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
+      int par = 1;
+      for (int it = 0; it < 64; ++it) {
+        float f, df;
+        par ^= 1;
+        f_df<float>(cand, nc, t, beta, ipow, solo, sh, par, f, df);
+        if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
+          t = um - 1.0f;
+          continue;
+        }
+        const float step = f / (beta * df);
+        if (!(step > 0.0f)) break;
+        t += step;
+        if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+      }
+      double tt = t;
+      if (closed) {
+        for (int rep = 0; rep < 4; ++rep) {
+          double c = 0.0, s1 = 0.0, s2 = 0.0;
+          for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
+            const double u = cand[i];
+            if (u > tt) {
+              c += 1.0;
+              s1 += u;
+              s2 += u * u;
+            }
+          }
+          if (solo) {
+            c = warp_sum(c);
+            s1 = warp_sum(s1);
+            s2 = warp_sum(s2);
+          } else {
+            cta_sum3(c, s1, s2, sh);
+          }
+          if (c < 1.0) break;
+          const double t_new = closed_tau(ipow, c, s1, s2);
+          if (t_new == tt) break;
+          tt = t_new;
+        }
+      } else {
+        double f, df;
+        f_df<double>(cand, nc, tt, static_cast<double>(beta), ipow, solo, sh, 0, f, df);
+        if (df > 0.0) tt += f / (static_cast<double>(beta) * df);
+      }
+      if (tid == 0) sh.tau = tt;
+    }
+    __syncthreads();
+    tau = sh.tau;
+    __syncthreads();
   }
+  return static_cast<float>(tau);
 }
 
 template <int D, int G>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a, FusedGeom f) {
   constexpr int KP = D / 32, NT = (G + 7) / 8, DPL = D / 32;
-  constexpr int VCH = G >= 8 ? 8 : 16;  // V rows in flight per warp
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint64_t bars[kFWarps * kFMaxSpw];
+  __shared__ uint64_t vbars[kFMaxVSlots];
   __shared__ TauShared tsh;
   __shared__ float s_tau[G];
   __shared__ float s_mloc[G];
+  __shared__ float mlocs[kFMaxHeads][kFMaxCluster];  // run maxima of the heads this CTA solves
+  __shared__ int s_vcount;
   __shared__ int scan_scratch[32];
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -292,15 +372,20 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   int* phys_s = reinterpret_cast<int*>(smem + f.off_ints);  // [spc]
   int* nv_s = phys_s + spc;                                  // [spc]
   int* list_s = nv_s + spc;                                  // [spc]
+  int* vslot_s = list_s + spc;                               // [spc] staged V slot or −1
   float* pm = reinterpret_cast<float*>(smem + f.off_pm);     // [G][spc] page maxima of z
   float* zs = reinterpret_cast<float*>(smem + f.off_zs);     // [G][zpitch] scores z
-  float* out_s = reinterpret_cast<float*>(smem + f.off_out); // [G][D] CTA partial output
+  float* inbox = reinterpret_cast<float*>(smem + f.off_inbox);  // [C][chunk] partial outputs
   unsigned char* ring = smem + f.off_ring;
+  unsigned char* vtiles = ring + f.off_v;
 
   if (tid == 0) {
     for (int s = 0; s < kFWarps * spw; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < f.nvslots; ++s) mbar_init(&vbars[s], 1);
     fence_mbar_init();
+    s_vcount = 0;
   }
+  for (int i = tid; i < kTauBinsF; i += kFThreads) tsh.hist[i] = 0;
   __syncthreads();
   grid_dep_enter();
   int L;
@@ -394,62 +479,76 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     }
   }
   __syncthreads();
-  // V tiles of the pages that can hold support (a page maximum within 1 of
-  // this run's maximum, in u) start moving to L2 while τ is solved
-  if (!a.dense_v) {
-    for (int h = warp; h < G; h += kFWarps) {
-      float m = -INFINITY;
-      for (int j = lane; j < np; j += 32) m = fmaxf(m, pm[h * spc + j]);
-      m = warp_max(m);
-      if (lane == 0) s_mloc[h] = m;
+  // run maxima per head, pushed to the head's solver
+  for (int h = warp; h < G; h += kFWarps) {
+    float m = -INFINITY;
+    for (int j = lane; j < np; j += 32) m = fmaxf(m, pm[h * spc + j]);
+    m = warp_max(m);
+    if (lane == 0) {
+      s_mloc[h] = m;
+      cluster.map_shared_rank(&mlocs[0][0], h % C)[(h / C) * kFMaxCluster + rank] = m;
     }
-    __syncthreads();
   }
+  __syncthreads();
+  // V tiles of the pages that can hold support start moving into shared memory
   for (int j = tid; j < np; j += kFThreads) {
     const int ph = phys_s[j];
-    if (ph < 0) continue;
-    bool cand = a.dense_v != 0;
+    bool cand = ph >= 0 && a.dense_v != 0;
+    if (ph >= 0 && !cand) {
 #pragma unroll
-    for (int h = 0; h < G; ++h)
-      if (!cand && pm[h * spc + j] > -INFINITY && a.am1 * pm[h * spc + j] > a.am1 * s_mloc[h] - 1.0f) cand = true;
-    if (cand)
-      prefetch_l2_bulk(static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems,
-                       static_cast<unsigned int>(f.tile_bytes));
+      for (int h = 0; h < G; ++h) {
+        const float pz = pm[h * spc + j];
+        if (pz > -INFINITY && a.am1 * pz > a.am1 * s_mloc[h] - 1.0f) cand = true;
+      }
+    }
+    int vs = -1;
+    if (cand) {
+      const int sidx = atomicAdd(&s_vcount, 1);
+      if (sidx < f.nvslots) {
+        vs = sidx;
+        fence_proxy_async_smem();  // K tiles read from this area come before the copy
+        mbar_arrive_expect_tx(&vbars[vs], static_cast<unsigned int>(f.tile_bytes));
+        bulk_g2s(vtiles + static_cast<size_t>(vs) * f.tile_bytes,
+                 static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems,
+                 static_cast<unsigned int>(f.tile_bytes), &vbars[vs]);
+      }
+    }
+    vslot_s[j] = vs;
   }
   cluster.sync();
 
   // ---------------------------------------------------------------- 2. τ
-  // Head h is solved by CTA h mod C on the unit's scores gathered in token
-  // order; the solver also writes the head's support bits and count.
   const int tpc = spc * S;
   const int n_tok = n_slots * S;
   float* zh = reinterpret_cast<float*>(ring);
   float* cand = zh + ((n_tok + 31) & ~31);
   const size_t words = static_cast<size_t>(a.words);
-  for (int h = rank; h < G; h += C) {
+  for (int h = rank, hl = 0; h < G; h += C, ++hl) {
     const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h;
-    for (int i = tid; i < kTauBinsF; i += kFThreads) tsh.hist[i] = 0;
     float m = -INFINITY;
-    for (int i = 4 * tid; i < n_tok; i += 4 * kFThreads) {
-      const int r = i / tpc;
-      const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(zs, r) + h * zp + (i - r * tpc));
-      *reinterpret_cast<float4*>(zh + i) = v;
-      m = fmaxf(fmaxf(m, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
-    }
-    m = warp_max(m);
-    if (lane == 0) tsh.f[0][warp] = m;
-    __syncthreads();
-    m = tsh.f[0][0];
-#pragma unroll
-    for (int w = 1; w < kFWarps; ++w) m = fmaxf(m, tsh.f[0][w]);
+    for (int r = 0; r < C; ++r) m = fmaxf(m, mlocs[hl][r]);
     float tau = INFINITY;  // no finite score: no support, zero output
-    if (m > -INFINITY) tau = cta_solve_tau(zh, n_tok, m, cand, a.am1, a.beta, a.ibeta, a.ipow, tsh);
+    if (m > -INFINITY) {
+      const float um = a.am1 * m;
+      for (int i = 4 * tid; i < n_tok; i += 4 * kFThreads) {
+        const int r = i / tpc;
+        const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(zs, r) + h * zp + (i - r * tpc));
+        *reinterpret_cast<float4*>(zh + i) = v;
+        const float uu[4] = {a.am1 * v.x, a.am1 * v.y, a.am1 * v.z, a.am1 * v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (uu[k] > um - 1.0f)
+            atomicAdd(&tsh.hist[min(kTauBinsF - 1, static_cast<int>((um - uu[k]) * kTauBinsF))], 1);
+      }
+      __syncthreads();
+      tau = cta_solve_tau(zh, n_tok, um, cand, a.am1, a.beta, a.ipow, tsh);
+    }
     if (tid < C) cluster.map_shared_rank(s_tau, tid)[h] = tau;
     if (tid == 0 && a.tau_out) a.tau_out[orow] = tau;
     int cnt = 0;
     for (int base = 0; base < n_tok; base += kFThreads) {
       const int i = base + tid;
-      const bool in = i < n_tok && a.am1 * zh[i] > tau;
+      const bool in = i < n_tok && tau < INFINITY && a.am1 * zh[i] > tau;
       cnt += in ? 1 : 0;
       const unsigned int bal = __ballot_sync(0xffffffffu, in);
       if (a.bits_out && lane == 0 && i < n_tok) a.bits_out[orow * words + i / 32] = bal;
@@ -457,7 +556,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     if (a.bits_out)
       for (int w = (n_tok + 31) / 32 + tid; w < a.words; w += kFThreads) a.bits_out[orow * words + w] = 0u;
     cnt = warp_sum(cnt);
-    __syncthreads();  // tsh.i and zh are free again after this
     if (lane == 0) tsh.i[warp] = cnt;
     __syncthreads();
     if (tid == 0 && a.count_out) {
@@ -465,6 +563,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
       for (int w = 0; w < kFWarps; ++w) c += tsh.i[w];
       a.count_out[orow] = c;
     }
+    __syncthreads();  // zh, cand and tsh are reused by the next head
   }
   cluster.sync();
 
@@ -489,50 +588,57 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   }
   __syncthreads();
 
+  // All warps walk the same support pages; warp r takes rows r, r+16, ...
+  // of each page and accumulates p·v over its rows for every head.
   float acc[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
-  for (int e = warp; e < nsup; e += kFWarps) {
-    const int j = list_s[e], ph = phys_s[j], nvv = nv_s[j];
-    const bf16* vrow = static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems + lane * DPL;
-    for (int t0 = 0; t0 < nvv; t0 += 32) {
-      float p[G];
+#pragma unroll 1
+  for (int e = 0; e < nsup; ++e) {
+    const int j = list_s[e], nvv = nv_s[j], vs = vslot_s[j];
+    const bf16* vbase;
+    if (vs >= 0) {
+      if (!mbar_wait(&vbars[vs], 0u)) mbar_wait(&vbars[vs], 0u);
+      vbase = reinterpret_cast<const bf16*>(vtiles + static_cast<size_t>(vs) * f.tile_bytes);
+    } else {
+      vbase = static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * tile_elems;
+    }
+#pragma unroll 1
+    for (int r = warp; r < nvv; r += kFWarps) {
+      float v[DPL];
+      const bf16* src = vbase + static_cast<size_t>(r) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        v[0] = __uint_as_float(w.x << 16);
+        v[1] = __uint_as_float(w.x & 0xffff0000u);
+        v[2] = __uint_as_float(w.y << 16);
+        v[3] = __uint_as_float(w.y & 0xffff0000u);
+      } else {
+        const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
+        v[0] = __uint_as_float(w << 16);
+        v[1] = __uint_as_float(w & 0xffff0000u);
+      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        p[h] = 0.f;
-        if (t0 + lane < nvv) {
-          const float w = a.am1 * zs[h * zp + j * S + t0 + lane] - s_tau[h];
-          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ipow);
-        }
-      }
-      const int nt32 = min(32, nvv - t0);
-      for (int t1 = 0; t1 < nt32; t1 += VCH) {
-        float vv[VCH][DPL];
+        const float w = a.am1 * zs[h * zp + j * S + r] - s_tau[h];
+        if (w > 0.f) {
+          const float p = pow_beta_fast(w, a.beta, a.ipow);
 #pragma unroll
-        for (int tt = 0; tt < VCH; ++tt) {
-          if (t1 + tt < nt32) {
-            load_v<DPL>(vrow + static_cast<size_t>(t0 + t1 + tt) * D, vv[tt]);
-          } else {
-#pragma unroll
-            for (int e2 = 0; e2 < DPL; ++e2) vv[tt][e2] = 0.f;
-          }
-        }
-#pragma unroll
-        for (int tt = 0; tt < VCH; ++tt) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pt = __shfl_sync(0xffffffffu, p[h], (t1 + tt) & 31);
-#pragma unroll
-            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(pt, vv[tt][e2], acc[h][e2]);
-          }
+          for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(p, v[e2], acc[h][e2]);
         }
       }
     }
   }
-  // warp partials → CTA partial (warp order)
-  float* red = reinterpret_cast<float*>(ring);  // [kFWarps][G][D]
+  // every staged copy has landed before its area is reused or the CTA exits
+  {
+    const int issued = min(s_vcount, f.nvslots);
+    for (int s = tid; s < issued; s += kFThreads)
+      if (!mbar_wait(&vbars[s], 0u)) mbar_wait(&vbars[s], 0u);
+  }
+  // warp partials → CTA partial (warp order) → the owner's inbox
+  float* red = reinterpret_cast<float*>(ring);  // [kFWarps][G][D], over the finished τ scratch
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -542,20 +648,21 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     float pw[kFWarps];
 #pragma unroll
     for (int w = 0; w < kFWarps; ++w) pw[w] = red[w * G * D + i];
-    out_s[i] = tree16(pw);
+    const int owner = i / f.chunk;
+    cluster.map_shared_rank(inbox, owner)[rank * f.chunk + (i - owner * f.chunk)] = tree16(pw);
   }
   cluster.sync();
 
-  // ---------------------------------------------------------------- 4. cluster sum
-  const int GD = G * D, chunk = (GD + C - 1) / C;
-  const int i_end = min(GD, (rank + 1) * chunk);
-  for (int i = rank * chunk + tid; i < i_end; i += kFThreads) {
+  // ---------------------------------------------------------------- 4. owner sums
+  const int GD = G * D;
+  for (int k = tid; k < f.chunk; k += kFThreads) {
+    const int i = rank * f.chunk + k;
+    if (i >= GD) break;
     float s = 0.f;
-    for (int r = 0; r < C; ++r) s += cluster.map_shared_rank(out_s, r)[i];
+    for (int r = 0; r < C; ++r) s += inbox[r * f.chunk + k];
     const int h = i / D, d = i - h * D;
     a.out[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h) * D + d] = s;
   }
-  cluster.sync();  // no CTA leaves while another still reads its shared memory
 }
 
 // ------------------------------------------------------------------ host side
@@ -591,25 +698,32 @@ FusedGeom plan(int C, int cap, int S, int smem_limit) {
   f.spc = round_up(f.spc, step);
   f.zpitch = f.spc * S + 4;
   f.tile_bytes = S * D * 2;
+  f.chunk = (G * D + C - 1) / C;
   int off = 0;
   f.off_ints = off;
-  off += round_up(3 * f.spc * 4, 128);
+  off += round_up(4 * f.spc * 4, 128);
   f.off_pm = off;
   off += round_up(G * f.spc * 4, 128);
   f.off_zs = off;
   off += round_up(G * f.zpitch * 4, 128);
-  f.off_out = off;
-  off += round_up(G * D * 4, 128);
+  f.off_inbox = off;
+  off += round_up(C * f.chunk * 4, 128);
   f.off_ring = off;
   const int n_tok_max = cap * S;
-  const int ring_min = std::max(2 * round_up(n_tok_max, 32) * 4, kFWarps * G * D * 4);
+  f.off_v = round_up(std::max(2 * round_up(n_tok_max, 32) * 4, kFWarps * G * D * 4), 128);
   const int pages_per_warp = (f.spc + kFWarps - 1) / kFWarps;
   const int avail = smem_limit - off;
-  int spw = std::min(std::min(pages_per_warp, kFMaxSpw), avail / (kFWarps * f.tile_bytes));
+  const int spw = std::min(std::min(pages_per_warp, kFMaxSpw), avail / (kFWarps * f.tile_bytes));
   if (spw < 1) return FusedGeom{};
   f.spw = spw;
-  const int ring = std::max(kFWarps * spw * f.tile_bytes, ring_min);
+  const int ring_k = kFWarps * spw * f.tile_bytes;
+  int ring = std::max(ring_k, f.off_v);
+  // staged V tiles in what is left, up to one per page of the run
+  const int want = std::min(kFMaxVSlots, f.spc);
+  const int room = std::min(avail, f.off_v + want * f.tile_bytes);
+  ring = std::max(ring, room);
   if (off + ring > smem_limit) return FusedGeom{};
+  f.nvslots = std::max(0, std::min(want, (ring - f.off_v) / f.tile_bytes));
   f.smem = off + ring;
   return f;
 }

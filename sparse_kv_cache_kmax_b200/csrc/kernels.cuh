@@ -32,10 +32,13 @@ struct GaussWs {
 cudaError_t launch_build_meta(const ekv_cache& c, const ekv_seqs& s, cudaStream_t st);
 cudaError_t launch_append(const ekv_cache& c, const ekv_seqs& s, const void* k_new,
                           const void* v_new, cudaStream_t st);
+// after_append = 1: the previous kernel on the stream is launch_append, and
+// the bf16 kernels overlap it (only tiles holding a sequence's last page wait).
 cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq, float scale,
-                         float* ub, cudaStream_t st);
+                         float* ub, cudaStream_t st, int after_append = 0);
 cudaError_t launch_gauss_stats(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
-                               float scale, float alpha, const GaussWs& ws, cudaStream_t st);
+                               float scale, float alpha, const GaussWs& ws, cudaStream_t st,
+                               int after_append = 0);
 cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
                         int32_t* sel, int32_t* n_sel, cudaStream_t st);
 cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, float alpha,

@@ -121,8 +121,9 @@ __global__ void build_meta_kernel(const T* __restrict__ k_pool, T* __restrict__ 
     if (!phys_ok(phys, num_phys)) continue;
     const int n = min(S, L - p * S);
     const size_t ph = static_cast<size_t>(phys) * Hkv + h;
-    page_pair_meta<T>(k_pool + ph * S * D, D, n, j, -1, 0.f, 0.f, box + ph * 2 * D,
-                      mom + ph * 2 * D);
+    const size_t mh = static_cast<size_t>(h) * num_phys + phys;  // head-major metadata row
+    page_pair_meta<T>(k_pool + ph * S * D, D, n, j, -1, 0.f, 0.f, box + mh * 2 * D,
+                      mom + mh * 2 * D);
   }
 }
 
@@ -149,8 +150,9 @@ __global__ void append_kernel(T* __restrict__ k_pool, T* __restrict__ v_pool, T*
   Pair<T>::load(k_new + src, xa, xb);
   Pair<T>::copy(k_pool + (ph * S + slot) * D + j, k_new + src);
   Pair<T>::copy(v_pool + (ph * S + slot) * D + j, v_new + src);
-  page_pair_meta<T>(k_pool + ph * S * D, D, slot + 1, j, slot, xa, xb, box + ph * 2 * D,
-                    mom + ph * 2 * D);
+  const size_t mh = static_cast<size_t>(h) * num_phys + phys;  // head-major metadata row
+  page_pair_meta<T>(k_pool + ph * S * D, D, slot + 1, j, slot, xa, xb, box + mh * 2 * D,
+                    mom + mh * 2 * D);
 }
 
 }  // namespace

@@ -51,6 +51,10 @@ struct StreamArgs {
   GaussWs gws;               // Gaussian statistics outputs
   float scale, am1;
   int Hkv, Hq, S, num_phys, max_pages, batch;
+  // 1: the preceding kernel on the stream is the cache append, whose writes
+  // reach only the last page of every sequence; the bf16 kernel then waits
+  // for it just before the tiles holding those pages (see meta_direct_kernel)
+  int defer_wait;
 };
 
 // Walks a CTA's slice [f0, f1) of the flattened rows as ≤ kRows-row stages
@@ -196,7 +200,7 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) meta_stream_kernel
           const bool good = phys_ok(ids[k], a.num_phys);
           ok[stage * kRows + i] = good ? 1 : 0;
           if (good) {
-            src[k] = static_cast<const unsigned char*>(a.rows) + (static_cast<size_t>(ids[k]) * a.Hkv + h) * ROW;
+            src[k] = static_cast<const unsigned char*>(a.rows) + (static_cast<size_t>(h) * a.num_phys + ids[k]) * ROW;
             bytes += ROW;
           }
         }
@@ -449,7 +453,15 @@ struct DirectOcc {
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::value)
     meta_direct_kernel(StreamArgs a) {
-  grid_dep_enter();
+  // With defer_wait the kernel overlaps the append that precedes it: tiles
+  // without a sequence's last page never read what the append writes, so
+  // only a warp about to load such a tile waits for the append to finish.
+  if (a.defer_wait) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  } else {
+    grid_dep_enter();
+  }
+  bool waited = a.defer_wait == 0;
   constexpr int KP = 2 * D / 32;              // 32-element chunks per row
   constexpr int NT = Cols<G, GAUSS>::tiles;   // 8-column tiles of the B operand
   constexpr int ROW = 2 * D * 2;              // bytes per metadata row
@@ -479,43 +491,66 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
   const long long t0 = total * gw / nw, t1 = total * (gw + 1) / nw;
   if (t0 >= t1) return;
 
-  // tile index → (sequence, KV head, first page, rows, sequence length)
-  auto locate = [&](long long ti, int& b, int& h, int& p0, int& n, int& L) {
+  // Tile cursor: tiles of a sequence run KV head by KV head, 16 pages each;
+  // the first tile is found by search, later ones by stepping (no division
+  // per tile).
+  struct Cursor {
+    int b, h, p0, P, L;
+  };
+  auto seek = [&](long long ti, Cursor& c) {
     int lo = 0, hi = a.batch;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (prefix[mid] <= ti) lo = mid; else hi = mid;
     }
-    b = lo;
-    const int P = seq_pages(a.seq_lens, b, a.S, a.max_pages, &L);
-    const int tpu = (P + kTile - 1) / kTile;
-    const long long r = ti - prefix[b];
-    h = static_cast<int>(r / tpu);
-    p0 = static_cast<int>(r % tpu) * kTile;
-    n = min(kTile, P - p0);
+    c.b = lo;
+    c.P = seq_pages(a.seq_lens, c.b, a.S, a.max_pages, &c.L);
+    const int tpu = (c.P + kTile - 1) / kTile;
+    const int r = static_cast<int>(ti - prefix[c.b]);
+    c.h = r / tpu;
+    c.p0 = (r - c.h * tpu) * kTile;
   };
-  auto load_ids = [&](int b, int p0, int n) -> int {
-    return lane < n ? a.page_table[static_cast<size_t>(b) * a.max_pages + p0 + lane] : -1;
+  auto step = [&](Cursor& c) {
+    c.p0 += kTile;
+    if (c.p0 >= c.P) {
+      c.p0 = 0;
+      if (++c.h == a.Hkv) {
+        c.h = 0;
+        do {
+          ++c.b;
+          c.P = c.b < a.batch ? seq_pages(a.seq_lens, c.b, a.S, a.max_pages, &c.L) : 1;
+        } while (c.P == 0);
+      }
+    }
+  };
+  auto load_ids = [&](const Cursor& c) -> int {
+    const int n = min(kTile, c.P - c.p0);
+    return lane < n ? a.page_table[static_cast<size_t>(c.b) * a.max_pages + c.p0 + lane] : -1;
   };
 
   uint32_t bfrag[2 * KP][NT][2];
   int cur_unit = -1;
   float* my_tile = ctile + warp * 16 * 24;
-  int b, h, p0, n, L;
-  locate(t0, b, h, p0, n, L);
-  int ids = load_ids(b, p0, n);
+  Cursor cur;
+  seek(t0, cur);
+  int ids = load_ids(cur);
   for (long long ti = t0; ti < t1; ++ti) {
+    const int b = cur.b, h = cur.h, p0 = cur.p0, L = cur.L;
+    const int n = min(kTile, cur.P - p0);
     const int unit = b * a.Hkv + h;
+    if (!waited && p0 + n == cur.P) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      waited = true;
+    }
     const int id_lo = __shfl_sync(0xffffffffu, ids, g), id_hi = __shfl_sync(0xffffffffu, ids, g + 8);
     const bool ok_lo = g < n && id_lo >= 0 && id_lo < a.num_phys;
     const bool ok_hi = g + 8 < n && id_hi >= 0 && id_hi < a.num_phys;
     if ((g < n && !ok_lo) || (g + 8 < n && !ok_hi)) raise_flag(EKV_EFLAG_BAD_PAGE);
     // bit r: row r of the tile exists and has a valid page
     const unsigned int live_mask = __ballot_sync(0xffffffffu, lane < n && ids >= 0 && ids < a.num_phys);
-    const uint4* row_lo = reinterpret_cast<const uint4*>(
-        static_cast<const unsigned char*>(a.rows) + (static_cast<size_t>(ok_lo ? id_lo : 0) * a.Hkv + h) * ROW) + t;
-    const uint4* row_hi = reinterpret_cast<const uint4*>(
-        static_cast<const unsigned char*>(a.rows) + (static_cast<size_t>(ok_hi ? id_hi : 0) * a.Hkv + h) * ROW) + t;
+    const unsigned char* hrows = static_cast<const unsigned char*>(a.rows) + static_cast<size_t>(h) * a.num_phys * ROW;
+    const uint4* row_lo = reinterpret_cast<const uint4*>(hrows + static_cast<size_t>(ok_lo ? id_lo : 0) * ROW) + t;
+    const uint4* row_hi = reinterpret_cast<const uint4*>(hrows + static_cast<size_t>(ok_hi ? id_hi : 0) * ROW) + t;
     uint4 va[KP], vb[KP];
 #pragma unroll
     for (int c = 0; c < KP; ++c) {
@@ -523,10 +558,9 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
       vb[c] = ok_hi ? __ldcs(row_hi + 4 * c) : make_uint4(0, 0, 0, 0);
     }
     // next tile's page ids travel while this tile's rows do
-    int nb = b, nh = h, np0 = p0, nn = n, nL = L;
     if (ti + 1 < t1) {
-      locate(ti + 1, nb, nh, np0, nn, nL);
-      ids = load_ids(nb, np0, nn);
+      step(cur);
+      ids = load_ids(cur);
     }
     if (unit != cur_unit) {
       cur_unit = unit;
@@ -617,7 +651,6 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
       }
       __syncwarp();
     }
-    b = nb; h = nh; p0 = np0; n = nn; L = nL;
   }
 }
 
@@ -696,8 +729,9 @@ StreamArgs base_args(const ekv_cache& c, const ekv_seqs& s, const void* q, int H
 }  // namespace
 
 cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq, float scale,
-                         float* ub, cudaStream_t st) {
+                         float* ub, cudaStream_t st, int after_append) {
   StreamArgs a = base_args(c, s, q, Hq, scale);
+  a.defer_wait = after_append;
   a.rows = c.box;
   a.ub = ub;
   const int G = Hq / c.num_kv_heads;
@@ -706,8 +740,10 @@ cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, i
 }
 
 cudaError_t launch_gauss_stats(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
-                               float scale, float alpha, const GaussWs& ws, cudaStream_t st) {
+                               float scale, float alpha, const GaussWs& ws, cudaStream_t st,
+                               int after_append) {
   StreamArgs a = base_args(c, s, q, Hq, scale);
+  a.defer_wait = after_append;
   a.rows = c.mom;
   a.gws = ws;
   a.am1 = alpha - 1.0f;

@@ -25,7 +25,7 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kSmemKeys = 16384;
 constexpr int kBins = 4096;
 constexpr int kDigitBits = 12;
-constexpr int kBinsPerThread = kBins / kTopkThreads;
+constexpr int kRankMax = 256;  // keys of the k-th key's bin ranked directly
 
 __global__ void __launch_bounds__(kTopkThreads)
     topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
@@ -35,7 +35,9 @@ __global__ void __launch_bounds__(kTopkThreads)
   extern __shared__ uint32_t keys_s[];  // [min(max_pages, kSmemKeys)]
   __shared__ unsigned int hist[2][kBins];
   __shared__ unsigned int w_a[kTopkWarps], w_b[kTopkWarps];
-  __shared__ unsigned int s_lo, s_hi, s_above;
+  __shared__ uint32_t rk_key[kRankMax];
+  __shared__ int rk_idx[kRankMax];
+  __shared__ unsigned int s_lo, s_hi, s_above, s_count, s_fill;
 
   const int unit = blockIdx.x, b = unit / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -77,7 +79,8 @@ __global__ void __launch_bounds__(kTopkThreads)
   auto key_at = [&](int i) -> uint32_t { return cached ? keys_s[i] : float_key(row[i]); };
 
   // The interval [lo, hi] holds the k-th largest key; krem of its keys are
-  // still to be taken.  Each pass splits it into ≤ 4096 equal bins.
+  // still to be taken.  Each pass splits it into ≤ 4096 equal bins; once the
+  // bin of the k-th key holds few keys, they are ranked directly.
   unsigned int lo = kmin, hi = kmax, krem = static_cast<unsigned int>(k);
   int cur = 0;
   for (int pass = 0; pass < 4 && lo < hi; ++pass) {
@@ -102,101 +105,137 @@ __global__ void __launch_bounds__(kTopkThreads)
     }
     for (int i = tid; i < kBins; i += kTopkThreads) hist[cur ^ 1][i] = 0u;  // next pass's bins
     __syncthreads();
-    // thread t owns `per` consecutive bins counted from the top
-    const int per = (nbins + kTopkThreads - 1) / kTopkThreads;
-    unsigned int c[kBinsPerThread], local = 0u;
+    // warp w covers bins top − 128w − 32r − lane (r = 0..3), counted from the top
+    const int top = nbins - 1;
+    unsigned int wsum = 0u;
 #pragma unroll
-    for (int r = 0; r < kBinsPerThread; ++r) {
-      const int bin = nbins - 1 - per * tid - r;
-      c[r] = (r < per && bin >= 0) ? hc[bin] : 0u;
-      local += c[r];
+    for (int r = 0; r < kBins / kTopkThreads; ++r) {
+      const int bin = top - 128 * warp - 32 * r - lane;
+      wsum += bin >= 0 ? hc[bin] : 0u;
     }
-    unsigned int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) w_a[warp] = incl;
+    wsum = __reduce_add_sync(0xffffffffu, wsum);
+    if (lane == 0) w_a[warp] = wsum;
     __syncthreads();
-    unsigned int wt = w_a[lane], wincl = wt;
+    const unsigned int wt = w_a[lane];
+    unsigned int wincl = wt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned int y = __shfl_up_sync(0xffffffffu, wincl, o);
       if (lane >= o) wincl += y;
     }
-    const unsigned int warp_before = __shfl_sync(0xffffffffu, wincl - wt, warp);
-    const unsigned int before = warp_before + incl - local;
-    if (local > 0 && before < krem && before + local >= krem) {
-      unsigned int acc = before;
-      int r = 0;
-      while (r < per - 1 && acc + c[r] < krem) acc += c[r++];
-      const unsigned int bin = static_cast<unsigned int>(nbins - 1 - per * tid - r);
-      s_above = acc;
-      const unsigned long long base = static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bin) << shift);
-      s_lo = static_cast<unsigned int>(base);
-      s_hi = static_cast<unsigned int>(min(static_cast<unsigned long long>(hi), base + ((1ull << shift) - 1ull)));
+    unsigned int before = __shfl_sync(0xffffffffu, wincl - wt, warp);
+    const unsigned int mine = __shfl_sync(0xffffffffu, wt, warp);
+    if (before < krem && before + mine >= krem) {  // this warp holds the k-th key's bin
+#pragma unroll 1
+      for (int r = 0; r < kBins / kTopkThreads; ++r) {
+        const int bin = top - 128 * warp - 32 * r - lane;
+        const unsigned int c = bin >= 0 ? hc[bin] : 0u;
+        unsigned int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (c > 0 && before + incl - c < krem && before + incl >= krem) {
+          s_above = before + incl - c;
+          s_count = c;
+          s_fill = 0u;
+          const unsigned long long base = static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bin) << shift);
+          s_lo = static_cast<unsigned int>(base);
+          s_hi = static_cast<unsigned int>(min(static_cast<unsigned long long>(hi), base + ((1ull << shift) - 1ull)));
+        }
+        before += __shfl_sync(0xffffffffu, incl, 31);
+        if (before >= krem) break;
+      }
     }
     __syncthreads();
     krem -= s_above;
     lo = s_lo;
     hi = s_hi;
     cur ^= 1;
+    const unsigned int cnt = s_count;
+    if (lo < hi && cnt <= kRankMax) {
+      // rank the bin's keys by (key descending, page ascending): the one of
+      // rank krem − 1 is K*; of the keys equal to K*, krem − #{key > K*} go
+      for (int base = 0; base < P; base += kTopkThreads) {
+        const int i = base + tid;
+        if (i < P) {
+          const uint32_t key = key_at(i);
+          if (key >= lo && key <= hi) {
+            const unsigned int pos = atomicAdd(&s_fill, 1u);
+            rk_key[pos] = key;
+            rk_idx[pos] = i;
+          }
+        }
+      }
+      __syncthreads();
+      if (tid < static_cast<int>(cnt)) {
+        const uint32_t key = rk_key[tid];
+        const int idx = rk_idx[tid];
+        unsigned int rank = 0u, greater = 0u;
+        for (unsigned int c = 0; c < cnt; ++c) {
+          const uint32_t kc = rk_key[c];
+          greater += kc > key ? 1u : 0u;
+          rank += (kc > key || (kc == key && rk_idx[c] < idx)) ? 1u : 0u;
+        }
+        if (rank == krem - 1u) {
+          s_lo = key;
+          s_above = greater;
+        }
+      }
+      __syncthreads();
+      lo = hi = s_lo;
+      krem -= s_above;
+      break;
+    }
   }
 
-  // Output: contiguous runs per thread keep the ascending page order.  The
-  // selected pages are every key > K* and the first krem keys equal to K*;
-  // an element's position = #greater before it + min(#equal before it, krem).
+  // Output in ascending page order: warp w walks its chunk of pages with
+  // ballots; a taken page's slot = #{greater before} + min(#{equal before}, krem).
   const uint32_t kth = lo;
-  const int run = (P + kTopkThreads - 1) / kTopkThreads;
-  const int i0 = min(P, tid * run), i1 = min(P, i0 + run);
-  unsigned int n_gt = 0, n_eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    n_gt += key > kth ? 1u : 0u;
-    n_eq += key == kth ? 1u : 0u;
-  }
-  unsigned int g_incl = n_gt, e_incl = n_eq;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned int yg = __shfl_up_sync(0xffffffffu, g_incl, o);
-    const unsigned int ye = __shfl_up_sync(0xffffffffu, e_incl, o);
-    if (lane >= o) {
-      g_incl += yg;
-      e_incl += ye;
-    }
+  const int cw = (((P + kTopkWarps - 1) / kTopkWarps) + 31) & ~31;
+  const int c0 = warp * cw, c1 = min(P, c0 + cw);
+  unsigned int ng = 0u, ne = 0u;
+  for (int i0 = c0; i0 < c1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < c1 ? key_at(i) : 0u;
+    ng += __popc(__ballot_sync(0xffffffffu, i < c1 && key > kth));
+    ne += __popc(__ballot_sync(0xffffffffu, i < c1 && key == kth));
   }
   __syncthreads();  // w_a / w_b were read above
-  if (lane == 31) {
-    w_a[warp] = g_incl;
-    w_b[warp] = e_incl;
+  if (lane == 0) {
+    w_a[warp] = ng;
+    w_b[warp] = ne;
   }
   __syncthreads();
-  unsigned int wg = w_a[lane], we = w_b[lane], wg_incl = wg, we_incl = we;
+  unsigned int xg = w_a[lane], xe = w_b[lane], ig = xg, ie = xe;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned int yg = __shfl_up_sync(0xffffffffu, wg_incl, o);
-    const unsigned int ye = __shfl_up_sync(0xffffffffu, we_incl, o);
+    const unsigned int yg = __shfl_up_sync(0xffffffffu, ig, o);
+    const unsigned int ye = __shfl_up_sync(0xffffffffu, ie, o);
     if (lane >= o) {
-      wg_incl += yg;
-      we_incl += ye;
+      ig += yg;
+      ie += ye;
     }
   }
-  unsigned int gt_before = __shfl_sync(0xffffffffu, wg_incl - wg, warp) + g_incl - n_gt;
-  unsigned int eq_before = __shfl_sync(0xffffffffu, we_incl - we, warp) + e_incl - n_eq;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    if (key > kth) {
-      const unsigned int pos = gt_before + min(eq_before, krem);
+  unsigned int gt_before = __shfl_sync(0xffffffffu, ig - xg, warp);
+  unsigned int eq_before = __shfl_sync(0xffffffffu, ie - xe, warp);
+  const unsigned int lower = (1u << lane) - 1u;
+  for (int i0 = c0; i0 < c1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < c1 ? key_at(i) : 0u;
+    const bool gt = i < c1 && key > kth, eq = i < c1 && key == kth;
+    const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const unsigned int my_g = gt_before + __popc(bg & lower), my_e = eq_before + __popc(be & lower);
+    if (gt) {
+      const unsigned int pos = my_g + min(my_e, krem);
       if (pos < static_cast<unsigned int>(k)) out[pos] = i;
-      ++gt_before;
-    } else if (key == kth) {
-      if (eq_before < krem) {
-        const unsigned int pos = gt_before + eq_before;
-        if (pos < static_cast<unsigned int>(k)) out[pos] = i;
-      }
-      ++eq_before;
+    } else if (eq && my_e < krem) {
+      const unsigned int pos = my_g + my_e;
+      if (pos < static_cast<unsigned int>(k)) out[pos] = i;
     }
+    gt_before += __popc(bg);
+    eq_before += __popc(be);
   }
   if (tid == 0) n_sel[unit] = k;
 }
@@ -207,7 +246,7 @@ cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int 
                         int32_t* sel, int32_t* n_sel, cudaStream_t st) {
   const int keys = s.max_pages < kSmemKeys ? s.max_pages : kSmemKeys;
   const size_t smem = static_cast<size_t>(keys) * sizeof(uint32_t);
-  const size_t static_smem = 2 * kBins * sizeof(unsigned int) + 256;
+  const size_t static_smem = 2 * kBins * sizeof(unsigned int) + kRankMax * 8 + 512;
   if (smem + static_smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));

@@ -60,8 +60,8 @@ def test_metadata_bit_exact(case):
         for h in range(wl.num_kv_heads):
             meta = O.page_metadata(np64(inp["k_pool"][torch.as_tensor(phys).cuda(), h]), n_valid, wl.dtype)
             tdt = box.dtype
-            got_box = _bits(box[torch.as_tensor(phys).cuda(), h], wl.dtype)
-            got_mom = _bits(mom[torch.as_tensor(phys).cuda(), h], wl.dtype)
+            got_box = _bits(box[h, torch.as_tensor(phys).cuda()], wl.dtype)
+            got_mom = _bits(mom[h, torch.as_tensor(phys).cuda()], wl.dtype)
             want_box = _bits(torch.from_numpy(np.stack([meta["kmax"], meta["kmin"]], 1)).to(tdt), wl.dtype)
             want_mom = _bits(torch.from_numpy(np.stack([meta["mean"], meta["var"]], 1)).to(tdt), wl.dtype)
             assert np.array_equal(got_box, want_box), (b, h)
