@@ -39,10 +39,16 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one score-kernel launch at the default workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of
 # the kernel's sources; stale entries read as null.
-SCORE_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture
+# of the bench workload's shape, keyed by a hash of the kernel's sources (a
+# changed kernel has no measured traffic until it is captured again)
+SCORE_FILES = ("score.cu", "common.cuh", "kernels.cuh")
+DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh", "kernels.cuh")
+SCORE_TRAFFIC = {"20c008979d406865": 138512128}   # profiles/score_kernel_clustered_128k.md
+DECODE_TRAFFIC = {"c11b559320073018": 57956352}   # profiles/fused_decode_kernel_clustered_128k.md
 
 
-def kernel_hash(files=("score.cu", "common.cuh", "kernels.cuh")):
+def kernel_hash(files=SCORE_FILES):
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "sparse_kv_cache_kmax_b200", "csrc", f), "rb") as fh:
@@ -151,9 +157,12 @@ class L2Flush:
 
 
 # ---------------------------------------------------------------- bytes
-def algorithmic_bytes(inp, eng, support_pages):
+def algorithmic_bytes(inp, eng, support_pages, support_tokens):
     """Bytes one step must move: metadata rows, q, ub, selected K, V of
-    support pages, outputs, and the append (tail page + new rows + metadata)."""
+    support pages, outputs, and the append (tail page + new rows + metadata).
+    The decode kernel's own bytes count V token by token (the union of the
+    group heads' support), as the method needs them; the kernel reads whole
+    support pages, which the measured traffic shows."""
     wl = inp["workload"]
     es = inp["k_pool"].element_size()
     d, S, G = wl.head_dim, wl.page_size, wl.group
@@ -169,8 +178,10 @@ def algorithmic_bytes(inp, eng, support_pages):
     supV = int(support_pages) * S * d * es
     out = wl.batch * wl.num_q_heads * d * 4
     append = wl.units * (S * d * es + 2 * d * es + 4 * d * es)
+    supV_tok = int(support_tokens) * d * es
     return {"meta": meta, "q": q, "ub": ub, "sel_k": selK, "support_v": supV, "out": out,
             "append": append, "score_kernel": meta + q + ub,
+            "decode_kernel": selK + supV_tok + q + out,
             "step": meta + q + selK + supV + out + append}
 
 
@@ -269,13 +280,24 @@ def run_ours(args):
     tok = tok.view(wl.batch, wl.num_kv_heads, wl.group, -1).amax(dim=2)          # union over the group
     page_sup = tok.view(wl.batch, wl.num_kv_heads, k, wl.page_size).amax(dim=-1)
     support_pages = int(page_sup.sum())
-    nb = algorithmic_bytes(inp, eng, support_pages)
+    support_tokens = int(tok.sum())
+    nb = algorithmic_bytes(inp, eng, support_pages, support_tokens)
 
+    # per-kernel rooflines from the staged timing; the headline one is the
+    # kernel with the largest time (the launch list's largest share)
     peak, peak_kind = hbm_peak()
-    score_ms = float(stages[1])
-    achieved = nb["score_kernel"] / (score_ms * 1e-3) / 1e9
-    h = kernel_hash()
-    traffic = SCORE_TRAFFIC.get(h)
+    kern = {}
+    for name, idx, key, table, files in (("score", 1, "score_kernel", SCORE_TRAFFIC, SCORE_FILES),
+                                         ("decode", 3, "decode_kernel", DECODE_TRAFFIC, DECODE_FILES)):
+        ms = float(stages[idx])
+        ach = nb[key] / (ms * 1e-3) / 1e9
+        kern[name] = {"us": ms * 1e3, "algorithmic_bytes": nb[key], "achieved": ach, "frac": ach / peak,
+                      "traffic": table.get(kernel_hash(files))}
+    kern["topk"] = {"us": float(stages[2]) * 1e3, "bound": "latency (1 MiB of scores)"}
+    kern["append"] = {"us": float(stages[0]) * 1e3, "bound": "latency (one page per unit)"}
+    dom = max(("score", "decode"), key=lambda n: kern[n]["us"])
+    dom_name = {"score": "score (bounding-box page scores)",
+                "decode": "decode (fused: scores on selected K, tau, support V)"}[dom]
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -289,16 +311,17 @@ def run_ours(args):
         "stages_us": {"append": stages[0] * 1e3, "score": stages[1] * 1e3, "topk": stages[2] * 1e3,
                       "decode": stages[3] * 1e3, "sum": float(stages.sum()) * 1e3,
                       "note": "separate calls with events between stages (no launch overlap)"},
-        "roofline": {"bound": "hbm", "kernel": "score (bounding-box page scores)", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
-                     "algorithmic_bytes": nb["score_kernel"]},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": kern[dom]["achieved"],
+                     "peak": peak, "unit": "GB/s", "frac": kern[dom]["frac"],
+                     "peak_kind": f"{peak_kind} copy bandwidth", "traffic": kern[dom]["traffic"],
+                     "algorithmic_bytes": kern[dom]["algorithmic_bytes"]},
+        "kernels": kern,
         "step_roofline": {"bytes": nb["step"], "achieved_gbs": nb["step"] / (step_ms * 1e-3) / 1e9,
                           "frac": nb["step"] / (step_ms * 1e-3) / 1e9 / peak,
                           "breakdown": {kk: v for kk, v in nb.items() if kk not in ("step", "score_kernel")}},
         "support": {"mean_sel_pages": float(eng.n_sel.float().mean()), "support_pages_per_unit":
                     support_pages / wl.units, "mean_support_tokens_per_head": float(cnt.float().mean())},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": Bd.ekv_step_kernel_count(cache, seqs, eng.params, Hq) * args.steps,
         "clocks": clocks,
     }
 

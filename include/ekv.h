@@ -251,6 +251,16 @@ typedef enum {
 EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv_seqs* seqs,
                                    int32_t num_q_heads, int32_t cap);
 
+/*
+ * ekv_step_kernel_count — how many kernels one ekv_decode_step call with these
+ * arguments enqueues: the append (if params->append), the selection (2 for
+ * top-k, 3 for the Gaussian policy, 0 for every page) and the decode (1 when
+ * a bf16 selection fits the one-cluster-per-unit kernel, else 3).  Host-side
+ * only; returns 0 when the sizes are invalid.
+ */
+EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* seqs,
+                                      const ekv_step_params* params, int32_t num_q_heads);
+
 /* Reads the sticky device error word into *flags (EKV_EFLAG_* bits) and clears
  * it.  Synchronises the device. */
 EKV_API ekv_status ekv_get_error(uint32_t* flags);

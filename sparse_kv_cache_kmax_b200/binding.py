@@ -20,7 +20,7 @@ __all__ = [
     "make_cache", "make_seqs", "workspace", "ekv_build_page_meta", "ekv_append",
     "ekv_score_pages", "ekv_select_topk", "ekv_select_gauss", "ekv_entmax_decode",
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
-    "ekv_entmax_decode_static_ws",
+    "ekv_entmax_decode_static_ws", "ekv_step_kernel_count",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
@@ -76,6 +76,7 @@ _SIGS = {
     "ekv_decode_step": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams),
                         _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "ekv_workspace_bytes": [_I, ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _I, _I],
+    "ekv_step_kernel_count": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams), _I],
     "ekv_entmax_decode_static_ws": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P,
                                     _P, _I, _I, _P, _P, _P, _P, _P],
     "ekv_get_error": [ctypes.POINTER(ctypes.c_uint32)],
@@ -206,6 +207,12 @@ def ekv_decode_step(cache, seqs, params: StepParams, q, k_new, v_new, sel, n_sel
         ctypes.byref(cache), ctypes.byref(seqs), ctypes.byref(params), _ptr(q), q.shape[1],
         _ptr(k_new), _ptr(v_new), _ptr(sel), _ptr(n_sel), _ptr(out), _ptr(tau), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def ekv_step_kernel_count(cache, seqs, params: StepParams, num_q_heads) -> int:
+    """Kernels one ekv_decode_step call with these arguments enqueues."""
+    return int(lib().ekv_step_kernel_count(ctypes.byref(cache), ctypes.byref(seqs), ctypes.byref(params),
+                                           num_q_heads))
 
 
 def ekv_entmax_decode_static_ws(cache, seqs, q, scale, alpha, sel, n_sel, cap, out, *, dense_v=False,

@@ -293,6 +293,21 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
   }
 }
 
+EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* seqs,
+                                      const ekv_step_params* p, int32_t num_q_heads) {
+  if (p == nullptr || check_cache(cache, false, false) != EKV_OK || seqs == nullptr ||
+      seqs->batch < 1 || seqs->max_pages < 1 || check_heads(cache, num_q_heads) != EKV_OK)
+    return 0;
+  const bool full = p->policy == EKV_POLICY_FULL;
+  const int cap = full ? seqs->max_pages : p->cap;
+  if (cap < 1) return 0;
+  int n = p->append ? 1 : 0;
+  if (p->policy == EKV_POLICY_TOPK) n += 2;
+  else if (p->policy == EKV_POLICY_GAUSS) n += 3;
+  else if (!full) return 0;
+  return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap);
+}
+
 EKV_API ekv_status ekv_get_error(uint32_t* flags) {
   if (flags == nullptr) return EKV_ERR_INVALID_ARG;
   unsigned int v = 0u, zero = 0u;

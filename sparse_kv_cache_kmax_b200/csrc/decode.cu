@@ -631,6 +631,17 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
 
 }  // namespace
 
+int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap) {
+  const int G = Hq / c.num_kv_heads, U = s.batch * c.num_kv_heads;
+  if (c.dtype != EKV_BF16 || U > 65535) return 3;
+#define EKV_CNT_CASE(DD, GG) \
+  if (c.head_dim == DD && G == GG) return fused_decode_fits<DD, GG>(U, cap, c.page_size) ? 1 : 3;
+  EKV_CNT_CASE(128, 1) EKV_CNT_CASE(128, 2) EKV_CNT_CASE(128, 4) EKV_CNT_CASE(128, 8) EKV_CNT_CASE(128, 16)
+  EKV_CNT_CASE(64, 1) EKV_CNT_CASE(64, 2) EKV_CNT_CASE(64, 4) EKV_CNT_CASE(64, 8) EKV_CNT_CASE(64, 16)
+#undef EKV_CNT_CASE
+  return 3;
+}
+
 cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
                           float scale, float alpha, const int32_t* sel, const int32_t* n_sel,
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,

@@ -171,6 +171,94 @@ __device__ __forceinline__ double closed_tau(int ipow, double c, double s1, doub
   return M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
 }
 
+// Rare paths of cta_solve_tau, kept out of line so that the common path's
+// code stays compact (code that runs once per CTA is fetched, not cached).
+
+// Repeats the closed form on {u > τ} until the support is stable.
+__device__ __noinline__ double repair_closed_tau(const float* cand, int nc, int ipow, double tau,
+                                                  TauShared& sh) {
+  const int tid = threadIdx.x;
+  for (int rep = 0; rep < 8; ++rep) {
+    double c = 0.0, s1 = 0.0, s2 = 0.0;
+    for (int i = tid; i < nc; i += kFThreads) {
+      const double u = cand[i];
+      if (u > tau) {
+        c += 1.0;
+        s1 += u;
+        s2 += u * u;
+      }
+    }
+    cta_sum3(c, s1, s2, sh);
+    if (c < 1.0) break;
+    const double t_new = closed_tau(ipow, c, s1, s2);
+    if (t_new == tau) break;
+    tau = t_new;
+  }
+  return tau;
+}
+
+// Newton's method from the left in fp32 (f is convex and decreasing), then a
+// float64 finish: the closed form for β ∈ {1,2}, one Newton step otherwise.
+__device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_lo, float um,
+                                          float beta, int ipow, TauShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool closed = ipow == 1 || ipow == 2;
+  double tau;
+  const bool solo = nc <= 1024;
+  if (!solo || warp == 0) {
+    float t = static_cast<float>(tau_lo);
+    if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
+    int par = 1;
+    for (int it = 0; it < 64; ++it) {
+      float f, df;
+      par ^= 1;
+      f_df<float>(cand, nc, t, beta, ipow, solo, sh, par, f, df);
+      if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
+        t = um - 1.0f;
+        continue;
+      }
+      const float step = f / (beta * df);
+      if (!(step > 0.0f)) break;
+      t += step;
+      if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+    }
+    double tt = t;
+    if (closed) {
+      for (int rep = 0; rep < 4; ++rep) {
+        double c = 0.0, s1 = 0.0, s2 = 0.0;
+        for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
+          const double u = cand[i];
+          if (u > tt) {
+            c += 1.0;
+            s1 += u;
+            s2 += u * u;
+          }
+        }
+        if (solo) {
+          c = warp_sum(c);
+          s1 = warp_sum(s1);
+          s2 = warp_sum(s2);
+        } else {
+          cta_sum3(c, s1, s2, sh);
+        }
+        if (c < 1.0) break;
+        const double t_new = closed_tau(ipow, c, s1, s2);
+        if (t_new == tt) break;
+        tt = t_new;
+      }
+    } else {
+      double f, df;
+      f_df<double>(cand, nc, tt, static_cast<double>(beta), ipow, solo, sh, 0, f, df);
+      if (df > 0.0) tt += f / (static_cast<double>(beta) * df);
+    }
+    if (tid == 0) sh.tau = tt;
+  }
+  __syncthreads();
+  tau = sh.tau;
+  __syncthreads();
+  return tau;
+}
+
 // τ of one query head: Σ_i [u_i − τ]_+^β = 1, u_i = (α−1)·z_i, over the n
 // scores z[0..n) in shared memory whose histogram over (um − 1, um] (um =
 // (α−1)·max z, 256 bins from the top) is in sh.hist.  The whole CTA calls it;
@@ -208,7 +296,7 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     const int before = incl - tot;
     // c^(−1/β) without libm: exact-enough reciprocals for β ∈ {1,2}, fast
     // exp2/log2 otherwise; the slack below keeps τ_lo a lower bound
-#pragma unroll 1
+#pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int c = before + cnt[k];
       if (c > 0) {
@@ -220,13 +308,16 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     cb = warp_max(cb);
   }
   const double tau_lo = static_cast<double>(cb) - 4e-6 * (1.0 + fabs(static_cast<double>(um)));
+  // fp32 copy rounded down: comparisons against it stay on the safe side
+  float tau_lo_f = static_cast<float>(tau_lo);
+  if (static_cast<double>(tau_lo_f) > tau_lo) tau_lo_f = nextafterf(tau_lo_f, -INFINITY);
   // 2. compaction: warp w takes elements k·512 + 32w + lane; order (w, k, lane)
   int nc;
   {
     int mine = 0;
     for (int base = 0; base < n; base += kFThreads) {
       const int i = base + tid;
-      const bool in = i < n && static_cast<double>(am1 * z[i]) > tau_lo;
+      const bool in = i < n && am1 * z[i] > tau_lo_f;
       mine += __popc(__ballot_sync(0xffffffffu, in));
     }
     if (lane == 0) sh.i[warp] = mine;
@@ -242,7 +333,7 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     for (int base = 0; base < n; base += kFThreads) {
       const int i = base + tid;
       const float u = i < n ? am1 * z[i] : -INFINITY;
-      const bool in = i < n && static_cast<double>(u) > tau_lo;
+      const bool in = i < n && u > tau_lo_f;
       const unsigned int bal = __ballot_sync(0xffffffffu, in);
       if (in) cand[pos + __popc(bal & ((1u << lane) - 1u))] = u;
       pos += __popc(bal);
@@ -275,77 +366,9 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     cta_sum3(c, s1, s2, sh);
     tau = closed_tau(ipow, c, s1, s2);
     const bool bad = tid < nc && (in != (static_cast<double>(ut) > tau));
-    if (__syncthreads_or(bad)) {
-      for (int rep = 0; rep < 8; ++rep) {
-        c = s1 = s2 = 0.0;
-        for (int i = tid; i < nc; i += kFThreads) {
-          const double u = cand[i];
-          if (u > tau) {
-            c += 1.0;
-            s1 += u;
-            s2 += u * u;
-          }
-        }
-        cta_sum3(c, s1, s2, sh);
-        if (c < 1.0) break;
-        const double t_new = closed_tau(ipow, c, s1, s2);
-        if (t_new == tau) break;
-        tau = t_new;
-      }
-    }
+    if (__syncthreads_or(bad)) tau = repair_closed_tau(cand, nc, ipow, tau, sh);
   } else {
-    const bool solo = nc <= 1024;
-    if (!solo || warp == 0) {
-      float t = static_cast<float>(tau_lo);
-      if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
-      int par = 1;
-      for (int it = 0; it < 64; ++it) {
-        float f, df;
-        par ^= 1;
-        f_df<float>(cand, nc, t, beta, ipow, solo, sh, par, f, df);
-        if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
-          t = um - 1.0f;
-          continue;
-        }
-        const float step = f / (beta * df);
-        if (!(step > 0.0f)) break;
-        t += step;
-        if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
-      }
-      double tt = t;
-      if (closed) {
-        for (int rep = 0; rep < 4; ++rep) {
-          double c = 0.0, s1 = 0.0, s2 = 0.0;
-          for (int i = solo ? lane : tid; i < nc; i += solo ? 32 : kFThreads) {
-            const double u = cand[i];
-            if (u > tt) {
-              c += 1.0;
-              s1 += u;
-              s2 += u * u;
-            }
-          }
-          if (solo) {
-            c = warp_sum(c);
-            s1 = warp_sum(s1);
-            s2 = warp_sum(s2);
-          } else {
-            cta_sum3(c, s1, s2, sh);
-          }
-          if (c < 1.0) break;
-          const double t_new = closed_tau(ipow, c, s1, s2);
-          if (t_new == tt) break;
-          tt = t_new;
-        }
-      } else {
-        double f, df;
-        f_df<double>(cand, nc, tt, static_cast<double>(beta), ipow, solo, sh, 0, f, df);
-        if (df > 0.0) tt += f / (static_cast<double>(beta) * df);
-      }
-      if (tid == 0) sh.tau = tt;
-    }
-    __syncthreads();
-    tau = sh.tau;
-    __syncthreads();
+    tau = newton_tau(cand, nc, tau_lo, um, beta, ipow, sh);
   }
   return static_cast<float>(tau);
 }

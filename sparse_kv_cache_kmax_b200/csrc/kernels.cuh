@@ -49,6 +49,9 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
                           uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st);
 
+// Kernels one launch_decode enqueues for these sizes (1 fused, or 3).
+int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap);
+
 // Score-pass CTAs per unit: cap pages of S tokens, 256 tokens per CTA.
 inline int qk_splits(int cap, int S) {
   const int pages = kQkTokensPerCta / S;

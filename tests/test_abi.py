@@ -107,3 +107,19 @@ def test_workspace_sizes_are_host_only_and_monotone():
 def test_valid_call_without_a_device_reports_cuda_error():
     c, s = _cache(), _seqs()
     assert _decode(c, s) == 4
+
+
+def test_step_kernel_count_host_side():
+    L = B.lib()
+    c, s = _cache(), _seqs()
+    assert L.ekv_step_kernel_count(ctypes.byref(c), ctypes.byref(s), None, 32) == 0
+    assert L.ekv_step_kernel_count(ctypes.byref(c), ctypes.byref(s),
+                                   ctypes.byref(B.StepParams(9, 4, 0.5, 4, 1.5, 0.1, 0, 1)), 32) == 0
+    assert L.ekv_step_kernel_count(ctypes.byref(c), ctypes.byref(s),
+                                   ctypes.byref(B.StepParams(B.EKV_POLICY_TOPK, 4, 0.5, 4, 1.5, 0.1, 0, 1)), 24) == 0
+    # fp32 caches never take the fused decode: append + score + top-k + 3 decode kernels
+    f32 = _cache(dtype=B.EKV_F32)
+    topk = B.StepParams(B.EKV_POLICY_TOPK, 4, 0.5, 4, 1.5, 0.1, 0, 1)
+    assert L.ekv_step_kernel_count(ctypes.byref(f32), ctypes.byref(s), ctypes.byref(topk), 32) == 6
+    full = B.StepParams(B.EKV_POLICY_FULL, 0, 0.5, 4, 1.5, 0.1, 0, 0)
+    assert L.ekv_step_kernel_count(ctypes.byref(f32), ctypes.byref(s), ctypes.byref(full), 32) == 3
