@@ -445,3 +445,44 @@ def test_threshold_monotone_and_bound_certificate(alpha):
             certified += 1
             assert np.allclose(sparse["o"][h], full["o"][h], atol=1e-12)
     assert certified > 0
+
+
+# ---------------------------------------------------------------- softmax attention (full-cache baseline)
+def test_softmax_attention_matches_scipy_and_two_token_closed_form():
+    """The dense softmax decode of the full-cache baseline ([EntmaxKV] §4):
+    weights against scipy's softmax, the two-token case against the logistic
+    function, and invariance to shifting every score."""
+    from scipy.special import softmax, expit
+    rng = np.random.default_rng(7)
+    q = rng.normal(size=(3, 16))
+    K = rng.normal(size=(50, 16))
+    V = rng.normal(size=(50, 16))
+    scale = 0.25
+    r = O.softmax_attention(q, K, V, scale)
+    w = softmax(scale * (q @ K.T), axis=1)
+    assert np.allclose(r["p"], w, rtol=1e-13, atol=1e-15)
+    assert np.allclose(r["o"], w @ V, rtol=1e-12, atol=1e-13)
+    # two tokens: weight of the first = logistic(z1 − z2)
+    K2 = rng.normal(size=(2, 16))
+    r2 = O.softmax_attention(q, K2, np.eye(2, 16), scale)
+    z = scale * (q @ K2.T)
+    assert np.allclose(r2["p"][:, 0], expit(z[:, 0] - z[:, 1]), rtol=1e-13)
+    # adding c·q to every key shifts every score of a head equally: nothing changes
+    r3 = O.softmax_attention(q[:1], K + 0.0, V, scale)
+    Ks = K + 3.0 * q[0] / (q[0] @ q[0])
+    r4 = O.softmax_attention(q[:1], Ks, V, scale)
+    assert np.allclose(r3["o"], r4["o"], rtol=1e-11, atol=1e-12)
+
+
+def test_entmax_tends_to_softmax_as_alpha_tends_to_one():
+    """α-entmax → softmax as α → 1⁺ (the Tsallis family's limit): the gap
+    shrinks in proportion to α − 1, tying the two oracle functions together."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(11)
+    z = rng.normal(size=40)
+    gaps = []
+    for eps in (1e-2, 1e-3, 1e-4):
+        p, _ = O.entmax_probs(z, 1.0 + eps)
+        gaps.append(np.abs(p - softmax(z)).max())
+    assert gaps[2] < 1e-4 and gaps[1] < 1e-3
+    assert 5 < gaps[0] / gaps[1] < 20 and 5 < gaps[1] / gaps[2] < 20
