@@ -325,6 +325,7 @@ def run_ours(args):
         "clocks": clocks,
     }
 
+    result["softmax_full_cache"] = bench_softmax(args, wl, inp, eng, dev, flush, peak, step_ms)
     if not args.quick:
         result["gauss"] = bench_policy(args, wl, inp, "gauss", dev, flush)
         result["full_cache"] = bench_policy(args, wl, inp, "full", dev, flush)
@@ -367,6 +368,40 @@ def bench_policy(args, wl, inp, policy, dev, flush, dense_v=False):
         res["k_bytes"] = kv
         res["dense_v"] = bool(dense_v)
     return res
+
+
+def bench_softmax(args, wl, inp, eng, dev, flush, peak, sparse_step_ms):
+    """The full-cache softmax decode ([EntmaxKV] §4's baseline, split over
+    pages) on the same cache: time, roofline on the K and V bytes it must read,
+    and the sparse entmax step's speedup over it."""
+    from sparse_kv_cache_kmax_b200 import binding as Bd
+    if wl.dtype != "bf16":
+        return {"unavailable": "bf16 caches only"}
+    P = inp["max_pages"]
+    out = torch.empty(wl.batch, wl.num_q_heads, wl.head_dim, device=dev)
+    ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_SOFTMAX_DECODE, eng.cache, eng.seqs, wl.num_q_heads, P), dev)
+    scale = float(np.float32(wl.scale))
+    steps = max(3, min(args.steps, 100))
+    for _ in range(args.warmup):
+        flush.zero_()
+        Bd.ekv_softmax_decode(eng.cache, eng.seqs, inp["q"], scale, None, None, P, out, ws)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        Bd.ekv_softmax_decode(eng.cache, eng.seqs, inp["q"], scale, None, None, P, out, ws)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    es = inp["k_pool"].element_size()
+    tokens = sum(int(L) for L in inp["seq_lens"].tolist())
+    nbytes = 2 * tokens * wl.num_kv_heads * wl.head_dim * es
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"ms_per_step": ms, "value": wl.units / (ms * 1e-3), "unit": UNIT, "steps": steps,
+            "algorithmic_bytes": nbytes, "achieved_gbs": ach, "frac": ach / peak,
+            "sparse_entmax_step_speedup": ms / sparse_step_ms,
+            "kernel": "softmax_split_kernel (all pages, K and V, split over pages)"}
 
 
 def bench_e2e(args, wl, inp, eng, dev, flush, world):

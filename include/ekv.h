@@ -182,6 +182,25 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
                                      int32_t* support_count, uint32_t* support_bits, void* ws,
                                      size_t ws_bytes, void* stream);
 
+/*
+ * ekv_softmax_decode — softmax attention decode over the paged cache: the
+ * full-cache baseline of [EKV] §4 ("the full cache read dominates"), split
+ * over pages.  For every query head h, o_h = Σ_i e^{z_i − m}·v_i / Σ_i e^{z_i − m}
+ * with z_i = scale·q_h·k_i over every valid token of the selected pages
+ * (sel = NULL with n_sel NULL: every page of the sequence; cap ≥ max_pages).
+ * sel: device [batch, Hkv, cap] logical page indices with n_sel entries per
+ * unit (as ekv_entmax_decode).  Outputs (device): out fp32 [batch, Hq, d];
+ * lse (nullable) fp32 [batch, Hq] = m + ln Σ_i e^{z_i − m} (−inf for a
+ * sequence without tokens, whose output row is 0).  bf16 caches with a page
+ * size that is a multiple of 16; any other returns EKV_ERR_UNSUPPORTED.
+ * ws: ekv_workspace_bytes(EKV_OP_SOFTMAX_DECODE, ...) bytes; the call clears
+ * the part it needs.
+ */
+EKV_API ekv_status ekv_softmax_decode(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                      int32_t num_q_heads, float scale, const int32_t* sel,
+                                      const int32_t* n_sel, int32_t cap, float* out, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of the library-owned scratch array of ekv_entmax_decode_static_ws. */
 #define EKV_STATIC_WS_BYTES (16u << 20)
 
@@ -240,7 +259,8 @@ EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
 typedef enum {
   EKV_OP_SELECT_GAUSS = 1,
   EKV_OP_ENTMAX_DECODE = 2,
-  EKV_OP_DECODE_STEP = 3
+  EKV_OP_DECODE_STEP = 3,
+  EKV_OP_SOFTMAX_DECODE = 4
 } ekv_op;
 
 /*

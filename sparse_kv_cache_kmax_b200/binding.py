@@ -20,12 +20,12 @@ __all__ = [
     "make_cache", "make_seqs", "workspace", "ekv_build_page_meta", "ekv_append",
     "ekv_score_pages", "ekv_select_topk", "ekv_select_gauss", "ekv_entmax_decode",
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
-    "ekv_entmax_decode_static_ws", "ekv_step_kernel_count",
+    "ekv_entmax_decode_static_ws", "ekv_step_kernel_count", "ekv_softmax_decode", "EKV_OP_SOFTMAX_DECODE",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
 EKV_POLICY_TOPK, EKV_POLICY_GAUSS, EKV_POLICY_FULL = 0, 1, 2
-EKV_OP_SELECT_GAUSS, EKV_OP_ENTMAX_DECODE, EKV_OP_DECODE_STEP = 1, 2, 3
+EKV_OP_SELECT_GAUSS, EKV_OP_ENTMAX_DECODE, EKV_OP_DECODE_STEP, EKV_OP_SOFTMAX_DECODE = 1, 2, 3, 4
 EKV_EFLAG_BAD_PAGE, EKV_EFLAG_BAD_LEN, EKV_EFLAG_SEL_OVERFLOW, EKV_EFLAG_BAD_SEL = 1, 2, 4, 8
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libekv.so")
@@ -76,6 +76,8 @@ _SIGS = {
     "ekv_decode_step": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams),
                         _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "ekv_workspace_bytes": [_I, ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _I, _I],
+    "ekv_softmax_decode": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _P, _P, _I, _P, _P,
+                           _P, _SZ, _P],
     "ekv_step_kernel_count": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams), _I],
     "ekv_entmax_decode_static_ws": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P,
                                     _P, _I, _I, _P, _P, _P, _P, _P],
@@ -207,6 +209,13 @@ def ekv_decode_step(cache, seqs, params: StepParams, q, k_new, v_new, sel, n_sel
         ctypes.byref(cache), ctypes.byref(seqs), ctypes.byref(params), _ptr(q), q.shape[1],
         _ptr(k_new), _ptr(v_new), _ptr(sel), _ptr(n_sel), _ptr(out), _ptr(tau), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def ekv_softmax_decode(cache, seqs, q, scale, sel, n_sel, cap, out, ws, *, lse=None, stream=None):
+    """Softmax decode over the selected pages (sel None: every page)."""
+    _check("ekv_softmax_decode", lib().ekv_softmax_decode(
+        ctypes.byref(cache), ctypes.byref(seqs), _ptr(q), q.shape[1], scale, _ptr(sel), _ptr(n_sel), cap,
+        _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def ekv_step_kernel_count(cache, seqs, params: StepParams, num_q_heads) -> int:

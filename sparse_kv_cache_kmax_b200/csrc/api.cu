@@ -226,6 +226,19 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
                                    static_cast<cudaStream_t>(stream)));
 }
 
+EKV_API ekv_status ekv_softmax_decode(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                      int32_t num_q_heads, float scale, const int32_t* sel,
+                                      const int32_t* n_sel, int32_t cap, float* out, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  EKV_TRY(validate_decode(cache, seqs, q, num_q_heads, scale, 1.5f, sel, n_sel, cap, out));
+  if (cache->dtype != EKV_BF16 || cache->page_size % 16 != 0) return EKV_ERR_UNSUPPORTED;
+  const int U = seqs->batch * cache->num_kv_heads;
+  EKV_TRY(check_ws(ws, ws_bytes, softmax_ws_bytes(U, num_q_heads, cache->num_kv_heads,
+                                                  cache->head_dim, cap)));
+  return cuda_status(launch_softmax_decode(*cache, *seqs, q, num_q_heads, scale, sel, n_sel, cap, out,
+                                           lse, ws, static_cast<cudaStream_t>(stream)));
+}
+
 EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
                                    const ekv_step_params* p, const void* q, int32_t num_q_heads,
                                    const void* k_new, const void* v_new, int32_t* sel,
@@ -288,6 +301,9 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
       return cap < 1 ? 0 : decode_ws_bytes(cache, seqs, num_q_heads, cap);
     case EKV_OP_DECODE_STEP:
       return cap < 1 ? 0 : step_ws_bytes(cache, seqs, num_q_heads, cap);
+    case EKV_OP_SOFTMAX_DECODE:
+      return cap < 1 ? 0 : softmax_ws_bytes(seqs->batch * cache->num_kv_heads, num_q_heads,
+                                            cache->num_kv_heads, cache->head_dim, cap);
     default:
       return 0;
   }

@@ -25,15 +25,16 @@ struct DecodeArgs {
   int Hkv, Hq, S, num_phys, max_pages, cap, spp_pv, dense_v, words;
 };
 
-__device__ __forceinline__ int unit_slots(const DecodeArgs& a, int unit, int P) {
+template <class A>
+__device__ __forceinline__ int unit_slots(const A& a, int unit, int P) {
   if (a.sel == nullptr) return min(P, a.cap);
   const int n = a.n_sel[unit];
   return max(0, min(n, a.cap));
 }
 
 // Logical page of a selected slot → (physical page, valid tokens); −1 when bad.
-__device__ __forceinline__ int slot_page(const DecodeArgs& a, int unit, int b, int slot, int P,
-                                         int L, int* nv) {
+template <class A>
+__device__ __forceinline__ int slot_page(const A& a, int unit, int b, int slot, int P, int L, int* nv) {
   const int lp = a.sel ? a.sel[static_cast<size_t>(unit) * a.cap + slot] : slot;
   *nv = 0;
   if (lp < 0 || lp >= P) {
@@ -74,8 +75,8 @@ __device__ __forceinline__ float pow_beta_fast(float w, float beta, int ipow) {
 // fragments from one 16-byte load per row and 32-column chunk: chunk c,
 // k-step 2c takes columns 32c + 8t + {0..3}, k-step 2c+1 columns 32c + 8t +
 // {4..7} (so every row uses the same column order).
-template <int D, int G>
-__device__ __forceinline__ void load_q_frags(const DecodeArgs& a, int b, int kvh, int g, int t,
+template <int D, int G, class A>
+__device__ __forceinline__ void load_q_frags(const A& a, int b, int kvh, int g, int t,
                                              uint32_t (&bfrag)[D / 16][(G + 7) / 8][2]) {
   constexpr int KS = D / 16, NT = (G + 7) / 8;
   const bf16* qb = static_cast<const bf16*>(a.q) + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G) * D;

@@ -49,6 +49,13 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
                           uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st);
 
+// Softmax decode split over pages (softmax.cu).
+int softmax_splits(int units, int cap);
+size_t softmax_ws_bytes(int units, int Hq, int Hkv, int d, int cap);
+cudaError_t launch_softmax_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
+                                  float scale, const int32_t* sel, const int32_t* n_sel, int cap,
+                                  float* out, float* lse, void* ws, cudaStream_t st);
+
 // Kernels one launch_decode enqueues for these sizes (1 fused, or 3).
 int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap);
 

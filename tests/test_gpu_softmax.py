@@ -1,0 +1,105 @@
+"""GPU parity of the softmax decode (the full-cache baseline of [EntmaxKV] §4,
+split over pages) against the float64 oracle's dense softmax, over every page
+and over a top-k selection, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sparse_kv_cache_kmax_b200 import binding as B
+from sparse_kv_cache_kmax_b200.workloads import scaled_down
+
+from gpu_helpers import OUT_TOL, Gpu, gen, np64, q_group, row_rel_err, unit_arrays
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "gqa_32k": dict(batch=2, context=1500),
+    "clustered_128k": dict(batch=2, context=3005),
+    "short_scattered": dict(batch=5, context=900, context_min=300),
+    "long_512k": dict(batch=1, context=4007),
+}
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def case(request):
+    wl = scaled_down(request.param, **CASES[request.param])
+    inp = gen(wl, 3000 + list(CASES).index(request.param))
+    return wl, inp, Gpu(inp)
+
+
+def _run(gpu, sel=None, n_sel=None, cap=None):
+    wl, inp = gpu.wl, gpu.inp
+    cap = cap or inp["max_pages"]
+    out = torch.full((wl.batch, gpu.Hq, wl.head_dim), float("nan"), device="cuda")
+    lse = torch.full((wl.batch, gpu.Hq), float("nan"), device="cuda")
+    ws = B.workspace(B.ekv_workspace_bytes(B.EKV_OP_SOFTMAX_DECODE, gpu.cache, gpu.seqs, gpu.Hq, cap), "cuda")
+    B.ekv_softmax_decode(gpu.cache, gpu.seqs, inp["q"], gpu.scale, sel, n_sel, cap, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def _oracle(inp, b, h, pages=None):
+    wl = inp["workload"]
+    kp, vp, _, L = unit_arrays(inp, b, h)
+    S = wl.page_size
+    P = kp.shape[0]
+    pages = np.arange(P) if pages is None else np.asarray(pages)
+    K = np.concatenate([kp[p, 0, : min(S, L - p * S)] for p in pages])
+    V = np.concatenate([vp[p, 0, : min(S, L - p * S)] for p in pages])
+    qg = q_group(inp, b, h)
+    scale = float(np.float32(wl.scale))
+    r = O.softmax_attention(qg, K, V, scale)
+    z = scale * (qg @ K.T)
+    lse = z.max(axis=1) + np.log(np.exp(z - z.max(axis=1, keepdims=True)).sum(axis=1))
+    return r["o"], lse
+
+
+def test_softmax_full_cache_matches_oracle(case):
+    wl, inp, gpu = case
+    out, lse = _run(gpu)
+    G = wl.group
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            o_ref, lse_ref = _oracle(inp, b, h)
+            rows = slice(h * G, (h + 1) * G)
+            err = row_rel_err(np64(out[b, rows]), o_ref)
+            assert np.all(err <= OUT_TOL[wl.dtype]), (b, h, err.max())
+            assert np.allclose(np64(lse[b, rows]), lse_ref, rtol=0, atol=2e-4 * max(1.0, np.abs(lse_ref).max()))
+
+
+def test_softmax_over_a_selection_matches_oracle(case):
+    wl, inp, gpu = case
+    gpu.build_meta()
+    k = 8
+    sel, n = gpu.topk(gpu.score(), k)
+    out, lse = _run(gpu, sel, n, k)
+    G = wl.group
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            pages = sel[b, h, : int(n[b, h])].cpu().numpy()
+            o_ref, lse_ref = _oracle(inp, b, h, pages)
+            rows = slice(h * G, (h + 1) * G)
+            err = row_rel_err(np64(out[b, rows]), o_ref)
+            assert np.all(err <= OUT_TOL[wl.dtype]), (b, h, err.max())
+
+
+def test_softmax_empty_selection_gives_zero_and_minus_inf(case):
+    wl, inp, gpu = case
+    k = 4
+    sel = torch.zeros(wl.batch, wl.num_kv_heads, k, dtype=torch.int32, device="cuda")
+    n = torch.zeros(wl.batch, wl.num_kv_heads, dtype=torch.int32, device="cuda")
+    n[0, 0] = 0
+    n[1:] = 1 if wl.batch > 1 else 0
+    out, lse = _run(gpu, sel, n, k)
+    G = wl.group
+    assert torch.all(out[0, :G] == 0) and torch.all(torch.isneginf(lse[0, :G]))
+    assert torch.isfinite(out).all()
+
+
+def test_softmax_rejects_fp32_caches():
+    wl = scaled_down("tiny_fp32", context=600)
+    inp = gen(wl, 5)
+    gpu = Gpu(inp)
+    with pytest.raises(B.EkvError):
+        _run(gpu)
