@@ -46,6 +46,7 @@ __all__ = [
     "gauss_tau_hat", "select_gauss", "entmax_threshold", "entmax_probs",
     "entmax_attention", "softmax_attention", "unit_pages", "decode_unit",
     "build_page_meta", "append_token", "ENTMAX_SORT_ALPHAS",
+    "exactness_certificate", "adaptive_topk",
 ]
 
 ENTMAX_SORT_ALPHAS = (1.5, 2.0)
@@ -465,3 +466,40 @@ def decode_unit(k_pool, v_pool, page_table_row, seq_len, kv_head, q_group, *,
     out["token_page"] = np.concatenate([np.full(n_valid[p], p) for p in sel])
     out["token_slot"] = np.concatenate([np.arange(n_valid[p]) for p in sel])
     return out
+
+
+# --------------------------------------------------------------------------
+# exactness certificate — [EntmaxKV] §3 "Récupération du Support"
+# --------------------------------------------------------------------------
+def exactness_certificate(score, sel, tau, alpha):
+    """Per query head: True when no unselected page can hold a support token.
+
+    [EntmaxKV] §3: if the selected tokens contain the α-entmax support, the
+    sparse output equals the full-cache one.  Every token score of page p is
+    at most the page score (the bound maximised over the group's heads), so
+    when (α−1)·max_{p ∉ sel} score_p ≤ τ_h, no unselected token has
+    u = (α−1)z > τ_h; τ_h then also solves the full-cache equation (the extra
+    tokens add nothing to Σ[u − τ]_+^β), so the outputs agree.  score: [P]
+    unit scores; sel: selected page indices; tau: [G].  With nothing left
+    unselected the certificate holds trivially.
+    """
+    score = np.asarray(score, np.float64)
+    rest = np.setdiff1d(np.arange(score.shape[0]), np.asarray(sel, np.int64))
+    if rest.size == 0:
+        return np.ones(np.shape(tau), bool)
+    return (alpha - 1.0) * score[rest].max() <= np.asarray(tau, np.float64)
+
+
+def adaptive_topk(k_pool, v_pool, page_table_row, seq_len, kv_head, q_group, *, page_size,
+                  scale, alpha, dtype, k0):
+    """Grow the top-k budget (doubling from k0) until every head of the unit is
+    certified exact; returns (k, decode_unit result).  The certificate's
+    extension of [EntmaxKV] §3 into an adaptive budget."""
+    n_pages = -(-int(seq_len) // page_size)
+    k = max(1, int(k0))
+    while True:
+        r = decode_unit(k_pool, v_pool, page_table_row, seq_len, kv_head, q_group, page_size=page_size,
+                        scale=scale, alpha=alpha, dtype=dtype, policy="topk", k=k)
+        if k >= n_pages or np.all(exactness_certificate(r["score"], r["sel"], r["tau"], alpha)):
+            return k, r
+        k = min(2 * k, n_pages)

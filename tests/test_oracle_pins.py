@@ -486,3 +486,40 @@ def test_entmax_tends_to_softmax_as_alpha_tends_to_one():
         gaps.append(np.abs(p - softmax(z)).max())
     assert gaps[2] < 1e-4 and gaps[1] < 1e-3
     assert 5 < gaps[0] / gaps[1] < 20 and 5 < gaps[1] / gaps[2] < 20
+
+
+# ---------------------------------------------------------------- exactness certificate (unit scores)
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25])
+def test_unit_score_certificate_implies_full_cache_output(alpha):
+    """[EntmaxKV] §3: a head certified from the unit's page scores (the bound
+    maximised over the group) has the full-cache output exactly; the test
+    sees both certified and uncertified heads."""
+    rng = np.random.default_rng(61)
+    seen = {True: 0, False: 0}
+    for trial in range(40):
+        k_pool, v_pool, pt, L, q = _random_unit(rng)
+        kw = dict(page_size=8, scale=0.25, alpha=alpha, dtype="f32")
+        full = O.decode_unit(k_pool, v_pool, pt, L, 0, q, policy="all", **kw)
+        sparse = O.decode_unit(k_pool, v_pool, pt, L, 0, q, policy="topk", k=int(rng.integers(1, 30)), **kw)
+        cert = O.exactness_certificate(sparse["score"], sparse["sel"], sparse["tau"], alpha)
+        for h in range(q.shape[0]):
+            seen[bool(cert[h])] += 1
+            if cert[h]:
+                assert np.allclose(sparse["o"][h], full["o"][h], atol=1e-12)
+                assert abs(sparse["tau"][h] - full["tau"][h]) <= 1e-12
+    assert seen[True] > 0 and seen[False] > 0
+
+
+def test_adaptive_budget_reaches_the_full_cache_output():
+    """Doubling k until every head is certified ends at the full-cache output,
+    and the budget before the last doubling was not certified."""
+    rng = np.random.default_rng(67)
+    for trial in range(15):
+        k_pool, v_pool, pt, L, q = _random_unit(rng)
+        kw = dict(page_size=8, scale=0.25, alpha=1.5, dtype="f32")
+        full = O.decode_unit(k_pool, v_pool, pt, L, 0, q, policy="all", **kw)
+        k, r = O.adaptive_topk(k_pool, v_pool, pt, L, 0, q, k0=2, **kw)
+        assert np.allclose(r["o"], full["o"], atol=1e-12)
+        if k > 2:
+            prev = O.decode_unit(k_pool, v_pool, pt, L, 0, q, policy="topk", k=k // 2, **kw)
+            assert not np.all(O.exactness_certificate(prev["score"], prev["sel"], prev["tau"], 1.5))
