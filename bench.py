@@ -274,8 +274,11 @@ def run_ours(args):
     words = (k * wl.page_size + 31) // 32
     bits = torch.zeros(wl.batch, Hq, words, dtype=torch.int32, device=dev)
     cnt = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=dev)
+    tau_last = torch.zeros(wl.batch, Hq, device=dev)
     Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws,
-                         support_count=cnt, support_bits=bits)
+                         tau=tau_last, support_count=cnt, support_bits=bits)
+    cert = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=dev)
+    Bd.ekv_exactness_certificate(seqs, wl.num_kv_heads, wl.page_size, alpha, ub, eng.sel, eng.n_sel, tau_last, cert)
     tok = ((bits.view(torch.int32).unsqueeze(-1) >> torch.arange(32, device=dev, dtype=torch.int32)) & 1)
     tok = tok.view(wl.batch, wl.num_kv_heads, wl.group, -1).amax(dim=2)          # union over the group
     page_sup = tok.view(wl.batch, wl.num_kv_heads, k, wl.page_size).amax(dim=-1)
@@ -319,6 +322,7 @@ def run_ours(args):
         "step_roofline": {"bytes": nb["step"], "achieved_gbs": nb["step"] / (step_ms * 1e-3) / 1e9,
                           "frac": nb["step"] / (step_ms * 1e-3) / 1e9 / peak,
                           "breakdown": {kk: v for kk, v in nb.items() if kk not in ("step", "score_kernel")}},
+        "certificate": certificate_stats(cert, inp, wl, alpha, k),
         "support": {"mean_sel_pages": float(eng.n_sel.float().mean()), "support_pages_per_unit":
                     support_pages / wl.units, "mean_support_tokens_per_head": float(cnt.float().mean())},
         "gpu_launches": Bd.ekv_step_kernel_count(cache, seqs, eng.params, Hq) * args.steps,
@@ -370,6 +374,18 @@ def bench_policy(args, wl, inp, policy, dev, flush, dense_v=False):
     return res
 
 
+def certificate_stats(cert, inp, wl, alpha, k):
+    """Exactness certificate at the bench's budget, and the budget the doubling
+    adaptive decode needs until every head is certified (untimed)."""
+    from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
+                       policy="topk", k=k, alpha=alpha)
+    eng.build_meta()
+    _, k_needed = eng.decode_adaptive(inp["q"], k0=k)
+    return {"certified_heads_frac_at_k": float(cert.float().mean()), "k": k,
+            "adaptive_k_all_certified": int(k_needed)}
+
+
 def bench_softmax(args, wl, inp, eng, dev, flush, peak, sparse_step_ms):
     """The full-cache softmax decode ([EntmaxKV] §4's baseline, split over
     pages) on the same cache: time, roofline on the K and V bytes it must read,
@@ -401,7 +417,41 @@ def bench_softmax(args, wl, inp, eng, dev, flush, peak, sparse_step_ms):
     return {"ms_per_step": ms, "value": wl.units / (ms * 1e-3), "unit": UNIT, "steps": steps,
             "algorithmic_bytes": nbytes, "achieved_gbs": ach, "frac": ach / peak,
             "sparse_entmax_step_speedup": ms / sparse_step_ms,
-            "kernel": "softmax_split_kernel (all pages, K and V, split over pages)"}
+            "kernel": "softmax_split_kernel (all pages, K and V, split over pages)",
+            "dropped_mass": dropped_mass(wl, inp, eng, dev, out, ws, scale)}
+
+
+def dropped_mass(wl, inp, eng, dev, out_full_sm, ws_sm, scale):
+    """Quality of the kept set (untimed; [EntmaxKV] §3–§4): under the same
+    top-k pages, the softmax weight left outside them (1 − e^(lse_sel − lse_full))
+    and its output error, against the entmax output error (zero whenever the
+    kept pages hold the support).  Errors are per (sequence, query head) row:
+    max_i |o_i − ô_i| / max_i |ô_i|."""
+    from sparse_kv_cache_kmax_b200 import binding as Bd
+    P, k, Hq = inp["max_pages"], eng.cap, wl.num_q_heads
+    alpha = eng.params.alpha
+    lse_full = torch.empty(wl.batch, Hq, device=dev)
+    lse_sel = torch.empty(wl.batch, Hq, device=dev)
+    out_sel = torch.empty_like(out_full_sm)
+    Bd.ekv_softmax_decode(eng.cache, eng.seqs, inp["q"], scale, None, None, P, out_full_sm, ws_sm, lse=lse_full)
+    ws_k = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_SOFTMAX_DECODE, eng.cache, eng.seqs, Hq, k), dev)
+    Bd.ekv_softmax_decode(eng.cache, eng.seqs, inp["q"], scale, eng.sel, eng.n_sel, k, out_sel, ws_k, lse=lse_sel)
+    ent_full = torch.empty_like(out_full_sm)
+    ent_sel = torch.empty_like(out_full_sm)
+    ws_f = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, eng.cache, eng.seqs, Hq, P), dev)
+    Bd.ekv_entmax_decode(eng.cache, eng.seqs, inp["q"], scale, alpha, None, None, P, ent_full, ws_f)
+    ws_s = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, eng.cache, eng.seqs, Hq, k), dev)
+    Bd.ekv_entmax_decode(eng.cache, eng.seqs, inp["q"], scale, alpha, eng.sel, eng.n_sel, k, ent_sel, ws_s)
+    torch.cuda.synchronize()
+
+    def rel(a, b):
+        return ((a - b).abs().amax(-1) / b.abs().amax(-1).clamp_min(1e-6)).flatten()
+
+    drop = (1.0 - torch.exp(lse_sel.double() - lse_full.double())).flatten()
+    e_sm, e_ent = rel(out_sel, out_full_sm), rel(ent_sel, ent_full)
+    return {"k": int(k), "softmax_dropped_mass_mean": float(drop.mean()), "softmax_dropped_mass_max": float(drop.max()),
+            "softmax_rel_err_median": float(e_sm.median()), "softmax_rel_err_max": float(e_sm.max()),
+            "entmax_rel_err_median": float(e_ent.median()), "entmax_rel_err_max": float(e_ent.max())}
 
 
 def bench_e2e(args, wl, inp, eng, dev, flush, world):

@@ -201,6 +201,24 @@ EKV_API ekv_status ekv_softmax_decode(const ekv_cache* cache, const ekv_seqs* se
                                       const int32_t* n_sel, int32_t cap, float* out, float* lse,
                                       void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * ekv_exactness_certificate — [EKV] §3 "Récupération du Support": the sparse
+ * output equals the full-cache output when the selection holds the α-entmax
+ * support.  certified[b, hq] = 1 when (α−1)·max_{p ∉ sel} ub[b, kvh, p] ≤
+ * tau[b, hq] over the valid unselected pages p of unit (b, kvh = hq / G), or
+ * when no valid page is left unselected; else 0.  A head whose τ is +inf (no
+ * finite score among the selected tokens) is certified only in the latter
+ * case.  ub: device [batch, Hkv, max_pages] unit scores from ekv_score_pages;
+ * sel / n_sel / cap as for ekv_entmax_decode (non-NULL); tau: device
+ * [batch, Hq] from the decode of that selection; certified: device int32
+ * [batch, Hq].  max_pages above 393216 returns EKV_ERR_UNSUPPORTED.
+ */
+EKV_API ekv_status ekv_exactness_certificate(const ekv_seqs* seqs, int32_t num_kv_heads,
+                                             int32_t page_size, int32_t num_q_heads, float alpha,
+                                             const float* ub, const int32_t* sel,
+                                             const int32_t* n_sel, int32_t cap, const float* tau,
+                                             int32_t* certified, void* stream);
+
 /* Bytes of the library-owned scratch array of ekv_entmax_decode_static_ws. */
 #define EKV_STATIC_WS_BYTES (16u << 20)
 

@@ -21,6 +21,7 @@ __all__ = [
     "ekv_score_pages", "ekv_select_topk", "ekv_select_gauss", "ekv_entmax_decode",
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
     "ekv_entmax_decode_static_ws", "ekv_step_kernel_count", "ekv_softmax_decode", "EKV_OP_SOFTMAX_DECODE",
+    "ekv_exactness_certificate",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
@@ -78,6 +79,7 @@ _SIGS = {
     "ekv_workspace_bytes": [_I, ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _I, _I],
     "ekv_softmax_decode": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _P, _P, _I, _P, _P,
                            _P, _SZ, _P],
+    "ekv_exactness_certificate": [ctypes.POINTER(Seqs), _I, _I, _I, _F, _P, _P, _P, _I, _P, _P, _P],
     "ekv_step_kernel_count": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams), _I],
     "ekv_entmax_decode_static_ws": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P,
                                     _P, _I, _I, _P, _P, _P, _P, _P],
@@ -216,6 +218,14 @@ def ekv_softmax_decode(cache, seqs, q, scale, sel, n_sel, cap, out, ws, *, lse=N
     _check("ekv_softmax_decode", lib().ekv_softmax_decode(
         ctypes.byref(cache), ctypes.byref(seqs), _ptr(q), q.shape[1], scale, _ptr(sel), _ptr(n_sel), cap,
         _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def ekv_exactness_certificate(seqs, num_kv_heads, page_size, alpha, ub, sel, n_sel, tau, certified, *,
+                              stream=None):
+    """certified[b, hq] = 1 when head hq's sparse output equals its full-cache one."""
+    _check("ekv_exactness_certificate", lib().ekv_exactness_certificate(
+        ctypes.byref(seqs), num_kv_heads, page_size, tau.shape[1], alpha, _ptr(ub), _ptr(sel), _ptr(n_sel),
+        sel.shape[-1], _ptr(tau), _ptr(certified), _stream(stream)))
 
 
 def ekv_step_kernel_count(cache, seqs, params: StepParams, num_q_heads) -> int:

@@ -226,6 +226,22 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
                                    static_cast<cudaStream_t>(stream)));
 }
 
+EKV_API ekv_status ekv_exactness_certificate(const ekv_seqs* seqs, int32_t num_kv_heads,
+                                             int32_t page_size, int32_t num_q_heads, float alpha,
+                                             const float* ub, const int32_t* sel,
+                                             const int32_t* n_sel, int32_t cap, const float* tau,
+                                             int32_t* certified, void* stream) {
+  EKV_TRY(check_seqs(seqs));
+  EKV_TRY(check_alpha(alpha));
+  if (num_kv_heads < 1 || page_size < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads != 0)
+    return EKV_ERR_INVALID_ARG;
+  if (ub == nullptr || sel == nullptr || n_sel == nullptr || tau == nullptr || certified == nullptr || cap < 1)
+    return EKV_ERR_INVALID_ARG;
+  if (!certificate_smem_ok(seqs->max_pages)) return EKV_ERR_UNSUPPORTED;
+  return cuda_status(launch_certificate(*seqs, num_kv_heads, page_size, num_q_heads, alpha, ub, sel, n_sel,
+                                        cap, tau, certified, static_cast<cudaStream_t>(stream)));
+}
+
 EKV_API ekv_status ekv_softmax_decode(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
                                       int32_t num_q_heads, float scale, const int32_t* sel,
                                       const int32_t* n_sel, int32_t cap, float* out, float* lse,

@@ -49,6 +49,12 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
                           uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st);
 
+// Exactness certificate per query head (certify.cu).
+int certificate_smem_ok(int max_pages);
+cudaError_t launch_certificate(const ekv_seqs& s, int Hkv, int S, int Hq, float alpha, const float* ub,
+                               const int32_t* sel, const int32_t* n_sel, int cap, const float* tau,
+                               int32_t* cert, cudaStream_t st);
+
 // Softmax decode split over pages (softmax.cu).
 int softmax_splits(int units, int cap);
 size_t softmax_ws_bytes(int units, int Hq, int Hkv, int d, int cap);
