@@ -213,6 +213,8 @@ def run_ours(args):
     scale = float(np.float32(wl.scale))
     ub = torch.empty(wl.batch, wl.num_kv_heads, inp["max_pages"], device=dev)
     dec_ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, cache, seqs, Hq, k), dev)
+    n_tk = Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_TOPK, cache, seqs, Hq, k)
+    tk_ws = Bd.workspace(n_tk, dev) if n_tk else None
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
@@ -222,7 +224,7 @@ def run_ours(args):
         ev[1].record(stream)
         Bd.ekv_score_pages(cache, seqs, q, scale, ub, stream)
         ev[2].record(stream)
-        Bd.ekv_select_topk(seqs, wl.num_kv_heads, wl.page_size, ub, k, eng.sel, eng.n_sel, stream)
+        Bd.ekv_select_topk(seqs, wl.num_kv_heads, wl.page_size, ub, k, eng.sel, eng.n_sel, stream, ws=tk_ws)
         ev[3].record(stream)
         Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws, stream=stream)
         ev[4].record(stream)
@@ -630,13 +632,15 @@ def run_kernel(args):
         sel = torch.zeros(B, Hkv, max(k, P), dtype=torch.int32, device=dev)
         n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
         tau_hat = torch.zeros(B, Hq, device=dev)
+        n_tk = Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_TOPK, cache, seqs, Hq, k)
+        tk_ws = Bd.workspace(n_tk, dev) if n_tk else None
         gws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_GAUSS, cache, seqs, Hq, P), dev)
 
         def launch():
             if args.kernel == "score":
                 Bd.ekv_score_pages(cache, seqs, q, scale, ub, stream)
             elif args.kernel == "topk":
-                Bd.ekv_select_topk(seqs, Hkv, S, ub, k, sel, n_sel, stream)
+                Bd.ekv_select_topk(seqs, Hkv, S, ub, k, sel, n_sel, stream, ws=tk_ws)
             else:
                 Bd.ekv_select_gauss(cache, seqs, q, scale, args.alpha, wl.delta or 0.5, P, sel, n_sel, tau_hat,
                                     gws, stream)

@@ -135,11 +135,15 @@ EKV_API ekv_status ekv_score_pages(const ekv_cache* cache, const ekv_seqs* seqs,
  * when ⌈L_b/S⌉ ≤ k), written ascending to sel[b, kvh, 0..n_sel) with
  * n_sel = min(k, ⌈L_b/S⌉).  page_size S turns seq_lens into page counts.
  * ub: device [batch, Hkv, max_pages] (ekv_score_pages); sel: device
- * [batch, Hkv, k]; n_sel: [batch, Hkv].
+ * [batch, Hkv, k]; n_sel: [batch, Hkv].  ws: ekv_workspace_bytes(
+ * EKV_OP_SELECT_TOPK, ..., cap = k) bytes, which is 0 (ws may be NULL) up to
+ * 16384 pages per sequence; longer sequences with that scratch are selected
+ * in two stages (chunks of 8192 pages keep their k best, then k among those),
+ * without it in one slower stage.
  */
 EKV_API ekv_status ekv_select_topk(const ekv_seqs* seqs, int32_t num_kv_heads, int32_t page_size,
                                    const float* ub, int32_t k, int32_t* sel, int32_t* n_sel,
-                                   void* stream);
+                                   void* ws, size_t ws_bytes, void* stream);
 
 /*
  * ekv_select_gauss — [EntmaxKV] §2.A "Statistiques Gaussiennes" + §2.B.2,
@@ -278,7 +282,8 @@ typedef enum {
   EKV_OP_SELECT_GAUSS = 1,
   EKV_OP_ENTMAX_DECODE = 2,
   EKV_OP_DECODE_STEP = 3,
-  EKV_OP_SOFTMAX_DECODE = 4
+  EKV_OP_SOFTMAX_DECODE = 4,
+  EKV_OP_SELECT_TOPK = 5
 } ekv_op;
 
 /*
@@ -292,7 +297,8 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
 /*
  * ekv_step_kernel_count — how many kernels one ekv_decode_step call with these
  * arguments enqueues: the append (if params->append), the selection (2 for
- * top-k, 3 for the Gaussian policy, 0 for every page) and the decode (1 when
+ * top-k, 3 when it runs in two stages (more than 16384 pages per sequence),
+ * 3 for the Gaussian policy, 0 for every page) and the decode (1 when
  * a bf16 selection fits the one-cluster-per-unit kernel, else 3).  Host-side
  * only; returns 0 when the sizes are invalid.
  */

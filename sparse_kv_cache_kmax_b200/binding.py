@@ -21,12 +21,13 @@ __all__ = [
     "ekv_score_pages", "ekv_select_topk", "ekv_select_gauss", "ekv_entmax_decode",
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
     "ekv_entmax_decode_static_ws", "ekv_step_kernel_count", "ekv_softmax_decode", "EKV_OP_SOFTMAX_DECODE",
-    "ekv_exactness_certificate",
+    "ekv_exactness_certificate", "EKV_OP_SELECT_TOPK",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
 EKV_POLICY_TOPK, EKV_POLICY_GAUSS, EKV_POLICY_FULL = 0, 1, 2
 EKV_OP_SELECT_GAUSS, EKV_OP_ENTMAX_DECODE, EKV_OP_DECODE_STEP, EKV_OP_SOFTMAX_DECODE = 1, 2, 3, 4
+EKV_OP_SELECT_TOPK = 5
 EKV_EFLAG_BAD_PAGE, EKV_EFLAG_BAD_LEN, EKV_EFLAG_SEL_OVERFLOW, EKV_EFLAG_BAD_SEL = 1, 2, 4, 8
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libekv.so")
@@ -69,7 +70,7 @@ _SIGS = {
     "ekv_build_page_meta": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P],
     "ekv_append": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _P, _P],
     "ekv_score_pages": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _P, _P],
-    "ekv_select_topk": [ctypes.POINTER(Seqs), _I, _I, _P, _I, _P, _P, _P],
+    "ekv_select_topk": [ctypes.POINTER(Seqs), _I, _I, _P, _I, _P, _P, _P, _SZ, _P],
     "ekv_select_gauss": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _F, _I,
                          _P, _P, _P, _P, _SZ, _P],
     "ekv_entmax_decode": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P, _P,
@@ -186,9 +187,12 @@ def ekv_score_pages(cache, seqs, q, scale, ub, stream=None):
                                                     q.shape[1], scale, _ptr(ub), _stream(stream)))
 
 
-def ekv_select_topk(seqs, num_kv_heads, page_size, ub, k, sel, n_sel, stream=None):
+def ekv_select_topk(seqs, num_kv_heads, page_size, ub, k, sel, n_sel, stream=None, *, ws=None):
+    """ws: ekv_workspace_bytes(EKV_OP_SELECT_TOPK, ..., k) bytes (None when 0,
+    or to select long sequences in one stage)."""
     _check("ekv_select_topk", lib().ekv_select_topk(ctypes.byref(seqs), num_kv_heads, page_size, _ptr(ub),
-                                                    k, _ptr(sel), _ptr(n_sel), _stream(stream)))
+                                                    k, _ptr(sel), _ptr(n_sel), _ptr(ws),
+                                                    0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def ekv_select_gauss(cache, seqs, q, scale, alpha, delta, cap, sel, n_sel, tau_hat, ws, stream=None):

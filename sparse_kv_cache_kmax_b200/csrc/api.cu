@@ -116,7 +116,7 @@ DecodeWs carve_decode(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq,
 size_t step_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   return a256(U * static_cast<size_t>(s->max_pages) * sizeof(float)) + gauss_ws_bytes(c, s, Hq) +
-         decode_ws_bytes(c, s, Hq, cap);
+         decode_ws_bytes(c, s, Hq, cap) + a256(topk_ws_bytes_upto(static_cast<int>(U), s->max_pages, cap));
 }
 
 ekv_status check_ws(void* ws, size_t have, size_t need) {
@@ -180,12 +180,15 @@ EKV_API ekv_status ekv_score_pages(const ekv_cache* cache, const ekv_seqs* seqs,
 
 EKV_API ekv_status ekv_select_topk(const ekv_seqs* seqs, int32_t num_kv_heads, int32_t page_size,
                                    const float* ub, int32_t k, int32_t* sel, int32_t* n_sel,
-                                   void* stream) {
+                                   void* ws, size_t ws_bytes, void* stream) {
   EKV_TRY(check_seqs(seqs));
   if (num_kv_heads < 1 || ub == nullptr || sel == nullptr || n_sel == nullptr || k < 1)
     return EKV_ERR_INVALID_ARG;
   if (page_size != 16 && page_size != 32) return EKV_ERR_UNSUPPORTED;
+  const size_t need = topk_ws_bytes(seqs->batch * num_kv_heads, seqs->max_pages, k);
+  if (ws != nullptr) EKV_TRY(check_ws(ws, ws_bytes, need));
   return cuda_status(launch_topk(*seqs, num_kv_heads, page_size, ub, k, k, sel, n_sel,
+                                 ws != nullptr && need > 0 ? ws : nullptr,
                                  static_cast<cudaStream_t>(stream)));
 }
 
@@ -284,6 +287,7 @@ EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
   float* ub = cv.take<float>(U * static_cast<size_t>(seqs->max_pages));
   const GaussWs gw = carve_gauss(cv, cache, seqs, num_q_heads);
   const DecodeWs dw = carve_decode(cv, cache, seqs, num_q_heads, cap);
+  void* tws = cv.base + cv.used;  // top-k scratch (sized for any k ≤ cap)
 
   if (p->append) EKV_TRY(cuda_status(launch_append(*cache, *seqs, k_new, v_new, st)));
   const int32_t* use_sel = sel;
@@ -291,7 +295,9 @@ EKV_API ekv_status ekv_decode_step(const ekv_cache* cache, const ekv_seqs* seqs,
   if (p->policy == EKV_POLICY_TOPK) {
     EKV_TRY(cuda_status(launch_score(*cache, *seqs, q, num_q_heads, p->scale, ub, st, p->append ? 1 : 0)));
     EKV_TRY(cuda_status(launch_topk(*seqs, cache->num_kv_heads, cache->page_size, ub, p->k, cap,
-                                    sel, n_sel, st)));
+                                    sel, n_sel,
+                                    topk_ws_bytes(static_cast<int>(U), seqs->max_pages, p->k) > 0 ? tws : nullptr,
+                                    st)));
   } else if (p->policy == EKV_POLICY_GAUSS) {
     EKV_TRY(cuda_status(launch_gauss_stats(*cache, *seqs, q, num_q_heads, p->scale, p->alpha, gw, st,
                                            p->append ? 1 : 0)));
@@ -317,6 +323,8 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
       return cap < 1 ? 0 : decode_ws_bytes(cache, seqs, num_q_heads, cap);
     case EKV_OP_DECODE_STEP:
       return cap < 1 ? 0 : step_ws_bytes(cache, seqs, num_q_heads, cap);
+    case EKV_OP_SELECT_TOPK:
+      return cap < 1 ? 0 : topk_ws_bytes(seqs->batch * cache->num_kv_heads, seqs->max_pages, cap);
     case EKV_OP_SOFTMAX_DECODE:
       return cap < 1 ? 0 : softmax_ws_bytes(seqs->batch * cache->num_kv_heads, num_q_heads,
                                             cache->num_kv_heads, cache->head_dim, cap);
@@ -334,7 +342,8 @@ EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* se
   const int cap = full ? seqs->max_pages : p->cap;
   if (cap < 1) return 0;
   int n = p->append ? 1 : 0;
-  if (p->policy == EKV_POLICY_TOPK) n += 2;
+  if (p->policy == EKV_POLICY_TOPK)
+    n += 1 + (topk_ws_bytes(seqs->batch * cache->num_kv_heads, seqs->max_pages, p->k) > 0 ? 2 : 1);
   else if (p->policy == EKV_POLICY_GAUSS) n += 3;
   else if (!full) return 0;
   return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap);

@@ -39,8 +39,12 @@ cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, i
 cudaError_t launch_gauss_stats(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq,
                                float scale, float alpha, const GaussWs& ws, cudaStream_t st,
                                int after_append = 0);
+// ws: topk_ws_bytes(U, max_pages, k) bytes (NULL when that is 0, or for the
+// one-stage path).
+size_t topk_ws_bytes(int units, int max_pages, int k);
+size_t topk_ws_bytes_upto(int units, int max_pages, int cap);  // the most any k ≤ cap needs
 cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
-                        int32_t* sel, int32_t* n_sel, cudaStream_t st);
+                        int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t st);
 cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, float alpha,
                                 float delta, int cap, const GaussWs& ws, int32_t* sel,
                                 int32_t* n_sel, float* tau_hat, cudaStream_t st);

@@ -2,8 +2,12 @@
 // 2605.21649) §2.B, "Sélection de Pages Top-k": per (sequence, KV head), the k
 // pages with the largest bounding-box score, ties to the lower logical page.
 //
-// One CTA per unit.  Scores become order-preserving uint32 keys, cached in
-// shared memory when the unit has at most kSmemKeys pages.  The k-th largest
+// One CTA per list.  Scores become order-preserving uint32 keys, cached in
+// shared memory when the list has at most kSmemKeys entries.  A unit with
+// more pages than that is done in two stages: chunks of kChunk pages each
+// keep their own k best (any page of the unit's k best is among its chunk's
+// k best under the same order), then one CTA selects k among those winners,
+// read through their page indices, so ties and order are unchanged.  The k-th largest
 // key K* is found by a radix select whose digits adapt to the keys: each
 // pass bins the keys of the current interval [lo, hi] into at most 4096
 // equal bins that span exactly that interval (bin = (key − lo) >> shift), so
@@ -23,37 +27,28 @@ namespace {
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kSmemKeys = 16384;
+constexpr int kChunk = 8192;    // pages per first-stage chunk of a long unit
 constexpr int kBins = 4096;
 constexpr int kDigitBits = 12;
 constexpr int kRankMax = 256;  // keys of the k-th key's bin ranked directly
 
-__global__ void __launch_bounds__(kTopkThreads)
-    topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
-                int max_pages, int Hkv, int k, int stride, int32_t* __restrict__ sel,
-                int32_t* __restrict__ n_sel) {
-  grid_dep_enter();
-  extern __shared__ uint32_t keys_s[];  // [min(max_pages, kSmemKeys)]
+// The k largest of n > k entries (key_of(i): order-preserving key of entry
+// i), ties to the lower position; writes idx_of(position) of each, in
+// ascending position order, to out[0..k) and k to *n_out.  The whole CTA
+// calls it.  keys_s: shared scratch of n keys when cache_keys.
+template <class KeyOf, class IdxOf>
+__device__ void select_k(int P, int k, KeyOf key_of, IdxOf idx_of, uint32_t* keys_s, bool cache_keys,
+                         int32_t* __restrict__ out, int32_t* __restrict__ n_out) {
   __shared__ unsigned int hist[2][kBins];
   __shared__ unsigned int w_a[kTopkWarps], w_b[kTopkWarps];
   __shared__ uint32_t rk_key[kRankMax];
   __shared__ int rk_idx[kRankMax];
   __shared__ unsigned int s_lo, s_hi, s_above, s_count, s_fill;
-
-  const int unit = blockIdx.x, b = unit / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int L;
-  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
-  int32_t* out = sel + static_cast<size_t>(unit) * stride;
-  const float* row = ub + static_cast<size_t>(unit) * max_pages;
-  if (P <= k) {
-    for (int i = tid; i < P; i += kTopkThreads) out[i] = i;
-    if (tid == 0) n_sel[unit] = P;
-    return;
-  }
-  const bool cached = P <= kSmemKeys;
+  const bool cached = cache_keys;
   unsigned int kmin = 0xffffffffu, kmax = 0u;
   for (int i = tid; i < P; i += kTopkThreads) {
-    const uint32_t key = float_key(row[i]);
+    const uint32_t key = key_of(i);
     if (cached) keys_s[i] = key;
     kmin = min(kmin, key);
     kmax = max(kmax, key);
@@ -76,7 +71,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
-  auto key_at = [&](int i) -> uint32_t { return cached ? keys_s[i] : float_key(row[i]); };
+  auto key_at = [&](int i) -> uint32_t { return cached ? keys_s[i] : key_of(i); };
 
   // The interval [lo, hi] holds the k-th largest key; krem of its keys are
   // still to be taken.  Each pass splits it into ≤ 4096 equal bins; once the
@@ -229,30 +224,153 @@ __global__ void __launch_bounds__(kTopkThreads)
     const unsigned int my_g = gt_before + __popc(bg & lower), my_e = eq_before + __popc(be & lower);
     if (gt) {
       const unsigned int pos = my_g + min(my_e, krem);
-      if (pos < static_cast<unsigned int>(k)) out[pos] = i;
+      if (pos < static_cast<unsigned int>(k)) out[pos] = idx_of(i);
     } else if (eq && my_e < krem) {
       const unsigned int pos = my_g + my_e;
-      if (pos < static_cast<unsigned int>(k)) out[pos] = i;
+      if (pos < static_cast<unsigned int>(k)) out[pos] = idx_of(i);
     }
     gt_before += __popc(bg);
     eq_before += __popc(be);
   }
-  if (tid == 0) n_sel[unit] = k;
+  if (tid == 0) *n_out = k;
+}
+
+// One unit per CTA (units of at most kSmemKeys pages).
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
+                int max_pages, int Hkv, int k, int stride, int32_t* __restrict__ sel,
+                int32_t* __restrict__ n_sel) {
+  grid_dep_enter();
+  extern __shared__ uint32_t keys_s[];  // [min(max_pages, kSmemKeys)]
+  const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
+  int L;
+  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
+  int32_t* out = sel + static_cast<size_t>(unit) * stride;
+  const float* row = ub + static_cast<size_t>(unit) * max_pages;
+  if (P <= k) {
+    for (int i = tid; i < P; i += kTopkThreads) out[i] = i;
+    if (tid == 0) n_sel[unit] = P;
+    return;
+  }
+  select_k(P, k, [&](int i) { return float_key(row[i]); }, [](int i) { return i; }, keys_s,
+           P <= kSmemKeys, out, n_sel + unit);
+}
+
+// First stage of a long unit: chunk c keeps its k best pages.
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_chunk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
+                      int max_pages, int Hkv, int k, int nchunk, int32_t* __restrict__ cand,
+                      int32_t* __restrict__ ccount) {
+  grid_dep_enter();
+  extern __shared__ uint32_t keys_s[];  // [kChunk]
+  const int c = blockIdx.x, unit = blockIdx.y, b = unit / Hkv, tid = threadIdx.x;
+  int L;
+  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
+  const int base = c * kChunk, n = max(0, min(kChunk, P - base));
+  int32_t* out = cand + (static_cast<size_t>(unit) * nchunk + c) * k;
+  int32_t* cnt = ccount + static_cast<size_t>(unit) * nchunk + c;
+  if (n <= k) {
+    for (int i = tid; i < n; i += kTopkThreads) out[i] = base + i;
+    if (tid == 0) *cnt = n;
+    return;
+  }
+  const float* row = ub + static_cast<size_t>(unit) * max_pages + base;
+  select_k(n, k, [&](int i) { return float_key(row[i]); }, [&](int i) { return base + i; }, keys_s, true,
+           out, cnt);
+}
+
+// Second stage: the unit's k best among its chunks' winners (in page order).
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_merge_kernel(const float* __restrict__ ub, int max_pages, int k, int nchunk,
+                      const int32_t* __restrict__ cand, const int32_t* __restrict__ ccount, int stride,
+                      int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
+  grid_dep_enter();
+  extern __shared__ uint32_t dyn_m[];  // [nchunk·k] page indices, then [nchunk·k] keys
+  __shared__ int s_off[65];
+  const int unit = blockIdx.x, tid = threadIdx.x;
+  int* cl = reinterpret_cast<int*>(dyn_m);
+  uint32_t* keys_s = dyn_m + static_cast<size_t>(nchunk) * k;
+  if (tid == 0) {
+    int o = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      s_off[c] = o;
+      o += max(0, min(k, ccount[static_cast<size_t>(unit) * nchunk + c]));
+    }
+    s_off[nchunk] = o;
+  }
+  __syncthreads();
+  for (int c = 0; c < nchunk; ++c) {
+    const int n = s_off[c + 1] - s_off[c];
+    const int32_t* src = cand + (static_cast<size_t>(unit) * nchunk + c) * k;
+    for (int i = tid; i < n; i += kTopkThreads) cl[s_off[c] + i] = src[i];
+  }
+  __syncthreads();
+  const int n2 = s_off[nchunk];
+  int32_t* out = sel + static_cast<size_t>(unit) * stride;
+  if (n2 <= k) {
+    for (int i = tid; i < n2; i += kTopkThreads) out[i] = cl[i];
+    if (tid == 0) n_sel[unit] = n2;
+    return;
+  }
+  const float* row = ub + static_cast<size_t>(unit) * max_pages;
+  select_k(n2, k, [&](int i) { return float_key(row[cl[i]]); }, [&](int i) { return cl[i]; }, keys_s, true,
+           out, n_sel + unit);
 }
 
 }  // namespace
 
+int topk_chunks(int max_pages) { return (max_pages + kChunk - 1) / kChunk; }
+
+size_t topk_ws_bytes(int units, int max_pages, int k) {
+  if (max_pages <= kSmemKeys) return 0;
+  const int nchunk = topk_chunks(max_pages);
+  if (nchunk > 64 || static_cast<size_t>(nchunk) * k > static_cast<size_t>(kSmemKeys)) return 0;  // single stage
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  return al(static_cast<size_t>(units) * nchunk * k * sizeof(int32_t)) +
+         al(static_cast<size_t>(units) * nchunk * sizeof(int32_t));
+}
+
+size_t topk_ws_bytes_upto(int units, int max_pages, int cap) {
+  if (max_pages <= kSmemKeys) return 0;
+  const int kmax = kSmemKeys / topk_chunks(max_pages);
+  return topk_ws_bytes(units, max_pages, cap < kmax ? cap : kmax);
+}
+
 cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
-                        int32_t* sel, int32_t* n_sel, cudaStream_t st) {
+                        int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t st) {
+  const int U = s.batch * Hkv;
+  const size_t static_smem = 2 * kBins * sizeof(unsigned int) + kRankMax * 8 + 1024;
+  if (ws != nullptr && topk_ws_bytes(U, s.max_pages, k) > 0) {
+    const int nchunk = topk_chunks(s.max_pages);
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    int32_t* cand = static_cast<int32_t*>(ws);
+    int32_t* ccount = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + al(static_cast<size_t>(U) * nchunk * k * sizeof(int32_t)));
+    const size_t smem1 = static_cast<size_t>(kChunk) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem1));
+    if (e != cudaSuccess) return e;
+    e = launch_k(topk_chunk_kernel, dim3(nchunk, U), dim3(kTopkThreads), smem1, st, ub, s.seq_lens, S,
+                 s.max_pages, Hkv, k, nchunk, cand, ccount);
+    if (e != cudaSuccess) return e;
+    const size_t smem2 = 2 * static_cast<size_t>(nchunk) * k * sizeof(uint32_t);
+    if (smem2 + static_smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem2));
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_k(topk_merge_kernel, dim3(U), dim3(kTopkThreads), smem2, st, ub, s.max_pages, k, nchunk,
+                 cand, ccount, stride, sel, n_sel);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   const int keys = s.max_pages < kSmemKeys ? s.max_pages : kSmemKeys;
   const size_t smem = static_cast<size_t>(keys) * sizeof(uint32_t);
-  const size_t static_smem = 2 * kBins * sizeof(unsigned int) + kRankMax * 8 + 512;
   if (smem + static_smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  const cudaError_t le = launch_k(topk_kernel, dim3(s.batch * Hkv), dim3(kTopkThreads), smem, st, ub,
+  const cudaError_t le = launch_k(topk_kernel, dim3(U), dim3(kTopkThreads), smem, st, ub,
                                   s.seq_lens, S, s.max_pages, Hkv, k, stride, sel, n_sel);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();

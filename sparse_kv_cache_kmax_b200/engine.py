@@ -80,7 +80,10 @@ class DecodeEngine:
         k = max(1, min(int(k0 or self.params.k or 1), P))
         while True:
             sel = a["sel"][: Bsz * Hkv * k].view(Bsz, Hkv, k)
-            B.ekv_select_topk(self.seqs, Hkv, self.S, a["ub"], k, sel, a["n"], stream)
+            if k not in a.setdefault("tk", {}):
+                n_tk = B.ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, self.cache, self.seqs, self.Hq, k)
+                a["tk"][k] = B.workspace(n_tk, dev) if n_tk else None
+            B.ekv_select_topk(self.seqs, Hkv, self.S, a["ub"], k, sel, a["n"], stream, ws=a["tk"][k])
             B.ekv_entmax_decode(self.cache, self.seqs, q, scale, alpha, sel, a["n"], k, a["out"], a["ws"],
                                 tau=a["tau"], stream=stream)
             B.ekv_exactness_certificate(self.seqs, Hkv, self.S, alpha, a["ub"], sel, a["n"], a["tau"], a["cert"],

@@ -106,7 +106,9 @@ class Gpu:
     def topk(self, ub, k):
         sel = torch.full((self.wl.batch, self.wl.num_kv_heads, k), -1, dtype=torch.int32, device="cuda")
         n = torch.zeros(self.wl.batch, self.wl.num_kv_heads, dtype=torch.int32, device="cuda")
-        B.ekv_select_topk(self.seqs, self.wl.num_kv_heads, self.wl.page_size, ub, k, sel, n)
+        n_tk = B.ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, self.cache, self.seqs, self.Hq, k)
+        ws = B.workspace(n_tk, "cuda") if n_tk else None
+        B.ekv_select_topk(self.seqs, self.wl.num_kv_heads, self.wl.page_size, ub, k, sel, n, ws=ws)
         return sel, n
 
     def gauss(self, alpha, delta, cap=None):

@@ -71,8 +71,13 @@ def test_validation_rejects_before_launch():
     assert L.ekv_score_pages(ctypes.byref(c), ctypes.byref(s), FAKE, 12, 0.1, FAKE, None) == 1   # Hq % Hkv
     assert L.ekv_score_pages(ctypes.byref(c), ctypes.byref(s), FAKE, 24, 0.1, FAKE, None) == 2   # G = 3
     assert L.ekv_score_pages(ctypes.byref(c), ctypes.byref(s), FAKE, 32, -1.0, FAKE, None) == 1
-    assert L.ekv_select_topk(ctypes.byref(s), 8, 16, FAKE, 0, FAKE, FAKE, None) == 1
-    assert L.ekv_select_topk(ctypes.byref(s), 8, 12, FAKE, 4, FAKE, FAKE, None) == 2
+    assert L.ekv_select_topk(ctypes.byref(s), 8, 16, FAKE, 0, FAKE, FAKE, None, 0, None) == 1
+    assert L.ekv_select_topk(ctypes.byref(s), 8, 12, FAKE, 4, FAKE, FAKE, None, 0, None) == 2
+    long = _seqs(max_pages=65536)
+    assert B.lib().ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, ctypes.byref(c), ctypes.byref(s), 32, 4) == 0
+    need = B.lib().ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, ctypes.byref(c), ctypes.byref(long), 32, 512)
+    assert need > 0
+    assert L.ekv_select_topk(ctypes.byref(long), 8, 16, FAKE, 512, FAKE, FAKE, 0x100000, 16, None) == 3
     assert _decode(c, s, alpha=1.0) == 1
     assert _decode(c, s, alpha=float("nan")) == 1
     assert _decode(c, s, sel=None) == 1                 # sel without n_sel

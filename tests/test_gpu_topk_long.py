@@ -1,0 +1,44 @@
+"""Top-k over sequences longer than one CTA's shared-memory key cache: the
+two-stage selection (chunks keep their k best, then k among those) against the
+one-stage kernel and the oracle's rule on the same scores ([EntmaxKV] §2.B)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sparse_kv_cache_kmax_b200 import binding as B
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("k,dup", [(512, False), (100, True), (2000, False)])
+def test_two_stage_topk_matches_one_stage_and_oracle(k, dup):
+    g = torch.Generator(device="cuda").manual_seed(77 + k)
+    batch, hkv, S, P = 2, 3, 16, 19000
+    lens = torch.tensor([P * S, (P - 777) * S - 5], dtype=torch.int32, device="cuda")
+    pt = torch.arange(batch * P, dtype=torch.int32, device="cuda").view(batch, P)
+    seqs = B.make_seqs(pt, lens)
+    ub = torch.randn(batch, hkv, P, generator=g, device="cuda")
+    if dup:  # heavy ties: scores on a coarse grid
+        ub = torch.round(ub * 4) / 4
+    kv = torch.empty(1, hkv, S, 128, dtype=torch.bfloat16, device="cuda")
+    cache = B.make_cache(kv, kv)
+    cache.num_phys_pages = batch * P
+    need = B.ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, cache, seqs, 4 * hkv, k)
+    assert need > 0
+    ws = B.workspace(need, "cuda")
+    s2 = torch.full((batch, hkv, k), -1, dtype=torch.int32, device="cuda")
+    n2 = torch.zeros(batch, hkv, dtype=torch.int32, device="cuda")
+    B.ekv_select_topk(seqs, hkv, S, ub, k, s2, n2, ws=ws)
+    s1 = torch.full_like(s2, -1)
+    n1 = torch.zeros_like(n2)
+    B.ekv_select_topk(seqs, hkv, S, ub, k, s1, n1)
+    torch.cuda.synchronize()
+    assert torch.equal(s1, s2) and torch.equal(n1, n2)
+    ubh = ub.double().cpu().numpy()
+    for b in range(batch):
+        pages = -(-int(lens[b]) // S)
+        for h in range(hkv):
+            want = O.select_topk(ubh[b, h, :pages], k)
+            assert int(n2[b, h]) == len(want)
+            assert np.array_equal(s2[b, h, : len(want)].cpu().numpy(), want), (b, h)
