@@ -305,6 +305,16 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
 EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* seqs,
                                       const ekv_step_params* params, int32_t num_q_heads);
 
+/*
+ * ekv_selftest_wait_timeout — exercises the failure path every bounded wait
+ * of the library shares: one GPU thread waits, for `polls` polls (1 to
+ * 1048576), on an mbarrier that nothing ever completes; the wait gives up,
+ * ORs EKV_EFLAG_TIMEOUT into the device error word and the kernel returns, so
+ * the context stays usable.  No source-page counterpart: a diagnostic for
+ * failure detection.
+ */
+EKV_API ekv_status ekv_selftest_wait_timeout(uint32_t polls, void* stream);
+
 /* Reads the sticky device error word into *flags (EKV_EFLAG_* bits) and clears
  * it.  Synchronises the device. */
 EKV_API ekv_status ekv_get_error(uint32_t* flags);

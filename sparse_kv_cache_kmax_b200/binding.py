@@ -21,7 +21,7 @@ __all__ = [
     "ekv_score_pages", "ekv_select_topk", "ekv_select_gauss", "ekv_entmax_decode",
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
     "ekv_entmax_decode_static_ws", "ekv_step_kernel_count", "ekv_softmax_decode", "EKV_OP_SOFTMAX_DECODE",
-    "ekv_exactness_certificate", "EKV_OP_SELECT_TOPK",
+    "ekv_exactness_certificate", "EKV_OP_SELECT_TOPK", "ekv_selftest_wait_timeout", "EKV_EFLAG_TIMEOUT",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
@@ -29,6 +29,7 @@ EKV_POLICY_TOPK, EKV_POLICY_GAUSS, EKV_POLICY_FULL = 0, 1, 2
 EKV_OP_SELECT_GAUSS, EKV_OP_ENTMAX_DECODE, EKV_OP_DECODE_STEP, EKV_OP_SOFTMAX_DECODE = 1, 2, 3, 4
 EKV_OP_SELECT_TOPK = 5
 EKV_EFLAG_BAD_PAGE, EKV_EFLAG_BAD_LEN, EKV_EFLAG_SEL_OVERFLOW, EKV_EFLAG_BAD_SEL = 1, 2, 4, 8
+EKV_EFLAG_TIMEOUT = 16
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libekv.so")
 
@@ -81,6 +82,7 @@ _SIGS = {
     "ekv_softmax_decode": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _P, _P, _I, _P, _P,
                            _P, _SZ, _P],
     "ekv_exactness_certificate": [ctypes.POINTER(Seqs), _I, _I, _I, _F, _P, _P, _P, _I, _P, _P, _P],
+    "ekv_selftest_wait_timeout": [ctypes.c_uint32, _P],
     "ekv_step_kernel_count": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams), _I],
     "ekv_entmax_decode_static_ws": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P,
                                     _P, _I, _I, _P, _P, _P, _P, _P],
@@ -230,6 +232,11 @@ def ekv_exactness_certificate(seqs, num_kv_heads, page_size, alpha, ub, sel, n_s
     _check("ekv_exactness_certificate", lib().ekv_exactness_certificate(
         ctypes.byref(seqs), num_kv_heads, page_size, tau.shape[1], alpha, _ptr(ub), _ptr(sel), _ptr(n_sel),
         sel.shape[-1], _ptr(tau), _ptr(certified), _stream(stream)))
+
+
+def ekv_selftest_wait_timeout(polls=1024, stream=None):
+    """One bounded wait that nothing satisfies: raises EKV_EFLAG_TIMEOUT."""
+    _check("ekv_selftest_wait_timeout", lib().ekv_selftest_wait_timeout(polls, _stream(stream)))
 
 
 def ekv_step_kernel_count(cache, seqs, params: StepParams, num_q_heads) -> int:

@@ -349,6 +349,11 @@ EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* se
   return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap);
 }
 
+EKV_API ekv_status ekv_selftest_wait_timeout(uint32_t polls, void* stream) {
+  if (polls < 1 || polls > (1u << 20)) return EKV_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_timeout_selftest(polls, static_cast<cudaStream_t>(stream)));
+}
+
 EKV_API ekv_status ekv_get_error(uint32_t* flags) {
   if (flags == nullptr) return EKV_ERR_INVALID_ARG;
   unsigned int v = 0u, zero = 0u;

@@ -53,6 +53,21 @@ __global__ void __launch_bounds__(kCertThreads)
 
 }  // namespace
 
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that
+// nothing ever arrives at, for `polls` polls; the wait gives up, raises
+// EKV_EFLAG_TIMEOUT and the kernel returns normally.
+__global__ void wait_timeout_selftest_kernel(unsigned int polls) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0u, polls);
+}
+
+cudaError_t launch_wait_timeout_selftest(unsigned int polls, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 1, 0, st>>>(polls);
+  return cudaGetLastError();
+}
+
 int certificate_smem_ok(int max_pages) { return (max_pages + 31) / 32 * 4 <= 48 * 1024; }
 
 cudaError_t launch_certificate(const ekv_seqs& s, int Hkv, int S, int Hq, float alpha, const float* ub,

@@ -315,8 +315,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned int parity
       : "memory");
   return done != 0u;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned int parity) {
-  for (unsigned int i = 0; i < kSpinLimit; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned int parity,
+                                          unsigned int limit = kSpinLimit) {
+  for (unsigned int i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   raise_flag(EKV_EFLAG_TIMEOUT);
   return false;

@@ -53,6 +53,12 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
                           int cap, int dense_v, float* out, float* tau, int32_t* support_count,
                           uint32_t* support_bits, const DecodeWs& ws, cudaStream_t st);
 
+// One bounded wait that nothing satisfies (certify.cu): raises EKV_EFLAG_TIMEOUT.
+cudaError_t launch_wait_timeout_selftest(unsigned int polls, cudaStream_t st);
+
+// Streaming multiprocessors of the current device (score.cu).
+int sm_count();
+
 // Exactness certificate per query head (certify.cu).
 int certificate_smem_ok(int max_pages);
 cudaError_t launch_certificate(const ekv_seqs& s, int Hkv, int S, int Hq, float alpha, const float* ub,

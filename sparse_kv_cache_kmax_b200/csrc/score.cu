@@ -654,17 +654,6 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
   }
 }
 
-int sm_count() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
 
 template <typename T, int D, int G, bool GAUSS>
 cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
@@ -727,6 +716,19 @@ StreamArgs base_args(const ekv_cache& c, const ekv_seqs& s, const void* q, int H
 }
 
 }  // namespace
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
 
 cudaError_t launch_score(const ekv_cache& c, const ekv_seqs& s, const void* q, int Hq, float scale,
                          float* ub, cudaStream_t st, int after_append) {

@@ -4,10 +4,10 @@
 //
 // One CTA per list.  Scores become order-preserving uint32 keys, cached in
 // shared memory when the list has at most kSmemKeys entries.  A unit with
-// more pages than that is done in two stages: chunks of kChunk pages each
-// keep their own k best (any page of the unit's k best is among its chunk's
-// k best under the same order), then one CTA selects k among those winners,
-// read through their page indices, so ties and order are unchanged.  The k-th largest
+// more pages than that is done in two stages: chunks of pages each keep their own k best (any page of
+// the unit's k best is among its chunk's k best under the same order), then
+// one CTA selects k among those winners, read through their page indices, so
+// ties and order are unchanged.  The k-th largest
 // key K* is found by a radix select whose digits adapt to the keys: each
 // pass bins the keys of the current interval [lo, hi] into at most 4096
 // equal bins that span exactly that interval (bin = (key − lo) >> shift), so
@@ -259,14 +259,14 @@ __global__ void __launch_bounds__(kTopkThreads)
 // First stage of a long unit: chunk c keeps its k best pages.
 __global__ void __launch_bounds__(kTopkThreads)
     topk_chunk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
-                      int max_pages, int Hkv, int k, int nchunk, int32_t* __restrict__ cand,
+                      int max_pages, int Hkv, int k, int chunk, int nchunk, int32_t* __restrict__ cand,
                       int32_t* __restrict__ ccount) {
   grid_dep_enter();
-  extern __shared__ uint32_t keys_s[];  // [kChunk]
+  extern __shared__ uint32_t keys_s[];  // [chunk]
   const int c = blockIdx.x, unit = blockIdx.y, b = unit / Hkv, tid = threadIdx.x;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
-  const int base = c * kChunk, n = max(0, min(kChunk, P - base));
+  const int base = c * chunk, n = max(0, min(chunk, P - base));
   int32_t* out = cand + (static_cast<size_t>(unit) * nchunk + c) * k;
   int32_t* cnt = ccount + static_cast<size_t>(unit) * nchunk + c;
   if (n <= k) {
@@ -319,38 +319,59 @@ __global__ void __launch_bounds__(kTopkThreads)
 
 }  // namespace
 
-int topk_chunks(int max_pages) { return (max_pages + kChunk - 1) / kChunk; }
+// Two-stage plan: chunk pages per first-stage CTA (0: one stage).  Only
+// units whose keys exceed one CTA's cache split (measured: splitting shorter
+// units to fill the GPU costs more in the second launch and its barriers
+// than it saves).
+struct TopkPlan {
+  int chunk, nchunk;
+};
+
+TopkPlan topk_plan(int units, int max_pages, int k) {
+  (void)units;
+  TopkPlan pl{0, 1};
+  if (max_pages <= kSmemKeys) return pl;
+  const int nchunk = (max_pages + kChunk - 1) / kChunk;
+  if (nchunk > 64 || static_cast<size_t>(nchunk) * k > static_cast<size_t>(kSmemKeys)) return pl;
+  const int chunk = ((max_pages + nchunk - 1) / nchunk + 31) / 32 * 32;
+  pl.chunk = chunk;
+  pl.nchunk = (max_pages + chunk - 1) / chunk;
+  return pl;
+}
 
 size_t topk_ws_bytes(int units, int max_pages, int k) {
-  if (max_pages <= kSmemKeys) return 0;
-  const int nchunk = topk_chunks(max_pages);
-  if (nchunk > 64 || static_cast<size_t>(nchunk) * k > static_cast<size_t>(kSmemKeys)) return 0;  // single stage
+  const TopkPlan pl = topk_plan(units, max_pages, k);
+  if (pl.chunk == 0) return 0;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  return al(static_cast<size_t>(units) * nchunk * k * sizeof(int32_t)) +
-         al(static_cast<size_t>(units) * nchunk * sizeof(int32_t));
+  return al(static_cast<size_t>(units) * pl.nchunk * k * sizeof(int32_t)) +
+         al(static_cast<size_t>(units) * pl.nchunk * sizeof(int32_t));
 }
 
 size_t topk_ws_bytes_upto(int units, int max_pages, int cap) {
-  if (max_pages <= kSmemKeys) return 0;
-  const int kmax = kSmemKeys / topk_chunks(max_pages);
-  return topk_ws_bytes(units, max_pages, cap < kmax ? cap : kmax);
+  size_t most = 0;
+  for (int k = 1; k <= cap && k <= max_pages; ++k) {
+    const size_t b = topk_ws_bytes(units, max_pages, k);
+    if (b > most) most = b;
+  }
+  return most;
 }
 
 cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
                         int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t st) {
   const int U = s.batch * Hkv;
   const size_t static_smem = 2 * kBins * sizeof(unsigned int) + kRankMax * 8 + 1024;
-  if (ws != nullptr && topk_ws_bytes(U, s.max_pages, k) > 0) {
-    const int nchunk = topk_chunks(s.max_pages);
+  const TopkPlan pl = topk_plan(U, s.max_pages, k);
+  if (ws != nullptr && pl.chunk > 0) {
+    const int nchunk = pl.nchunk;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     int32_t* cand = static_cast<int32_t*>(ws);
     int32_t* ccount = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + al(static_cast<size_t>(U) * nchunk * k * sizeof(int32_t)));
-    const size_t smem1 = static_cast<size_t>(kChunk) * sizeof(uint32_t);
+    const size_t smem1 = static_cast<size_t>(pl.chunk) * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem1));
     if (e != cudaSuccess) return e;
     e = launch_k(topk_chunk_kernel, dim3(nchunk, U), dim3(kTopkThreads), smem1, st, ub, s.seq_lens, S,
-                 s.max_pages, Hkv, k, nchunk, cand, ccount);
+                 s.max_pages, Hkv, k, pl.chunk, nchunk, cand, ccount);
     if (e != cudaSuccess) return e;
     const size_t smem2 = 2 * static_cast<size_t>(nchunk) * k * sizeof(uint32_t);
     if (smem2 + static_smem > 48 * 1024) {

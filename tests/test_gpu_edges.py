@@ -1,6 +1,8 @@
 """GPU edge cases: single-token and ragged sequences, budgets that cover the
 whole sequence, and data errors (bad page ids, lengths, selections, a full
 Gaussian selection buffer) that the kernels turn into error flags."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -121,3 +123,17 @@ def test_fp32_cache_full_size_tiny_config():
     if not np.array_equal(got, orc["sel"]):
         orc = oracle_unit(inp, 0, 0, sel=got)
     assert row_rel_err(np64(eng.out[0]), orc["o"]).max() <= OUT_TOL["f32"]
+
+
+def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
+    """Failure detection without a fault: a wait on an mbarrier that nothing
+    completes gives up after its poll limit, the sticky error word reports
+    EKV_EFLAG_TIMEOUT, and the next library call runs normally."""
+    flags = ctypes.c_uint32(0)
+    B.lib().ekv_get_error(ctypes.byref(flags))          # start from a clean word
+    B.ekv_selftest_wait_timeout(4096)
+    assert B.lib().ekv_get_error(ctypes.byref(flags)) == 0
+    assert flags.value & B.EKV_EFLAG_TIMEOUT
+    assert B.lib().ekv_get_error(ctypes.byref(flags)) == 0 and flags.value == 0   # cleared
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0                      # the context still works
