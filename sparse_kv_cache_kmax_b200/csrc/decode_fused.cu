@@ -611,15 +611,17 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   }
   __syncthreads();
 
-  // All warps walk the same support pages; warp r takes rows r, r+16, ...
-  // of each page and accumulates p·v over its rows for every head.
+  // Warps take whole support pages (page e goes to warp e mod 16).  Lane t
+  // computes p = [u − τ]_+^β of the page's token t for every head once; the
+  // row loop broadcasts them by shuffle and reads the V rows (staged in
+  // shared memory, else global), four at a time.
   float acc[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
 #pragma unroll 1
-  for (int e = 0; e < nsup; ++e) {
+  for (int e = warp; e < nsup; e += kFWarps) {
     const int j = list_s[e], nvv = nv_s[j], vs = vslot_s[j];
     const bf16* vbase;
     if (vs >= 0) {
@@ -629,27 +631,37 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
       vbase = static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * tile_elems;
     }
 #pragma unroll 1
-    for (int r = warp; r < nvv; r += kFWarps) {
-      float v[DPL];
-      const bf16* src = vbase + static_cast<size_t>(r) * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        v[0] = __uint_as_float(w.x << 16);
-        v[1] = __uint_as_float(w.x & 0xffff0000u);
-        v[2] = __uint_as_float(w.y << 16);
-        v[3] = __uint_as_float(w.y & 0xffff0000u);
-      } else {
-        const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
-        v[0] = __uint_as_float(w << 16);
-        v[1] = __uint_as_float(w & 0xffff0000u);
-      }
+    for (int t0 = 0; t0 < nvv; t0 += 32) {
+      float p[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float w = a.am1 * zs[h * zp + j * S + r] - s_tau[h];
-        if (w > 0.f) {
-          const float p = pow_beta_fast(w, a.beta, a.ipow);
+        p[h] = 0.f;
+        if (t0 + lane < nvv) {
+          const float w = a.am1 * zs[h * zp + j * S + t0 + lane] - s_tau[h];
+          if (w > 0.f) p[h] = pow_beta_fast(w, a.beta, a.ipow);
+        }
+      }
+      const int nr = min(32, nvv - t0);
+#pragma unroll 4
+      for (int r = 0; r < nr; ++r) {
+        float v[DPL];
+        const bf16* src = vbase + static_cast<size_t>(t0 + r) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(src);
+          v[0] = __uint_as_float(w.x << 16);
+          v[1] = __uint_as_float(w.x & 0xffff0000u);
+          v[2] = __uint_as_float(w.y << 16);
+          v[3] = __uint_as_float(w.y & 0xffff0000u);
+        } else {
+          const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
+          v[0] = __uint_as_float(w << 16);
+          v[1] = __uint_as_float(w & 0xffff0000u);
+        }
 #pragma unroll
-          for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(p, v[e2], acc[h][e2]);
+        for (int h = 0; h < G; ++h) {
+          const float pt = __shfl_sync(0xffffffffu, p[h], r);
+#pragma unroll
+          for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(pt, v[e2], acc[h][e2]);
         }
       }
     }
