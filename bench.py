@@ -36,16 +36,13 @@ UNIT = "(sequence×KV-head) decode steps/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic of one score-kernel launch at the default workload, from an ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of
-# the kernel's sources; stale entries read as null.
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture
 # of the bench workload's shape, keyed by a hash of the kernel's sources (a
 # changed kernel has no measured traffic until it is captured again)
 SCORE_FILES = ("score.cu", "common.cuh", "kernels.cuh")
 DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh", "kernels.cuh")
-SCORE_TRAFFIC = {"20c008979d406865": 138512128}   # profiles/score_kernel_clustered_128k.md
-DECODE_TRAFFIC = {"c11b559320073018": 57956352}   # profiles/fused_decode_kernel_clustered_128k.md
+SCORE_TRAFFIC = {"d0d585139e2ad614": 137794048}   # profiles/score_kernel_clustered_128k.md
+DECODE_TRAFFIC = {"c53939cbead460f5": 58092032}   # profiles/fused_decode_kernel_clustered_128k.md
 
 
 def kernel_hash(files=SCORE_FILES):
