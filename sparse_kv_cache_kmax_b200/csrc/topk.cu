@@ -2,208 +2,387 @@
 // 2605.21649) §2.B, "Sélection de Pages Top-k": per (sequence, KV head), the k
 // pages with the largest bounding-box score, ties to the lower logical page.
 //
-// One CTA per list.  Scores become order-preserving uint32 keys, cached in
-// shared memory when the list has at most kSmemKeys entries.  A unit with
-// more pages than that is done in two stages: chunks of pages each keep their own k best (any page of
+// One CTA per list.  Scores become order-preserving uint32 keys.  A list of
+// at most kRegKeys entries is held in registers, each thread owning a
+// contiguous run of 8 or 16 positions; a unit with more pages than that is
+// done in two stages: chunks of pages each keep their own k best (any page of
 // the unit's k best is among its chunk's k best under the same order), then
 // one CTA selects k among those winners, read through their page indices, so
-// ties and order are unchanged.  The k-th largest
-// key K* is found by a radix select whose digits adapt to the keys: each
-// pass bins the keys of the current interval [lo, hi] into at most 4096
-// equal bins that span exactly that interval (bin = (key − lo) >> shift), so
-// scores spread over all bins instead of piling into the few bins their
-// exponent bits would give.  The bin holding the k-th largest key becomes the
-// next interval; a pass with shift 0 leaves a single key value, K*, after at
-// most three passes (often two).  The output pass gives each thread a
-// contiguous run of pages, so one block scan of "taken" counts writes every
-// key > K* and the lowest-index (k − #{key > K*}) keys equal to K* in
-// ascending page order.  All arithmetic on keys is integer.
+// ties and order are unchanged.  The k-th largest key K* is found by a radix
+// select whose digits adapt to the keys: each pass bins the keys of the
+// current interval [lo, hi] into at most 4096 equal bins that span exactly
+// that interval (bin = (key − lo) >> shift), so scores spread over all bins
+// instead of piling into the few bins their exponent bits would give.  The bin
+// holding the k-th largest key becomes the next interval; once it holds few
+// keys they are ranked directly, and a pass with shift 0 leaves a single key
+// value, K*, after at most three passes.  The output gives each thread its run
+// of positions: one block scan of (#key > K*, #key = K*) places every key
+// > K* and the lowest-position (k − #{key > K*}) keys equal to K* in ascending
+// page order.  All arithmetic on keys is integer.
 #include "kernels.cuh"
 
 namespace ekv {
 
 namespace {
 
-constexpr int kTopkThreads = 1024;
+#ifndef EKV_TOPK_THREADS
+#define EKV_TOPK_THREADS 1024
+#endif
+constexpr int kTopkThreads = EKV_TOPK_THREADS;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kSmemKeys = 16384;
-constexpr int kChunk = 8192;    // pages per first-stage chunk of a long unit
+constexpr int kKeysPerThread = 8192 / kTopkThreads;   // registers per thread for lists ≤ 8192
+constexpr int kRegKeys = 2 * kKeysPerThread * kTopkThreads;   // longest list held in registers
+constexpr int kChunk = 8192;                  // pages per first-stage chunk of a long unit
 constexpr int kBins = 4096;
 constexpr int kDigitBits = 12;
 constexpr int kRankMax = 256;  // keys of the k-th key's bin ranked directly
+static_assert(kTopkThreads >= kRankMax && kTopkThreads <= 1024 && kTopkThreads % 32 == 0, "block size");
+static_assert(kBins % kTopkThreads == 0 && 8192 % kTopkThreads == 0, "bins and keys per thread");
 
-// The k largest of n > k entries (key_of(i): order-preserving key of entry
-// i), ties to the lower position; writes idx_of(position) of each, in
-// ascending position order, to out[0..k) and k to *n_out.  The whole CTA
-// calls it.  keys_s: shared scratch of n keys when cache_keys.
-template <class KeyOf, class IdxOf>
-__device__ void select_k(int P, int k, KeyOf key_of, IdxOf idx_of, uint32_t* keys_s, bool cache_keys,
-                         int32_t* __restrict__ out, int32_t* __restrict__ n_out) {
-  __shared__ unsigned int hist[2][kBins];
-  __shared__ unsigned int w_a[kTopkWarps], w_b[kTopkWarps];
-  __shared__ uint32_t rk_key[kRankMax];
-  __shared__ int rk_idx[kRankMax];
-  __shared__ unsigned int s_lo, s_hi, s_above, s_count, s_fill;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool cached = cache_keys;
-  unsigned int kmin = 0xffffffffu, kmax = 0u;
-  for (int i = tid; i < P; i += kTopkThreads) {
-    const uint32_t key = key_of(i);
-    if (cached) keys_s[i] = key;
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
+struct SelectShared {
+  unsigned int hist[2][kBins];
+  unsigned int w_a[kTopkWarps], w_b[kTopkWarps];
+  uint32_t rk_key[kRankMax];
+  int rk_idx[kRankMax];
+  unsigned int rk_rank[kRankMax];
+  unsigned int s_lo, s_hi, s_above, s_count, s_fill;
+};
+
+// Keys of a contiguous row of scores.
+struct RowKeys {
+  const float* row;
+  __device__ uint32_t operator()(int i) const { return float_key(row[i]); }
+  template <int KPT>
+  __device__ void load(int i0, int n, uint32_t (&key)[KPT]) const {
+    const float* src = row + i0;
+    if (i0 + KPT <= n && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+#pragma unroll
+      for (int v = 0; v < KPT / 4; ++v) {
+        const float4 f = reinterpret_cast<const float4*>(src)[v];
+        key[4 * v] = float_key(f.x);
+        key[4 * v + 1] = float_key(f.y);
+        key[4 * v + 2] = float_key(f.z);
+        key[4 * v + 3] = float_key(f.w);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) key[j] = i0 + j < n ? float_key(src[j]) : 0u;
+    }
   }
-  for (int i = tid; i < kBins; i += kTopkThreads) hist[0][i] = 0u;
+};
+
+// Keys of scattered entries of a row, read through a list of page indices.
+struct ListKeys {
+  const float* row;
+  const int* list;
+  __device__ uint32_t operator()(int i) const { return float_key(row[list[i]]); }
+  template <int KPT>
+  __device__ void load(int i0, int n, uint32_t (&key)[KPT]) const {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) key[j] = i0 + j < n ? float_key(row[list[i0 + j]]) : 0u;
+  }
+};
+
+// The interval [lo, hi] holds the k-th largest key with krem keys of it
+// still to take: bins its keys (count_bins(hc, lo, shift) adds every key of
+// the interval to hc), then moves [lo, hi] to the bin of the k-th key.  The
+// whole CTA calls it; returns the bin's key count.
+template <class CountBins>
+__device__ unsigned int narrow(SelectShared& sh, int cur, unsigned int& lo, unsigned int& hi,
+                               unsigned int& krem, CountBins count_bins) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned int range = hi - lo;
+  const int width = 32 - __clz(range);
+  const int shift = width > kDigitBits ? width - kDigitBits : 0;
+  const int top = static_cast<int>(range >> shift);
+  unsigned int* hc = sh.hist[cur];
+  count_bins(hc, lo, hi, shift);
+  for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[cur ^ 1][i] = 0u;  // next pass's bins
+  __syncthreads();
+  // thread t covers bins top − 4t − r (r = 0..3), counted from the top
+  unsigned int c[kBins / kTopkThreads], mine = 0u;
+#pragma unroll
+  for (int r = 0; r < kBins / kTopkThreads; ++r) {
+    const int bin = top - (kBins / kTopkThreads) * tid - r;
+    c[r] = bin >= 0 ? hc[bin] : 0u;
+    mine += c[r];
+  }
+  unsigned int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.w_a[warp] = incl;
+  __syncthreads();
+  const unsigned int wt = lane < kTopkWarps ? sh.w_a[lane] : 0u;
+  unsigned int wincl = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, wincl, o);
+    if (lane >= o) wincl += y;
+  }
+  unsigned int before = __shfl_sync(0xffffffffu, wincl - wt, warp) + incl - mine;
+  if (before < krem && before + mine >= krem) {  // this thread holds the k-th key's bin
+#pragma unroll
+    for (int r = 0; r < kBins / kTopkThreads; ++r) {
+      if (before < krem && before + c[r] >= krem) {
+        const int bin = top - (kBins / kTopkThreads) * tid - r;
+        sh.s_above = before;
+        sh.s_count = c[r];
+        const unsigned long long base =
+            static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bin) << shift);
+        sh.s_lo = static_cast<unsigned int>(base);
+        sh.s_hi = static_cast<unsigned int>(min(static_cast<unsigned long long>(hi), base + ((1ull << shift) - 1ull)));
+      }
+      before += c[r];
+    }
+  }
+  if (tid == 0) sh.s_fill = 0u;
+  __syncthreads();
+  krem -= sh.s_above;
+  lo = sh.s_lo;
+  hi = sh.s_hi;
+  return sh.s_count;
+}
+
+// K* from the cnt ≤ kRankMax keys in [lo, hi] gathered into rk_key/rk_idx:
+// ranked by (key descending, position ascending), the one of rank krem − 1.
+// The threads split into as many slices of the list as fit; each key's rank
+// is the sum over the slices.
+__device__ void rank_bin(SelectShared& sh, unsigned int cnt, unsigned int& lo, unsigned int& hi,
+                         unsigned int& krem) {
+  const int tid = threadIdx.x;
+  const int per = cnt <= 64u ? 64 : cnt <= 128u ? 128 : kRankMax;
+  const int nslice = kTopkThreads / per;
+  const int e = tid % per, slice = tid / per;
+  if (e < static_cast<int>(cnt) && slice < nslice) {
+    const uint32_t key = sh.rk_key[e];
+    const int idx = sh.rk_idx[e];
+    const unsigned int c0 = cnt * slice / nslice, c1 = cnt * (slice + 1) / nslice;
+    unsigned int rank = 0u, greater = 0u;
+    for (unsigned int c = c0; c < c1; ++c) {
+      const uint32_t kc = sh.rk_key[c];
+      greater += kc > key ? 1u : 0u;
+      rank += (kc > key || (kc == key && sh.rk_idx[c] < idx)) ? 1u : 0u;
+    }
+    if (c1 > c0) atomicAdd(&sh.rk_rank[e], rank | (greater << 16));
+  }
+  __syncthreads();
+  for (int i = tid; i < static_cast<int>(cnt); i += kTopkThreads) {
+    const unsigned int rg = sh.rk_rank[i];
+    if ((rg & 0xffffu) == krem - 1u) {
+      sh.s_lo = sh.rk_key[i];
+      sh.s_above = rg >> 16;
+    }
+  }
+  __syncthreads();
+  lo = hi = sh.s_lo;
+  krem -= sh.s_above;
+}
+
+// The k largest of n entries (kRegKeys ≥ n > k; keys.load fills a thread's
+// run of KPT positions), ties to the lower position; writes idx_of(position)
+// of each, in ascending position order, to out[0..k) and k to *n_out.  The
+// whole CTA calls it.
+template <int KPT, class Keys, class IdxOf>
+__device__ void select_k_reg(SelectShared& sh, int n, int k, const Keys& keys, IdxOf idx_of,
+                             int32_t* __restrict__ out, int32_t* __restrict__ n_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = tid * KPT;
+  uint32_t key[KPT];
+  keys.template load<KPT>(i0, n, key);
+  const int nv = max(0, min(KPT, n - i0));  // valid positions of this thread
+  unsigned int kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (j < nv) {
+      kmin = min(kmin, key[j]);
+      kmax = max(kmax, key[j]);
+    }
+  }
+  for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[0][i] = 0u;
+  for (int i = tid; i < kRankMax; i += kTopkThreads) sh.rk_rank[i] = 0u;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
   if (lane == 0) {
-    w_a[warp] = kmin;
-    w_b[warp] = kmax;
+    sh.w_a[warp] = kmin;
+    sh.w_b[warp] = kmax;
   }
   __syncthreads();
-  kmin = w_a[lane];
-  kmax = w_b[lane];
+  kmin = lane < kTopkWarps ? sh.w_a[lane] : 0xffffffffu;
+  kmax = lane < kTopkWarps ? sh.w_b[lane] : 0u;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
-  auto key_at = [&](int i) -> uint32_t { return cached ? keys_s[i] : key_of(i); };
+  __syncthreads();  // w_a / w_b are reused below
 
-  // The interval [lo, hi] holds the k-th largest key; krem of its keys are
-  // still to be taken.  Each pass splits it into ≤ 4096 equal bins; once the
-  // bin of the k-th key holds few keys, they are ranked directly.
   unsigned int lo = kmin, hi = kmax, krem = static_cast<unsigned int>(k);
   int cur = 0;
-  for (int pass = 0; pass < 4 && lo < hi; ++pass) {
-    const unsigned int range = hi - lo;
-    const int width = 32 - __clz(range);
-    const int shift = width > kDigitBits ? width - kDigitBits : 0;
-    const int nbins = static_cast<int>(range >> shift) + 1;
-    unsigned int* hc = hist[cur];
-    for (int base = 0; base < P; base += kTopkThreads) {
-      const int i = base + tid;
-      unsigned int bin = 0xffffffffu;  // outside the interval
-      if (i < P) {
-        const uint32_t key = key_at(i);
-        if (key >= lo && key <= hi) bin = (key - lo) >> shift;
-      }
-      const unsigned int b0 = __shfl_sync(0xffffffffu, bin, 0);
-      if (__all_sync(0xffffffffu, bin == b0)) {  // one bin for the whole warp
-        if (lane == 0 && b0 != 0xffffffffu) atomicAdd(&hc[b0], 32u);
-      } else if (bin != 0xffffffffu) {
-        atomicAdd(&hc[bin], 1u);
-      }
-    }
-    for (int i = tid; i < kBins; i += kTopkThreads) hist[cur ^ 1][i] = 0u;  // next pass's bins
-    __syncthreads();
-    // warp w covers bins top − 128w − 32r − lane (r = 0..3), counted from the top
-    const int top = nbins - 1;
-    unsigned int wsum = 0u;
-#pragma unroll
-    for (int r = 0; r < kBins / kTopkThreads; ++r) {
-      const int bin = top - 128 * warp - 32 * r - lane;
-      wsum += bin >= 0 ? hc[bin] : 0u;
-    }
-    wsum = __reduce_add_sync(0xffffffffu, wsum);
-    if (lane == 0) w_a[warp] = wsum;
-    __syncthreads();
-    const unsigned int wt = w_a[lane];
-    unsigned int wincl = wt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned int y = __shfl_up_sync(0xffffffffu, wincl, o);
-      if (lane >= o) wincl += y;
-    }
-    unsigned int before = __shfl_sync(0xffffffffu, wincl - wt, warp);
-    const unsigned int mine = __shfl_sync(0xffffffffu, wt, warp);
-    if (before < krem && before + mine >= krem) {  // this warp holds the k-th key's bin
 #pragma unroll 1
-      for (int r = 0; r < kBins / kTopkThreads; ++r) {
-        const int bin = top - 128 * warp - 32 * r - lane;
-        const unsigned int c = bin >= 0 ? hc[bin] : 0u;
-        unsigned int incl = c;
+  for (int pass = 0; pass < 4 && lo < hi; ++pass) {
+    // neighbouring positions often share a bin: one atomic per run of them
+    const unsigned int cnt = narrow(sh, cur, lo, hi, krem, [&](unsigned int* hc, unsigned int l, unsigned int h, int shift) {
+      unsigned int prev = 0xffffffffu, run = 0u;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
+      for (int j = 0; j < KPT; ++j) {
+        const bool in = j < nv && key[j] >= l && key[j] <= h;
+        const unsigned int bin = in ? (key[j] - l) >> shift : 0xffffffffu;
+        if (bin != prev) {
+          if (prev != 0xffffffffu) atomicAdd(&hc[prev], run);
+          prev = bin;
+          run = 0u;
         }
-        if (c > 0 && before + incl - c < krem && before + incl >= krem) {
-          s_above = before + incl - c;
-          s_count = c;
-          s_fill = 0u;
-          const unsigned long long base = static_cast<unsigned long long>(lo) + (static_cast<unsigned long long>(bin) << shift);
-          s_lo = static_cast<unsigned int>(base);
-          s_hi = static_cast<unsigned int>(min(static_cast<unsigned long long>(hi), base + ((1ull << shift) - 1ull)));
-        }
-        before += __shfl_sync(0xffffffffu, incl, 31);
-        if (before >= krem) break;
+        run += in ? 1u : 0u;
       }
-    }
-    __syncthreads();
-    krem -= s_above;
-    lo = s_lo;
-    hi = s_hi;
+      if (prev != 0xffffffffu) atomicAdd(&hc[prev], run);
+    });
     cur ^= 1;
-    const unsigned int cnt = s_count;
     if (lo < hi && cnt <= kRankMax) {
-      // rank the bin's keys by (key descending, page ascending): the one of
-      // rank krem − 1 is K*; of the keys equal to K*, krem − #{key > K*} go
-      for (int base = 0; base < P; base += kTopkThreads) {
-        const int i = base + tid;
-        if (i < P) {
-          const uint32_t key = key_at(i);
-          if (key >= lo && key <= hi) {
-            const unsigned int pos = atomicAdd(&s_fill, 1u);
-            rk_key[pos] = key;
-            rk_idx[pos] = i;
-          }
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        if (j < nv && key[j] >= lo && key[j] <= hi) {
+          const unsigned int pos = atomicAdd(&sh.s_fill, 1u);
+          sh.rk_key[pos] = key[j];
+          sh.rk_idx[pos] = i0 + j;
         }
       }
       __syncthreads();
-      if (tid < static_cast<int>(cnt)) {
-        const uint32_t key = rk_key[tid];
-        const int idx = rk_idx[tid];
-        unsigned int rank = 0u, greater = 0u;
-        for (unsigned int c = 0; c < cnt; ++c) {
-          const uint32_t kc = rk_key[c];
-          greater += kc > key ? 1u : 0u;
-          rank += (kc > key || (kc == key && rk_idx[c] < idx)) ? 1u : 0u;
-        }
-        if (rank == krem - 1u) {
-          s_lo = key;
-          s_above = greater;
-        }
-      }
-      __syncthreads();
-      lo = hi = s_lo;
-      krem -= s_above;
+      rank_bin(sh, cnt, lo, hi, krem);
       break;
     }
   }
 
-  // Output in ascending page order: warp w walks its chunk of pages with
-  // ballots; a taken page's slot = #{greater before} + min(#{equal before}, krem).
+  // Output: this thread's run of positions, after a block scan of its counts
+  // of keys > K* (low half) and = K* (high half); both stay below 2^16.
+  const uint32_t kth = lo;
+  unsigned int gt = 0u, eq = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    gt += (j < nv && key[j] > kth) ? 1u : 0u;
+    eq += (j < nv && key[j] == kth) ? 1u : 0u;
+  }
+  const unsigned int mine = gt | (eq << 16);
+  unsigned int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.w_b[warp] = incl;
+  __syncthreads();
+  const unsigned int wt = lane < kTopkWarps ? sh.w_b[lane] : 0u;
+  unsigned int wincl = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, wincl, o);
+    if (lane >= o) wincl += y;
+  }
+  const unsigned int before = __shfl_sync(0xffffffffu, wincl - wt, warp) + incl - mine;
+  unsigned int g = before & 0xffffu, e = before >> 16;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (j < nv) {
+      if (key[j] > kth) {
+        const unsigned int pos = g + min(e, krem);
+        if (pos < static_cast<unsigned int>(k)) out[pos] = idx_of(i0 + j);
+        ++g;
+      } else if (key[j] == kth) {
+        if (e < krem) {
+          const unsigned int pos = g + e;
+          if (pos < static_cast<unsigned int>(k)) out[pos] = idx_of(i0 + j);
+        }
+        ++e;
+      }
+    }
+  }
+  if (tid == 0) *n_out = k;
+}
+
+// The same selection for lists longer than kRegKeys (no key cache: each pass
+// re-reads the keys through key_of).  Positions are visited in strides of
+// the block; the output walks each warp's contiguous chunk with ballots.
+template <class KeyOf, class IdxOf>
+__device__ void select_k_long(SelectShared& sh, int P, int k, KeyOf key_of, IdxOf idx_of,
+                              int32_t* __restrict__ out, int32_t* __restrict__ n_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned int kmin = 0xffffffffu, kmax = 0u;
+  for (int i = tid; i < P; i += kTopkThreads) {
+    const uint32_t key = key_of(i);
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  }
+  for (int i = tid; i < kBins; i += kTopkThreads) sh.hist[0][i] = 0u;
+  for (int i = tid; i < kRankMax; i += kTopkThreads) sh.rk_rank[i] = 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sh.w_a[warp] = kmin;
+    sh.w_b[warp] = kmax;
+  }
+  __syncthreads();
+  kmin = lane < kTopkWarps ? sh.w_a[lane] : 0xffffffffu;
+  kmax = lane < kTopkWarps ? sh.w_b[lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  __syncthreads();
+
+  unsigned int lo = kmin, hi = kmax, krem = static_cast<unsigned int>(k);
+  int cur = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 4 && lo < hi; ++pass) {
+    const unsigned int cnt = narrow(sh, cur, lo, hi, krem, [&](unsigned int* hc, unsigned int l, unsigned int h, int shift) {
+      for (int i = tid; i < P; i += kTopkThreads) {
+        const uint32_t key = key_of(i);
+        if (key >= l && key <= h) atomicAdd(&hc[(key - l) >> shift], 1u);
+      }
+    });
+    cur ^= 1;
+    if (lo < hi && cnt <= kRankMax) {
+      for (int i = tid; i < P; i += kTopkThreads) {
+        const uint32_t key = key_of(i);
+        if (key >= lo && key <= hi) {
+          const unsigned int pos = atomicAdd(&sh.s_fill, 1u);
+          sh.rk_key[pos] = key;
+          sh.rk_idx[pos] = i;
+        }
+      }
+      __syncthreads();
+      rank_bin(sh, cnt, lo, hi, krem);
+      break;
+    }
+  }
+
+  // warp w walks its chunk of pages with ballots; a taken page's slot =
+  // #{greater before} + min(#{equal before}, krem).
   const uint32_t kth = lo;
   const int cw = (((P + kTopkWarps - 1) / kTopkWarps) + 31) & ~31;
   const int c0 = warp * cw, c1 = min(P, c0 + cw);
   unsigned int ng = 0u, ne = 0u;
   for (int i0 = c0; i0 < c1; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t key = i < c1 ? key_at(i) : 0u;
+    const uint32_t key = i < c1 ? key_of(i) : 0u;
     ng += __popc(__ballot_sync(0xffffffffu, i < c1 && key > kth));
     ne += __popc(__ballot_sync(0xffffffffu, i < c1 && key == kth));
   }
-  __syncthreads();  // w_a / w_b were read above
   if (lane == 0) {
-    w_a[warp] = ng;
-    w_b[warp] = ne;
+    sh.w_a[warp] = ng;
+    sh.w_b[warp] = ne;
   }
   __syncthreads();
-  unsigned int xg = w_a[lane], xe = w_b[lane], ig = xg, ie = xe;
+  unsigned int xg = lane < kTopkWarps ? sh.w_a[lane] : 0u, xe = lane < kTopkWarps ? sh.w_b[lane] : 0u;
+  unsigned int ig = xg, ie = xe;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned int yg = __shfl_up_sync(0xffffffffu, ig, o);
@@ -218,7 +397,7 @@ __device__ void select_k(int P, int k, KeyOf key_of, IdxOf idx_of, uint32_t* key
   const unsigned int lower = (1u << lane) - 1u;
   for (int i0 = c0; i0 < c1; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t key = i < c1 ? key_at(i) : 0u;
+    const uint32_t key = i < c1 ? key_of(i) : 0u;
     const bool gt = i < c1 && key > kth, eq = i < c1 && key == kth;
     const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
     const unsigned int my_g = gt_before + __popc(bg & lower), my_e = eq_before + __popc(be & lower);
@@ -235,13 +414,29 @@ __device__ void select_k(int P, int k, KeyOf key_of, IdxOf idx_of, uint32_t* key
   if (tid == 0) *n_out = k;
 }
 
-// One unit per CTA (units of at most kSmemKeys pages).
+// Dispatch on the list length.
+template <class Keys, class IdxOf>
+__device__ void select_k(SelectShared& sh, int n, int k, const Keys& keys, IdxOf idx_of,
+                         int32_t* __restrict__ out, int32_t* __restrict__ n_out) {
+  if (k < 1) {
+    if (threadIdx.x == 0) *n_out = 0;
+    return;
+  }
+  if (n <= kKeysPerThread * kTopkThreads)
+    select_k_reg<kKeysPerThread>(sh, n, k, keys, idx_of, out, n_out);
+  else if (n <= kRegKeys)
+    select_k_reg<2 * kKeysPerThread>(sh, n, k, keys, idx_of, out, n_out);
+  else
+    select_k_long(sh, n, k, keys, idx_of, out, n_out);
+}
+
+// One unit per CTA.
 __global__ void __launch_bounds__(kTopkThreads)
     topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
                 int max_pages, int Hkv, int k, int stride, int32_t* __restrict__ sel,
                 int32_t* __restrict__ n_sel) {
   grid_dep_enter();
-  extern __shared__ uint32_t keys_s[];  // [min(max_pages, kSmemKeys)]
+  __shared__ SelectShared sh;
   const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
@@ -252,8 +447,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     if (tid == 0) n_sel[unit] = P;
     return;
   }
-  select_k(P, k, [&](int i) { return float_key(row[i]); }, [](int i) { return i; }, keys_s,
-           P <= kSmemKeys, out, n_sel + unit);
+  select_k(sh, P, k, RowKeys{row}, [](int i) { return i; }, out, n_sel + unit);
 }
 
 // First stage of a long unit: chunk c keeps its k best pages.
@@ -262,7 +456,7 @@ __global__ void __launch_bounds__(kTopkThreads)
                       int max_pages, int Hkv, int k, int chunk, int nchunk, int32_t* __restrict__ cand,
                       int32_t* __restrict__ ccount) {
   grid_dep_enter();
-  extern __shared__ uint32_t keys_s[];  // [chunk]
+  __shared__ SelectShared sh;
   const int c = blockIdx.x, unit = blockIdx.y, b = unit / Hkv, tid = threadIdx.x;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
@@ -275,8 +469,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     return;
   }
   const float* row = ub + static_cast<size_t>(unit) * max_pages + base;
-  select_k(n, k, [&](int i) { return float_key(row[i]); }, [&](int i) { return base + i; }, keys_s, true,
-           out, cnt);
+  select_k(sh, n, k, RowKeys{row}, [&](int i) { return base + i; }, out, cnt);
 }
 
 // Second stage: the unit's k best among its chunks' winners (in page order).
@@ -285,11 +478,10 @@ __global__ void __launch_bounds__(kTopkThreads)
                       const int32_t* __restrict__ cand, const int32_t* __restrict__ ccount, int stride,
                       int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
   grid_dep_enter();
-  extern __shared__ uint32_t dyn_m[];  // [nchunk·k] page indices, then [nchunk·k] keys
+  extern __shared__ int cl[];  // [nchunk·k] page indices of the chunks' winners
+  __shared__ SelectShared sh;
   __shared__ int s_off[65];
   const int unit = blockIdx.x, tid = threadIdx.x;
-  int* cl = reinterpret_cast<int*>(dyn_m);
-  uint32_t* keys_s = dyn_m + static_cast<size_t>(nchunk) * k;
   if (tid == 0) {
     int o = 0;
     for (int c = 0; c < nchunk; ++c) {
@@ -313,14 +505,13 @@ __global__ void __launch_bounds__(kTopkThreads)
     return;
   }
   const float* row = ub + static_cast<size_t>(unit) * max_pages;
-  select_k(n2, k, [&](int i) { return float_key(row[cl[i]]); }, [&](int i) { return cl[i]; }, keys_s, true,
-           out, n_sel + unit);
+  select_k(sh, n2, k, ListKeys{row, cl}, [&](int i) { return cl[i]; }, out, n_sel + unit);
 }
 
 }  // namespace
 
 // Two-stage plan: chunk pages per first-stage CTA (0: one stage).  Only
-// units whose keys exceed one CTA's cache split (measured: splitting shorter
+// units whose keys exceed one CTA's registers split (measured: splitting shorter
 // units to fill the GPU costs more in the second launch and its barriers
 // than it saves).
 struct TopkPlan {
@@ -330,9 +521,9 @@ struct TopkPlan {
 TopkPlan topk_plan(int units, int max_pages, int k) {
   (void)units;
   TopkPlan pl{0, 1};
-  if (max_pages <= kSmemKeys) return pl;
+  if (max_pages <= kRegKeys) return pl;
   const int nchunk = (max_pages + kChunk - 1) / kChunk;
-  if (nchunk > 64 || static_cast<size_t>(nchunk) * k > static_cast<size_t>(kSmemKeys)) return pl;
+  if (nchunk > 64 || static_cast<size_t>(nchunk) * k > static_cast<size_t>(kRegKeys)) return pl;
   const int chunk = ((max_pages + nchunk - 1) / nchunk + 31) / 32 * 32;
   pl.chunk = chunk;
   pl.nchunk = (max_pages + chunk - 1) / chunk;
@@ -359,22 +550,17 @@ size_t topk_ws_bytes_upto(int units, int max_pages, int cap) {
 cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int k, int stride,
                         int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t st) {
   const int U = s.batch * Hkv;
-  const size_t static_smem = 2 * kBins * sizeof(unsigned int) + kRankMax * 8 + 1024;
   const TopkPlan pl = topk_plan(U, s.max_pages, k);
   if (ws != nullptr && pl.chunk > 0) {
     const int nchunk = pl.nchunk;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     int32_t* cand = static_cast<int32_t*>(ws);
     int32_t* ccount = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + al(static_cast<size_t>(U) * nchunk * k * sizeof(int32_t)));
-    const size_t smem1 = static_cast<size_t>(pl.chunk) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem1));
+    cudaError_t e = launch_k(topk_chunk_kernel, dim3(nchunk, U), dim3(kTopkThreads), 0, st, ub, s.seq_lens, S,
+                             s.max_pages, Hkv, k, pl.chunk, nchunk, cand, ccount);
     if (e != cudaSuccess) return e;
-    e = launch_k(topk_chunk_kernel, dim3(nchunk, U), dim3(kTopkThreads), smem1, st, ub, s.seq_lens, S,
-                 s.max_pages, Hkv, k, pl.chunk, nchunk, cand, ccount);
-    if (e != cudaSuccess) return e;
-    const size_t smem2 = 2 * static_cast<size_t>(nchunk) * k * sizeof(uint32_t);
-    if (smem2 + static_smem > 48 * 1024) {
+    const size_t smem2 = static_cast<size_t>(nchunk) * k * sizeof(int32_t);
+    if (smem2 + sizeof(SelectShared) + 512 > 48 * 1024) {
       e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem2));
       if (e != cudaSuccess) return e;
@@ -384,14 +570,7 @@ cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int 
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  const int keys = s.max_pages < kSmemKeys ? s.max_pages : kSmemKeys;
-  const size_t smem = static_cast<size_t>(keys) * sizeof(uint32_t);
-  if (smem + static_smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  const cudaError_t le = launch_k(topk_kernel, dim3(U), dim3(kTopkThreads), smem, st, ub,
+  const cudaError_t le = launch_k(topk_kernel, dim3(U), dim3(kTopkThreads), 0, st, ub,
                                   s.seq_lens, S, s.max_pages, Hkv, k, stride, sel, n_sel);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();

@@ -42,3 +42,38 @@ def test_two_stage_topk_matches_one_stage_and_oracle(k, dup):
             want = O.select_topk(ubh[b, h, :pages], k)
             assert int(n2[b, h]) == len(want)
             assert np.array_equal(s2[b, h, : len(want)].cpu().numpy(), want), (b, h)
+
+
+@pytest.mark.parametrize("dup", [False, True])
+def test_one_stage_topk_lengths(dup):
+    """One CTA per unit at lengths on both sides of 8 and 16 keys per thread,
+    rows not 16-byte aligned (odd row pitch), k from 1 to P − 1."""
+    g = torch.Generator(device="cuda").manual_seed(5 + dup)
+    pages = [5, 300, 8191, 8192, 8193, 12345, 16383]
+    batch, hkv, S, maxp = len(pages), 2, 16, 16383
+    lens = torch.tensor([p * S - 3 for p in pages], dtype=torch.int32, device="cuda")
+    pt = torch.arange(batch * maxp, dtype=torch.int32, device="cuda").view(batch, maxp)
+    seqs = B.make_seqs(pt, lens)
+    ub = torch.randn(batch, hkv, maxp, generator=g, device="cuda")
+    if dup:
+        ub = torch.round(ub * 4) / 4
+    ubh = ub.double().cpu().numpy()
+    for k in (1, 256, 4000):
+        sel = torch.full((batch, hkv, k), -1, dtype=torch.int32, device="cuda")
+        n = torch.zeros(batch, hkv, dtype=torch.int32, device="cuda")
+        B.ekv_select_topk(seqs, hkv, S, ub, k, sel, n)
+        torch.cuda.synchronize()
+        for b, P in enumerate(pages):
+            for h in range(hkv):
+                want = O.select_topk(ubh[b, h, :P], k)
+                assert int(n[b, h]) == len(want) == min(k, P)
+                assert np.array_equal(sel[b, h, : len(want)].cpu().numpy(), want), (k, b, h)
+    # k = P − 1 on the longest unit
+    k = pages[-1] - 1
+    sel = torch.full((batch, hkv, k), -1, dtype=torch.int32, device="cuda")
+    n = torch.zeros(batch, hkv, dtype=torch.int32, device="cuda")
+    B.ekv_select_topk(seqs, hkv, S, ub, k, sel, n)
+    torch.cuda.synchronize()
+    for h in range(hkv):
+        want = O.select_topk(ubh[-1, h, : pages[-1]], k)
+        assert np.array_equal(sel[-1, h, :k].cpu().numpy(), want)
