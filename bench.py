@@ -42,7 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 SCORE_FILES = ("score.cu", "common.cuh", "kernels.cuh")
 DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh", "kernels.cuh")
 SCORE_TRAFFIC = {"d0d585139e2ad614": 137794048}   # profiles/score_kernel_clustered_128k.md
-DECODE_TRAFFIC = {"c53939cbead460f5": 58092032}   # profiles/fused_decode_kernel_clustered_128k.md
+DECODE_TRAFFIC = {"f4f00457b9e63761": 56003584}   # profiles/fused_decode_kernel_clustered_128k.md
 
 
 def kernel_hash(files=SCORE_FILES):

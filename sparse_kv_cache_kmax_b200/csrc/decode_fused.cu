@@ -11,10 +11,10 @@
 //     bulk async copies (one copy = one contiguous S×d K tile) and scores
 //     them on tensor cores (m16n8k16, rows of the tile loaded from shared
 //     memory straight into A fragments).  Scores z and page maxima stay in
-//     shared memory.  The CTA then pushes its per-head maxima to the CTAs
-//     that solve those heads and starts bulk copies of the V tiles of the
-//     pages that can hold support (a page maximum within 1 of the run's
-//     maximum, in u = (α−1)·z units: τ ≥ max u − 1).
+//     shared memory.  The CTA then pushes its per-head maxima to every CTA
+//     and, after the barrier, starts bulk copies of the V tiles of the pages
+//     that can hold support (a page maximum within 1 of the unit's maximum,
+//     in u = (α−1)·z units: τ ≥ max u − 1).
 //  2. τ: query head h is solved by CTA h mod C on the head's scores of the
 //     whole unit, gathered from the cluster's shared memory (DSMEM) in token
 //     order: Σ[u − τ]_+^β = 1, β = 1/(α−1) (see cta_solve_tau).  The solver
@@ -381,8 +381,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   __shared__ uint64_t vbars[kFMaxVSlots];
   __shared__ TauShared tsh;
   __shared__ float s_tau[G];
-  __shared__ float s_mloc[G];
-  __shared__ float mlocs[kFMaxHeads][kFMaxCluster];  // run maxima of the heads this CTA solves
+  __shared__ float mall[kFMaxHeads][kFMaxCluster];  // run maxima: [head][CTA rank]
   __shared__ int s_vcount;
   __shared__ int scan_scratch[32];
 
@@ -502,43 +501,76 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     }
   }
   __syncthreads();
-  // run maxima per head, pushed to the head's solver
+  // run maxima per head, pushed to every CTA of the cluster
   for (int h = warp; h < G; h += kFWarps) {
     float m = -INFINITY;
     for (int j = lane; j < np; j += 32) m = fmaxf(m, pm[h * spc + j]);
     m = warp_max(m);
-    if (lane == 0) {
-      s_mloc[h] = m;
-      cluster.map_shared_rank(&mlocs[0][0], h % C)[(h / C) * kFMaxCluster + rank] = m;
-    }
-  }
-  __syncthreads();
-  // V tiles of the pages that can hold support start moving into shared memory
-  for (int j = tid; j < np; j += kFThreads) {
-    const int ph = phys_s[j];
-    bool cand = ph >= 0 && a.dense_v != 0;
-    if (ph >= 0 && !cand) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pz = pm[h * spc + j];
-        if (pz > -INFINITY && a.am1 * pz > a.am1 * s_mloc[h] - 1.0f) cand = true;
-      }
-    }
-    int vs = -1;
-    if (cand) {
-      const int sidx = atomicAdd(&s_vcount, 1);
-      if (sidx < f.nvslots) {
-        vs = sidx;
-        fence_proxy_async_smem();  // K tiles read from this area come before the copy
-        mbar_arrive_expect_tx(&vbars[vs], static_cast<unsigned int>(f.tile_bytes));
-        bulk_g2s(vtiles + static_cast<size_t>(vs) * f.tile_bytes,
-                 static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * tile_elems,
-                 static_cast<unsigned int>(f.tile_bytes), &vbars[vs]);
-      }
-    }
-    vslot_s[j] = vs;
+    if (lane < C) cluster.map_shared_rank(&mall[0][0], lane)[h * kFMaxCluster + rank] = m;
   }
   cluster.sync();
+
+  // V tiles of the pages that can hold support start moving into shared
+  // memory: τ ≥ max u − 1 over the unit, so a page whose maximum is not above
+  // that for some head holds no support.  When the candidates outnumber the
+  // slots, the slots go to the pages nearest their head's maximum (ties to
+  // the lower page), where the support lies.
+  {
+    float top[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float m = -INFINITY;
+      for (int r = 0; r < C; ++r) m = fmaxf(m, mall[h][r]);
+      top[h] = a.am1 * m;
+    }
+    float* dist = reinterpret_cast<float*>(list_s);  // [np], until the V list reuses it
+    int ncand = 0;
+    for (int j0 = 0; j0 < np; j0 += kFThreads) {
+      const int j = j0 + tid;
+      float d = -INFINITY;
+      if (j < np && phys_s[j] >= 0) {
+        if (a.dense_v) {
+          d = 0.f;
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pz = pm[h * spc + j];
+            if (pz > -INFINITY) d = fmaxf(d, a.am1 * pz - top[h]);
+          }
+          if (!(d > -1.0f)) d = -INFINITY;
+        }
+      }
+      if (j < np) dist[j] = d;
+      ncand += __syncthreads_count(d > -INFINITY);
+    }
+    const bool ranked = ncand > f.nvslots;
+    if (ranked && tid == 0) s_vcount = ncand;
+    for (int j = tid; j < np; j += kFThreads) {
+      const float d = dist[j];
+      int vs = -1;
+      if (d > -INFINITY) {
+        int slot;
+        if (ranked) {
+          slot = 0;
+          for (int i = 0; i < np; ++i) {
+            const float di = dist[i];
+            slot += (di > d || (di == d && i < j)) ? 1 : 0;
+          }
+        } else {
+          slot = atomicAdd(&s_vcount, 1);
+        }
+        if (slot < f.nvslots) {
+          vs = slot;
+          fence_proxy_async_smem();  // K tiles read from this area come before the copy
+          mbar_arrive_expect_tx(&vbars[vs], static_cast<unsigned int>(f.tile_bytes));
+          bulk_g2s(vtiles + static_cast<size_t>(vs) * f.tile_bytes,
+                   static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * tile_elems,
+                   static_cast<unsigned int>(f.tile_bytes), &vbars[vs]);
+        }
+      }
+      vslot_s[j] = vs;
+    }
+  }
 
   // ---------------------------------------------------------------- 2. τ
   const int tpc = spc * S;
@@ -546,10 +578,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   float* zh = reinterpret_cast<float*>(ring);
   float* cand = zh + ((n_tok + 31) & ~31);
   const size_t words = static_cast<size_t>(a.words);
-  for (int h = rank, hl = 0; h < G; h += C, ++hl) {
+  for (int h = rank; h < G; h += C) {
     const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h;
     float m = -INFINITY;
-    for (int r = 0; r < C; ++r) m = fmaxf(m, mlocs[hl][r]);
+    for (int r = 0; r < C; ++r) m = fmaxf(m, mall[h][r]);
     float tau = INFINITY;  // no finite score: no support, zero output
     if (m > -INFINITY) {
       const float um = a.am1 * m;
