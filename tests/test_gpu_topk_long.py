@@ -1,4 +1,4 @@
-"""Top-k over sequences longer than one CTA's shared-memory key cache: the
+"""Top-k over sequences longer than one CTA holds in registers (16384 pages): the
 two-stage selection (chunks keep their k best, then k among those) against the
 one-stage kernel and the oracle's rule on the same scores ([EntmaxKV] §2.B)."""
 import numpy as np
