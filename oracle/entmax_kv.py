@@ -44,7 +44,7 @@ __all__ = [
     "round_bf16", "round_to", "page_metadata", "bbox_upper_bound",
     "page_scores", "select_topk", "gauss_truncated_power_mean",
     "gauss_tau_hat", "select_gauss", "entmax_threshold", "entmax_probs",
-    "entmax_attention", "softmax_attention", "unit_pages", "decode_unit",
+    "entmax_attention", "softmax_attention", "softmax_dropped_mass", "unit_pages", "decode_unit",
     "build_page_meta", "append_token", "ENTMAX_SORT_ALPHAS",
     "exactness_certificate", "adaptive_topk",
 ]
@@ -376,11 +376,28 @@ def entmax_attention(q, K, V, scale, alpha):
 
 
 def softmax_attention(q, K, V, scale):
-    """Dense softmax attention (the full-cache softmax decode of [EntmaxKV] §4)."""
+    """Dense softmax attention (the full-cache softmax decode of [EntmaxKV] §4).
+
+    Also returns lse [G] = log Σ_i e^{z_i}, computed as m + log Σ_i e^{z_i − m}
+    with m the row maximum, so that p_i = e^{z_i − lse}."""
     z = scale * (np.asarray(q, np.float64) @ np.asarray(K, np.float64).T)
-    w = np.exp(z - z.max(axis=1, keepdims=True))
-    w /= w.sum(axis=1, keepdims=True)
-    return {"o": w @ np.asarray(V, np.float64), "p": w}
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    s = e.sum(axis=1, keepdims=True)
+    w = e / s
+    return {"o": w @ np.asarray(V, np.float64), "p": w, "lse": (m + np.log(s))[:, 0]}
+
+
+def softmax_dropped_mass(q, K, kept, scale):
+    """Softmax weight that a kept token set leaves out, per query head.
+
+    [EntmaxKV] §3 "Borne d'Erreur": the error of attending over a subset is
+    bounded through the attention mass of the dropped tokens.  Here that mass
+    is the full-cache softmax weight summed over the tokens not kept:
+    δ_h = Σ_{i ∉ kept} p_{h,i}.  q: [G, d]; K: [T, d] every token; kept: [T]
+    booleans.  Returns δ [G]."""
+    p = softmax_attention(q, K, np.zeros((np.shape(K)[0], 1)), scale)["p"]
+    return p[:, ~np.asarray(kept, bool)].sum(axis=1)
 
 
 # --------------------------------------------------------------------------

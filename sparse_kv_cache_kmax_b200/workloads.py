@@ -217,3 +217,9 @@ def make_inputs(wl: Workload, seed: int, device="cpu", n_new: int = 1) -> dict:
         "max_pages": max_pages, "num_phys": num_phys,
         "scale": wl.scale,
     }
+
+
+def gauss_cap(wl: Workload, max_pages: int) -> int:
+    """Pages a unit may keep under the Gaussian policy (the ``cap`` of
+    ekv_select_gauss / ekv_decode_step): every page of the sequence."""
+    return int(max_pages)

@@ -50,9 +50,7 @@ def _oracle(inp, b, h, pages=None):
     qg = q_group(inp, b, h)
     scale = float(np.float32(wl.scale))
     r = O.softmax_attention(qg, K, V, scale)
-    z = scale * (qg @ K.T)
-    lse = z.max(axis=1) + np.log(np.exp(z - z.max(axis=1, keepdims=True)).sum(axis=1))
-    return r["o"], lse
+    return r["o"], r["lse"]
 
 
 def test_softmax_full_cache_matches_oracle(case):
@@ -82,6 +80,36 @@ def test_softmax_over_a_selection_matches_oracle(case):
             rows = slice(h * G, (h + 1) * G)
             err = row_rel_err(np64(out[b, rows]), o_ref)
             assert np.all(err <= OUT_TOL[wl.dtype]), (b, h, err.max())
+            assert np.allclose(np64(lse[b, rows]), lse_ref, rtol=0, atol=2e-4 * max(1.0, np.abs(lse_ref).max()))
+
+
+def test_dropped_mass_matches_oracle(case):
+    """[EntmaxKV] §3 "Borne d'Erreur": the softmax mass a top-k selection
+    leaves out, as the benchmark computes it from the two GPU decodes
+    (1 − e^(lse_sel − lse_full)), against the oracle's full-cache softmax
+    weight summed over the tokens of the pages not kept."""
+    wl, inp, gpu = case
+    gpu.build_meta()
+    k = 8
+    sel, n = gpu.topk(gpu.score(), k)
+    _, lse_sel = _run(gpu, sel, n, k)
+    _, lse_all = _run(gpu)
+    drop = 1.0 - np.exp(np64(lse_sel) - np64(lse_all))
+    G, S = wl.group, wl.page_size
+    scale = float(np.float32(wl.scale))
+    seen = 0
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            kp, _, _, L = unit_arrays(inp, b, h)
+            P = kp.shape[0]
+            K = np.concatenate([kp[p, 0, : min(S, L - p * S)] for p in range(P)])
+            page_of = np.concatenate([np.full(min(S, L - p * S), p) for p in range(P)])
+            kept = np.isin(page_of, sel[b, h, : int(n[b, h])].cpu().numpy())
+            want = O.softmax_dropped_mass(q_group(inp, b, h), K, kept, scale)
+            got = drop[b, h * G:(h + 1) * G]
+            assert np.allclose(got, want, rtol=0, atol=1e-4), (b, h, got, want)
+            seen += int(np.any(want > 1e-3))
+    assert seen > 0, "no unit dropped any mass: the check saw nothing"
 
 
 def test_softmax_empty_selection_gives_zero_and_minus_inf(case):

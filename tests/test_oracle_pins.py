@@ -523,3 +523,125 @@ def test_adaptive_budget_reaches_the_full_cache_output():
         if k > 2:
             prev = O.decode_unit(k_pool, v_pool, pt, L, 0, q, policy="topk", k=k // 2, **kw)
             assert not np.all(O.exactness_certificate(prev["score"], prev["sel"], prev["tau"], 1.5))
+
+
+# ---------------------------------------------------------------- paged cache plumbing
+def _paged_from_flat(rng, lens, S, Hkv, d, spare=2):
+    """A paged pool built from flat per-sequence token arrays through a random
+    page table (a permutation of a shared pool with spare pages per sequence),
+    plus the flat arrays themselves: tokens[b] is [Hkv, n_pages·S, d]."""
+    n_pages = [-(-L // S) + spare for L in lens]
+    num_phys = sum(n_pages)
+    perm = rng.permutation(num_phys)
+    max_pages = max(n_pages)
+    page_table = np.zeros((len(lens), max_pages), np.int64)
+    k_pool = np.zeros((num_phys, Hkv, S, d))
+    v_pool = np.zeros((num_phys, Hkv, S, d))
+    flat_k, flat_v, off = [], [], 0
+    for b, P in enumerate(n_pages):
+        page_table[b, :P] = perm[off:off + P]
+        off += P
+        fk = O.round_bf16(rng.normal(size=(Hkv, P * S, d)))
+        fv = O.round_bf16(rng.normal(size=(Hkv, P * S, d)))
+        flat_k.append(fk)
+        flat_v.append(fv)
+        for p in range(P):
+            k_pool[page_table[b, p]] = fk[:, p * S:(p + 1) * S]
+            v_pool[page_table[b, p]] = fv[:, p * S:(p + 1) * S]
+    return k_pool, v_pool, page_table, flat_k, flat_v
+
+
+def _flat_of(pool, page_table_row, P):
+    """Read a sequence back out of the pool: its pages in logical order."""
+    return np.concatenate([pool[page_table_row[p]] for p in range(P)], axis=1)
+
+
+def test_append_token_writes_position_L_minus_1_of_the_flat_sequence():
+    """[EntmaxKV] §2.A: the cache grows by one token per decode step.  After
+    append_token, reading each sequence back through its page table must give
+    the flat token array with exactly token L−1 replaced (L = the length that
+    already counts the new token), whatever slot of whatever page that is: a
+    mid-page slot, slot 0 of a fresh page and the last slot of a page are all
+    in the batch.  The returned n_valid is the page's token count after it."""
+    rng = np.random.default_rng(71)
+    S, Hkv, d = 8, 3, 5
+    lens = [13, 17, 24, 1, 9]          # slots 4, 0 (fresh page), 7 (last), 0 (first token), 0
+    k_pool, v_pool, pt, flat_k, flat_v = _paged_from_flat(rng, lens, S, Hkv, d)
+    before_k, before_v = k_pool.copy(), v_pool.copy()
+    k_new = O.round_bf16(rng.normal(size=(len(lens), Hkv, d)))
+    v_new = O.round_bf16(rng.normal(size=(len(lens), Hkv, d)))
+    touched = O.append_token(k_pool, v_pool, pt, lens, k_new, v_new, S)
+    assert [t[0] for t in touched] == list(range(len(lens)))
+    changed_pages = set()
+    for b, L in enumerate(lens):
+        P = -(-L // S) + 2
+        want_k = flat_k[b].copy()
+        want_v = flat_v[b].copy()
+        want_k[:, L - 1] = k_new[b]
+        want_v[:, L - 1] = v_new[b]
+        assert np.array_equal(_flat_of(k_pool, pt[b], P), want_k), b
+        assert np.array_equal(_flat_of(v_pool, pt[b], P), want_v), b
+        _, phys, n_valid = touched[b]
+        assert phys == pt[b][(L - 1) // S]
+        assert n_valid == L - S * ((L - 1) // S)       # tokens of that page up to L−1
+        changed_pages.add(phys)
+    # nothing outside the touched pages moved
+    untouched = np.setdiff1d(np.arange(k_pool.shape[0]), sorted(changed_pages))
+    assert np.array_equal(k_pool[untouched], before_k[untouched])
+    assert np.array_equal(v_pool[untouched], before_v[untouched])
+
+
+def test_build_page_meta_matches_flat_slices_on_a_permuted_pool():
+    """[EntmaxKV] §2.A: metadata of every (physical page, KV head) of a
+    scattered pool equals page_metadata of that page's tokens sliced straight
+    out of the flat sequence (logical page p = tokens p·S .. p·S + n_p − 1),
+    including a partial last page; pages no sequence uses get no entry."""
+    rng = np.random.default_rng(73)
+    S, Hkv, d = 8, 2, 6
+    lens = [21, 8, 30]
+    k_pool, _, pt, flat_k, _ = _paged_from_flat(rng, lens, S, Hkv, d, spare=1)
+    meta = O.build_page_meta(k_pool, pt, lens, S, "bf16")
+    used = set()
+    for b, L in enumerate(lens):
+        P = -(-L // S)
+        for p in range(P):
+            n = min(S, L - p * S)
+            phys = int(pt[b, p])
+            used.add(phys)
+            for h in range(Hkv):
+                ref = O.page_metadata(flat_k[b][h, p * S:p * S + S][None], [n], "bf16")
+                for f in ("kmax", "kmin", "mean", "var"):
+                    assert np.array_equal(meta[phys][f][h], ref[f][0]), (b, p, h, f)
+    assert set(meta) == used
+
+
+def test_softmax_lse_consistent_with_weights_and_equal_score_closed_form():
+    """The softmax log-sum-exp: n equal scores give z + ln n exactly in closed
+    form, and every weight (pinned against scipy above) equals e^(z_i − lse)."""
+    rng = np.random.default_rng(79)
+    d = 8
+    q = rng.normal(size=(2, d))
+    K = np.tile(rng.normal(size=(1, d)), (37, 1))
+    r = O.softmax_attention(q, K, np.ones((37, 1)), 0.5)
+    z = 0.5 * (q @ K[0])
+    assert np.allclose(r["lse"], z + math.log(37), rtol=0, atol=1e-13)
+    K2 = rng.normal(size=(50, d)) * 3.0
+    r2 = O.softmax_attention(q, K2, np.ones((50, 1)), 0.5)
+    assert np.allclose(np.exp(0.5 * (q @ K2.T) - r2["lse"][:, None]), r2["p"], rtol=1e-12, atol=1e-300)
+
+
+def test_softmax_dropped_mass_identity_and_limits():
+    """[EntmaxKV] §3 "Borne d'Erreur": the dropped softmax mass δ of a kept set
+    equals 1 − e^(lse_kept − lse_all) (the kept tokens' share of Σ e^z), is 0
+    when everything is kept and 1 − (kept/T) for equal scores."""
+    rng = np.random.default_rng(83)
+    q = rng.normal(size=(3, 10))
+    K = rng.normal(size=(60, 10))
+    kept = rng.random(60) < 0.3
+    delta = O.softmax_dropped_mass(q, K, kept, 0.4)
+    lse_all = O.softmax_attention(q, K, np.zeros((60, 1)), 0.4)["lse"]
+    lse_kept = O.softmax_attention(q, K[kept], np.zeros((int(kept.sum()), 1)), 0.4)["lse"]
+    assert np.allclose(delta, 1.0 - np.exp(lse_kept - lse_all), rtol=1e-12, atol=1e-14)
+    assert np.allclose(O.softmax_dropped_mass(q, K, np.ones(60, bool), 0.4), 0.0)
+    Keq = np.tile(K[:1], (60, 1))
+    assert np.allclose(O.softmax_dropped_mass(q, Keq, kept, 0.4), 1.0 - kept.sum() / 60.0, atol=1e-14)
