@@ -5,11 +5,15 @@
 One step = one decode token for every (sequence, KV head) unit of the
 workload: cache append + tail-page metadata, bounding-box page scores, top-k
 page selection, sparse α-entmax attention (scores over the selected K, τ,
-support-only V).  Inputs are resident in HBM; L2 is flushed (256 MiB read)
-between steps.  Prints one JSON line on rank 0.
+support-only V), as one ekv_decode_step call.  Inputs are resident in HBM;
+L2 is flushed (256 MiB read) between steps.  Prints one JSON line on rank 0.
 
-Workload (default): the clustered 128k-context decode — batch 4, 32 query /
-8 KV heads, d = 128, page size 16, bf16 cache, top-k k = 256, α = 1.5.
+Headline workload: the clustered 128k-context decode — batch 4, 32 query /
+8 KV heads, d = 128, page size 16, bf16 cache, top-k k = 256, α = 1.5.  The
+default run adds the Gaussian policy and the full-cache decodes on the same
+cache, the end-to-end figure through host buffers, every other workload of
+the set (``workloads``) and the float64 oracle timed on the host
+(``cpu_baseline``); ``--quick`` keeps the headline line only.
 """
 from __future__ import annotations
 
@@ -22,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -37,12 +42,12 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture
-# of the bench workload's shape, keyed by a hash of the kernel's sources (a
+# of the clustered 128k shape, keyed by a hash of the kernel's sources (a
 # changed kernel has no measured traffic until it is captured again)
 SCORE_FILES = ("score.cu", "common.cuh", "kernels.cuh")
-DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh", "kernels.cuh")
-SCORE_TRAFFIC = {"d0d585139e2ad614": 137794048}   # profiles/score_kernel_clustered_128k.md
-DECODE_TRAFFIC = {"f4f00457b9e63761": 56003584}   # profiles/fused_decode_kernel_clustered_128k.md
+DECODE_FILES = ("decode_split.cu", "decode.cuh", "common.cuh", "kernels.cuh")
+SCORE_TRAFFIC = {"d0d585139e2ad614": 137794048}
+DECODE_TRAFFIC = {}
 
 
 def kernel_hash(files=SCORE_FILES):
@@ -92,11 +97,10 @@ class ClockSampler:
     def __init__(self, uuid=None):
         self.uuid = uuid
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"ekv_clocks_{os.getpid()}_{id(self)}.csv")
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
@@ -154,38 +158,186 @@ class L2Flush:
 
 
 # ---------------------------------------------------------------- bytes
-def algorithmic_bytes(inp, eng, support_pages, support_tokens):
-    """Bytes one step must move: metadata rows, q, ub, selected K, V of
-    support pages, outputs, and the append (tail page + new rows + metadata).
-    The decode kernel's own bytes count V token by token (the union of the
-    group heads' support), as the method needs them; the kernel reads whole
-    support pages, which the measured traffic shows."""
+def step_bytes(inp, policy, n_sel, support_pages, support_tokens):
+    """Bytes one step must move, and each kernel's share (SURVEY §8(d)'s
+    per-unit figures × the units of the step): the metadata rows the
+    selection reads (box for top-k, mean/var for the Gaussian policy; none
+    for the full cache), q, the page scores, the selected K, the V rows of the
+    support (token by token for the decode kernel, as the method needs them;
+    page by page for the step, the pages that hold support), the output and
+    the append (tail page + new rows + its metadata rows)."""
     wl = inp["workload"]
     es = inp["k_pool"].element_size()
-    d, S, G = wl.head_dim, wl.page_size, wl.group
-    lens = inp["seq_lens"].tolist()
-    pages = [-(-L // S) for L in lens]
-    units_pages = sum(pages) * wl.num_kv_heads
-    meta = units_pages * 2 * d * es
+    d, S = wl.head_dim, wl.page_size
+    pages = sum(-(-int(L) // S) for L in inp["seq_lens"].tolist()) * wl.num_kv_heads
+    meta = 0 if policy == "full" else pages * 2 * d * es
     q = wl.batch * wl.num_q_heads * d * es
-    ub = units_pages * 4
-    n_sel = eng.n_sel.to(torch.int64)
-    sel_tokens = int(n_sel.sum()) * S                     # full pages (tail rounding ignored)
-    selK = sel_tokens * d * es
-    supV = int(support_pages) * S * d * es
+    ub = pages * 4 if policy == "topk" else 0
+    sel_k = int(n_sel) * S * d * es
+    sup_v_pages = int(support_pages) * S * d * es
+    sup_v_tok = int(support_tokens) * d * es
     out = wl.batch * wl.num_q_heads * d * 4
     append = wl.units * (S * d * es + 2 * d * es + 4 * d * es)
-    supV_tok = int(support_tokens) * d * es
-    return {"meta": meta, "q": q, "ub": ub, "sel_k": selK, "support_v": supV, "out": out,
-            "append": append, "score_kernel": meta + q + ub,
-            "decode_kernel": selK + supV_tok + q + out,
-            "step": meta + q + selK + supV + out + append}
+    return {"meta": meta, "q": q, "ub": ub, "sel_k": sel_k, "support_v": sup_v_pages, "out": out,
+            "append": append, "select_kernel": meta + q + ub,
+            "decode_kernel": sel_k + sup_v_tok + q + out,
+            "step": meta + q + sel_k + sup_v_pages + out + append}
+
+
+# ---------------------------------------------------------------- one timed line
+class Line:
+    """One workload × policy × α through the library, timed the way the
+    headline is: whole steps (one ekv_decode_step call each, L2 flushed
+    between steps) and a staged breakdown (the same kernels as separate calls
+    with events between them)."""
+
+    def __init__(self, wl, inp, policy, alpha, dev, flush, *, k=None, delta=None, cap=None, dense_v=False):
+        from sparse_kv_cache_kmax_b200 import binding as Bd
+        from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+        from sparse_kv_cache_kmax_b200.workloads import gauss_cap
+
+        self.Bd, self.wl, self.inp, self.policy, self.alpha = Bd, wl, inp, policy, alpha
+        self.dev, self.flush = dev, flush
+        if policy == "gauss" and cap is None:
+            cap = gauss_cap(wl, inp["max_pages"])
+        self.eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
+                                policy=policy, k=k, delta=delta, alpha=alpha, cap=cap, dense_v=dense_v)
+        self.eng.build_meta()
+        self.k, self.delta, self.cap, self.dense_v = k, delta, self.eng.cap, dense_v
+        self.scale = float(np.float32(wl.scale))
+        self.q, self.k_new, self.v_new = inp["q"], inp["k_new"][0], inp["v_new"][0]
+        e, Hq = self.eng, wl.num_q_heads
+        self.ub = torch.empty(wl.batch, wl.num_kv_heads, inp["max_pages"], device=dev)
+        self.dec_ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, e.cache, e.seqs, Hq, self.cap), dev)
+        n_tk = Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_TOPK, e.cache, e.seqs, Hq, k or 1) if policy == "topk" else 0
+        self.tk_ws = Bd.workspace(n_tk, dev) if n_tk else None
+        self.g_ws = (Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_GAUSS, e.cache, e.seqs, Hq, self.cap), dev)
+                     if policy == "gauss" else None)
+        self.tau_hat = torch.empty(wl.batch, Hq, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    # one whole step: the public one-call API
+    def step(self, ev):
+        ev[0].record(self.stream)
+        self.eng.step(self.q, self.k_new, self.v_new, self.stream)
+        ev[1].record(self.stream)
+
+    # the same kernels as separate calls: append | selection | decode
+    def staged(self, ev):
+        Bd, e, st, wl = self.Bd, self.eng, self.stream, self.wl
+        ev[0].record(st)
+        Bd.ekv_append(e.cache, e.seqs, self.k_new, self.v_new, st)
+        ev[1].record(st)
+        if self.policy == "topk":
+            Bd.ekv_score_pages(e.cache, e.seqs, self.q, self.scale, self.ub, st)
+            ev[2].record(st)
+            Bd.ekv_select_topk(e.seqs, wl.num_kv_heads, wl.page_size, self.ub, self.k, e.sel, e.n_sel, st,
+                               ws=self.tk_ws)
+        elif self.policy == "gauss":
+            ev[2].record(st)
+            Bd.ekv_select_gauss(e.cache, e.seqs, self.q, self.scale, self.alpha, self.delta, self.cap, e.sel, e.n_sel,
+                                self.tau_hat, self.g_ws, st)
+        else:
+            ev[2].record(st)
+        ev[3].record(st)
+        full = self.policy == "full"
+        Bd.ekv_entmax_decode(e.cache, e.seqs, self.q, self.scale, self.alpha, None if full else e.sel,
+                             None if full else e.n_sel, self.cap, e.out, self.dec_ws, dense_v=self.dense_v, stream=st)
+        ev[4].record(st)
+
+    def timed(self, fn, n_events, steps, warmup, world=1):
+        for _ in range(warmup):
+            self.flush.zero_()
+            fn([torch.cuda.Event(enable_timing=True) for _ in range(n_events)])
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            self.flush.zero_()
+            fn(evs[i])
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
+
+    def support(self):
+        """Support of the last step's selection (untimed): pages and tokens
+        whose V a step reads (union over each unit's query heads)."""
+        Bd, e, wl = self.Bd, self.eng, self.wl
+        Hq, S = wl.num_q_heads, wl.page_size
+        full = self.policy == "full"
+        words = (self.cap * S + 31) // 32
+        bits = torch.zeros(wl.batch, Hq, words, dtype=torch.int32, device=self.dev)
+        cnt = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=self.dev)
+        tau = torch.zeros(wl.batch, Hq, device=self.dev)
+        Bd.ekv_entmax_decode(e.cache, e.seqs, self.q, self.scale, self.alpha, None if full else e.sel,
+                             None if full else e.n_sel, self.cap, e.out, self.dec_ws, tau=tau, support_count=cnt,
+                             support_bits=bits)
+        tok = (bits.unsqueeze(-1) >> torch.arange(32, device=self.dev, dtype=torch.int32)) & 1
+        tok = tok.view(wl.batch, wl.num_kv_heads, wl.group, -1).amax(dim=2)
+        page_sup = tok[..., : self.cap * S].reshape(wl.batch, wl.num_kv_heads, self.cap, S).amax(dim=-1)
+        if full:
+            n_sel = sum(-(-int(L) // S) for L in self.inp["seq_lens"].tolist()) * wl.num_kv_heads
+        else:
+            n_sel = int(e.n_sel.sum())
+        return {"n_sel": n_sel, "support_pages": int(page_sup.sum()), "support_tokens": int(tok.sum()),
+                "mean_support_tokens_per_head": float(cnt.float().mean()), "tau": tau}
+
+    def measure(self, steps, warmup, peak, world=1, uuid=None):
+        with ClockSampler(uuid) as clk:
+            per_step = self.timed(self.step, 2, steps, warmup, world)[:, 0]
+        clocks = clk.summary()
+        staged = self.timed(self.staged, 5, max(3, min(steps, 200)), warmup).mean(axis=0)
+        sup = self.support()
+        nb = step_bytes(self.inp, self.policy, sup["n_sel"], sup["support_pages"], sup["support_tokens"])
+        step_ms = float(per_step.mean())
+        sel_name = {"topk": "score", "gauss": "gauss_select", "full": None}[self.policy]
+        kern = {"append": {"us": float(staged[0]) * 1e3, "bound": "latency (one page per unit)"}}
+        if self.policy == "topk":
+            kern["score"] = {"us": float(staged[1]) * 1e3}
+            kern["topk"] = {"us": float(staged[2]) * 1e3, "bound": "latency (scores from L2)"}
+        elif self.policy == "gauss":
+            kern["gauss_select"] = {"us": float(staged[2]) * 1e3,
+                                    "note": "page statistics + tau-hat + filter (three kernels)"}
+        kern["decode"] = {"us": float(staged[3]) * 1e3}
+        for name, key in ((sel_name, "select_kernel"), ("decode", "decode_kernel")):
+            if name is None:
+                continue
+            us = kern[name]["us"]
+            ach = nb[key] / (us * 1e-6) / 1e9
+            kern[name].update({"algorithmic_bytes": nb[key], "achieved": ach, "frac": ach / peak})
+        dom = max((n for n in (sel_name, "decode") if n), key=lambda n: kern[n]["us"])
+        return {
+            "ms_per_step": step_ms, "value": self.wl.units / (step_ms * 1e-3), "unit": UNIT, "steps": int(steps),
+            "total_s": float(per_step.sum()) / 1e3,
+            "stages_us": {"append": staged[0] * 1e3, "select": (staged[1] + staged[2]) * 1e3,
+                          "decode": staged[3] * 1e3, "sum": float(staged.sum()) * 1e3},
+            "kernels": kern, "dominant": dom,
+            "step_roofline": {"bytes": nb["step"], "achieved_gbs": nb["step"] / (step_ms * 1e-3) / 1e9,
+                              "frac": nb["step"] / (step_ms * 1e-3) / 1e9 / peak,
+                              "breakdown": {kk: v for kk, v in nb.items() if kk not in ("step",)}},
+            "support": {"mean_sel_pages": sup["n_sel"] / self.wl.units,
+                        "support_pages_per_unit": sup["support_pages"] / self.wl.units,
+                        "mean_support_tokens_per_head": sup["mean_support_tokens_per_head"]},
+            "clocks": clocks, "tau": sup["tau"],
+        }
+
+
+def short_line(m):
+    """The fields of a secondary line in the JSON (no tensors)."""
+    dom = m["dominant"]
+    return {"ms_per_step": m["ms_per_step"], "value": m["value"], "unit": m["unit"], "steps": m["steps"],
+            "step_frac": m["step_roofline"]["frac"], "dominant_kernel": dom,
+            "dominant_frac": m["kernels"][dom].get("frac"),
+            "kernels_us": {n: v["us"] for n, v in m["kernels"].items()},
+            "mean_sel_pages": m["support"]["mean_sel_pages"], "clocks": m["clocks"]}
 
 
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
     from sparse_kv_cache_kmax_b200 import binding as Bd
-    from sparse_kv_cache_kmax_b200.engine import DecodeEngine
     from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs
 
     world, rank, local = dist_env()
@@ -199,51 +351,17 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     Bd.lib()                                   # fail loudly if the library is missing
 
+    # the oracle's host threads start before any GPU work
+    cpu_pool = None
+    if rank == 0 and world == 1 and not args.quick:
+        from concurrent.futures import ThreadPoolExecutor
+        cpu_pool = ThreadPoolExecutor(max_workers=cpu_threads())
+
     wl = WORKLOADS[args.workload]
     inp = make_inputs(wl, seed=3000 + rank, device=dev, n_new=1)
-    q, k_new, v_new = inp["q"], inp["k_new"][0], inp["v_new"][0]
     alpha, k = args.alpha, args.k or wl.topk
-    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
-                       policy="topk", k=k, alpha=alpha)
-    eng.build_meta()
-    cache, seqs, Hq = eng.cache, eng.seqs, wl.num_q_heads
-    scale = float(np.float32(wl.scale))
-    ub = torch.empty(wl.batch, wl.num_kv_heads, inp["max_pages"], device=dev)
-    dec_ws = Bd.workspace(Bd.ekv_workspace_bytes(Bd.EKV_OP_ENTMAX_DECODE, cache, seqs, Hq, k), dev)
-    n_tk = Bd.ekv_workspace_bytes(Bd.EKV_OP_SELECT_TOPK, cache, seqs, Hq, k)
-    tk_ws = Bd.workspace(n_tk, dev) if n_tk else None
     flush = L2Flush(dev)
-    stream = torch.cuda.current_stream()
-
-    def stage_step(ev):
-        ev[0].record(stream)
-        Bd.ekv_append(cache, seqs, k_new, v_new, stream)
-        ev[1].record(stream)
-        Bd.ekv_score_pages(cache, seqs, q, scale, ub, stream)
-        ev[2].record(stream)
-        Bd.ekv_select_topk(seqs, wl.num_kv_heads, wl.page_size, ub, k, eng.sel, eng.n_sel, stream, ws=tk_ws)
-        ev[3].record(stream)
-        Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws, stream=stream)
-        ev[4].record(stream)
-
-    def timed(step_fn, n_events, steps, warmup):
-        for _ in range(warmup):
-            flush.zero_()
-            step_fn([torch.cuda.Event(enable_timing=True) for _ in range(n_events)])
-        torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        for i in range(steps):
-            flush.zero_()
-            step_fn(evs[i])
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
-        return per                              # ms, [steps, stages]
-
+    peak, peak_kind = hbm_peak()
     uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -251,126 +369,115 @@ def run_ours(args):
     except Exception:
         uuid = None
 
-    # headline: the whole step as one C-ABI call (its kernels chain with
-    # programmatic dependent launch), CUDA events at step boundaries only
-    def fused_step(ev):
-        ev[0].record(stream)
-        eng.step(q, k_new, v_new, stream)
-        ev[1].record(stream)
-
-    with ClockSampler(uuid) as clk:
-        per_step = timed(fused_step, 2, args.steps, args.warmup)[:, 0]
-    step_ms = float(per_step.mean())
-    total_s = float(per_step.sum()) / 1e3
-    max_s, units_all = reduce_timing(total_s, wl.units * args.steps)
+    line = Line(wl, inp, "topk", alpha, dev, flush, k=k)
+    m = line.measure(args.steps, args.warmup, peak, world, uuid)
+    max_s, units_all = reduce_timing(m["total_s"], wl.units * args.steps)
     value = units_all / max_s
-    clocks = clk.summary()
-    # breakdown: the same stages as separate calls with events between them
-    per = timed(stage_step, 5, max(3, min(args.steps, 300)), args.warmup)
-    stages = per.mean(axis=0)
-
-    # support statistics of the last step (untimed): pages whose V the step read
-    words = (k * wl.page_size + 31) // 32
-    bits = torch.zeros(wl.batch, Hq, words, dtype=torch.int32, device=dev)
-    cnt = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=dev)
-    tau_last = torch.zeros(wl.batch, Hq, device=dev)
-    Bd.ekv_entmax_decode(cache, seqs, q, scale, alpha, eng.sel, eng.n_sel, k, eng.out, dec_ws,
-                         tau=tau_last, support_count=cnt, support_bits=bits)
-    cert = torch.zeros(wl.batch, Hq, dtype=torch.int32, device=dev)
-    Bd.ekv_exactness_certificate(seqs, wl.num_kv_heads, wl.page_size, alpha, ub, eng.sel, eng.n_sel, tau_last, cert)
-    tok = ((bits.view(torch.int32).unsqueeze(-1) >> torch.arange(32, device=dev, dtype=torch.int32)) & 1)
-    tok = tok.view(wl.batch, wl.num_kv_heads, wl.group, -1).amax(dim=2)          # union over the group
-    page_sup = tok.view(wl.batch, wl.num_kv_heads, k, wl.page_size).amax(dim=-1)
-    support_pages = int(page_sup.sum())
-    support_tokens = int(tok.sum())
-    nb = algorithmic_bytes(inp, eng, support_pages, support_tokens)
-
-    # per-kernel rooflines from the staged timing; the headline one is the
-    # kernel with the largest time (the launch list's largest share)
-    peak, peak_kind = hbm_peak()
-    kern = {}
-    for name, idx, key, table, files in (("score", 1, "score_kernel", SCORE_TRAFFIC, SCORE_FILES),
-                                         ("decode", 3, "decode_kernel", DECODE_TRAFFIC, DECODE_FILES)):
-        ms = float(stages[idx])
-        ach = nb[key] / (ms * 1e-3) / 1e9
-        kern[name] = {"us": ms * 1e3, "algorithmic_bytes": nb[key], "achieved": ach, "frac": ach / peak,
-                      "traffic": table.get(kernel_hash(files))}
-    kern["topk"] = {"us": float(stages[2]) * 1e3, "bound": "latency (1 MiB of scores)"}
-    kern["append"] = {"us": float(stages[0]) * 1e3, "bound": "latency (one page per unit)"}
-    dom = max(("score", "decode"), key=lambda n: kern[n]["us"])
+    eng = line.eng
+    kern = m["kernels"]
+    dom = m["dominant"]
+    files = {"score": SCORE_FILES, "decode": DECODE_FILES}
+    tables = {"score": SCORE_TRAFFIC, "decode": DECODE_TRAFFIC}
+    for name in ("score", "decode"):
+        kern[name]["traffic"] = tables[name].get(kernel_hash(files[name]))
     dom_name = {"score": "score (bounding-box page scores)",
-                "decode": "decode (fused: scores on selected K, tau, support V)"}[dom]
+                "decode": "decode (scores on the selected K, tau, support V: one launch)"}[dom]
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": f"{wl.name}: batch {wl.batch}, {wl.num_q_heads} q / {wl.num_kv_heads} KV heads, "
                                f"d {wl.head_dim}, context {wl.context}, page size {wl.page_size}",
                    "policy": "topk", "k": k, "alpha": alpha, "global_batch": wl.batch * world,
                    "seq_len": wl.context, "parallelism": f"replicas x{world} (units sharded, no collective)",
                    "l2": "flushed between steps (256 MiB read)"},
-        "steps_per_s": 1e3 / step_ms,
-        "stages_us": {"append": stages[0] * 1e3, "score": stages[1] * 1e3, "topk": stages[2] * 1e3,
-                      "decode": stages[3] * 1e3, "sum": float(stages.sum()) * 1e3,
-                      "note": "separate calls with events between stages (no launch overlap)"},
+        "steps_per_s": 1e3 / m["ms_per_step"],
+        "stages_us": dict(m["stages_us"], note="separate calls with events between stages (no launch overlap)"),
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": kern[dom]["achieved"],
                      "peak": peak, "unit": "GB/s", "frac": kern[dom]["frac"],
                      "peak_kind": f"{peak_kind} copy bandwidth", "traffic": kern[dom]["traffic"],
                      "algorithmic_bytes": kern[dom]["algorithmic_bytes"]},
         "kernels": kern,
-        "step_roofline": {"bytes": nb["step"], "achieved_gbs": nb["step"] / (step_ms * 1e-3) / 1e9,
-                          "frac": nb["step"] / (step_ms * 1e-3) / 1e9 / peak,
-                          "breakdown": {kk: v for kk, v in nb.items() if kk not in ("step", "score_kernel")}},
-        "certificate": certificate_stats(cert, inp, wl, alpha, k),
-        "support": {"mean_sel_pages": float(eng.n_sel.float().mean()), "support_pages_per_unit":
-                    support_pages / wl.units, "mean_support_tokens_per_head": float(cnt.float().mean())},
-        "gpu_launches": Bd.ekv_step_kernel_count(cache, seqs, eng.params, Hq) * args.steps,
-        "clocks": clocks,
+        "step_roofline": m["step_roofline"],
+        "support": m["support"],
+        "gpu_launches": Bd.ekv_step_kernel_count(eng.cache, eng.seqs, eng.params, wl.num_q_heads) * args.steps,
+        "clocks": m["clocks"],
     }
-
-    result["softmax_full_cache"] = bench_softmax(args, wl, inp, eng, dev, flush, peak, step_ms)
+    cert = torch.zeros(wl.batch, wl.num_q_heads, dtype=torch.int32, device=dev)
+    Bd.ekv_score_pages(eng.cache, eng.seqs, inp["q"], line.scale, line.ub)
+    Bd.ekv_exactness_certificate(eng.seqs, wl.num_kv_heads, wl.page_size, alpha, line.ub, eng.sel, eng.n_sel,
+                                 m["tau"], cert)
+    result["certificate"] = certificate_stats(cert, inp, wl, alpha, k)
+    result["softmax_full_cache"] = bench_softmax(args, wl, inp, eng, dev, flush, peak, m["ms_per_step"])
+    dm = result["softmax_full_cache"].get("dropped_mass", {})
+    result["headline_exactness"] = {
+        "certified_heads_frac": result["certificate"]["certified_heads_frac_at_k"],
+        "entmax_rel_err_vs_full_cache_median": dm.get("entmax_rel_err_median"),
+        "entmax_rel_err_vs_full_cache_max": dm.get("entmax_rel_err_max"),
+        "note": "top-k k keeps a fixed budget: heads whose support reaches past the kept pages differ from "
+                "the full-cache output; the adaptive budget and the Gaussian policy are the exact-output points"}
     if not args.quick:
-        result["gauss"] = bench_policy(args, wl, inp, "gauss", dev, flush)
-        result["full_cache"] = bench_policy(args, wl, inp, "full", dev, flush)
-        result["full_cache_dense_v"] = bench_policy(args, wl, inp, "full", dev, flush, dense_v=True)
+        g = Line(wl, inp, "gauss", alpha, dev, flush, delta=wl.delta if wl.delta is not None else 0.5)
+        gm = g.measure(max(3, min(args.steps, 200)), args.warmup, peak)
+        result["gauss"] = dict(short_line(gm), delta=g.delta, cap=g.cap, stages_us=gm["stages_us"],
+                               support=gm["support"])
+        del g
+        for key, dense in (("full_cache", False), ("full_cache_dense_v", True)):
+            f = Line(wl, inp, "full", alpha, dev, flush, dense_v=dense)
+            fm = f.measure(max(3, min(args.steps, 100)), args.warmup, peak)
+            kb = sum(int(L) for L in inp["seq_lens"].tolist()) * wl.num_kv_heads * wl.head_dim * \
+                inp["k_pool"].element_size()
+            nbytes = kb * (2 if dense else 1) + (0 if dense else fm["step_roofline"]["breakdown"]["support_v"])
+            result[key] = dict(short_line(fm), dense_v=dense, k_bytes=kb, algorithmic_bytes=nbytes,
+                               achieved_gbs=nbytes / (fm["kernels"]["decode"]["us"] * 1e-6) / 1e9,
+                               frac=nbytes / (fm["kernels"]["decode"]["us"] * 1e-6) / 1e9 / peak)
+            del f
         result["e2e"] = bench_e2e(args, wl, inp, eng, dev, flush, world)
-    if rank == 0 and world == 1 and not args.quick:
-        result["cpu_baseline"] = cpu_baseline(wl, inp, k, alpha, budget_s=args.cpu_seconds)
+        if world == 1:
+            result["workloads"] = other_workloads(args, wl, dev, flush, peak, uuid)
+    if cpu_pool is not None:
+        result["cpu_baseline"] = cpu_baseline(wl, inp, k, alpha, cpu_pool, budget_s=args.cpu_seconds)
+        cpu_pool.shutdown()
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(result))
 
 
-def bench_policy(args, wl, inp, policy, dev, flush, dense_v=False):
-    """Whole-step timing (one ekv_decode_step call) of another policy."""
-    from sparse_kv_cache_kmax_b200.engine import DecodeEngine
+# (workload, policy, alpha, budget) of the other lines in the default run
+OTHER_LINES = [
+    ("clustered_128k", "topk", 1.25, None),
+    ("clustered_128k", "topk", 2.0, None),
+    ("gqa_32k", "topk", 1.5, None),
+    ("short_scattered", "topk", 1.5, None),
+    ("long_512k", "topk", 1.5, None),
+    ("long_512k", "gauss", 1.5, None),
+    ("ctx_1m", "topk", 1.5, None),
+    ("ctx_1m", "gauss", 1.5, None),
+]
 
-    eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
-                       policy=policy, k=wl.topk, delta=wl.delta if wl.delta is not None else 0.5,
-                       alpha=args.alpha, dense_v=dense_v)
-    eng.build_meta()
-    steps = max(3, min(args.steps, 200 if policy == "full" else args.steps))
-    for _ in range(args.warmup):
-        flush.zero_()
-        eng.step(inp["q"], inp["k_new"][0], inp["v_new"][0])
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for i in range(steps):
-        flush.zero_()
-        ev[i][0].record()
-        eng.step(inp["q"], inp["k_new"][0], inp["v_new"][0])
-        ev[i][1].record()
-    torch.cuda.synchronize()
-    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    res = {"ms_per_step": ms, "value": wl.units / (ms * 1e-3), "unit": UNIT, "steps": steps,
-           "mean_sel_pages": float(eng.n_sel.float().mean()) if policy != "full" else float(inp["max_pages"])}
-    if policy == "full":
-        es = inp["k_pool"].element_size()
-        kv = sum(int(L) for L in inp["seq_lens"].tolist()) * wl.num_kv_heads * wl.head_dim * es
-        res["k_bytes"] = kv
-        res["dense_v"] = bool(dense_v)
-    return res
+
+def other_workloads(args, head_wl, dev, flush, peak, uuid):
+    """Every other configuration of the workload set, one line each, measured
+    the way the headline is (whole steps, L2 flushed, staged breakdown)."""
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs
+
+    out, cur, inp = {}, None, None
+    for name, policy, alpha, _ in OTHER_LINES:
+        wl = WORKLOADS[name]
+        if name != cur:
+            inp = None
+            torch.cuda.empty_cache()
+            inp = make_inputs(wl, seed=3000, device=dev, n_new=1)
+            cur = name
+        kw = {"k": wl.topk} if policy == "topk" else {"delta": wl.delta}
+        ln = Line(wl, inp, policy, alpha, dev, flush, **kw)
+        mm = ln.measure(max(3, min(args.steps, 200)), args.warmup, peak, 1, uuid)
+        key = f"{name}/{policy}" + (f" k={wl.topk}" if policy == "topk" else f" delta={wl.delta}") + f"/alpha={alpha}"
+        out[key] = short_line(mm)
+        del ln
+    torch.cuda.empty_cache()
+    return out
 
 
 def certificate_stats(cert, inp, wl, alpha, k):
@@ -450,7 +557,8 @@ def dropped_mass(wl, inp, eng, dev, out_full_sm, ws_sm, scale):
     e_sm, e_ent = rel(out_sel, out_full_sm), rel(ent_sel, ent_full)
     return {"k": int(k), "softmax_dropped_mass_mean": float(drop.mean()), "softmax_dropped_mass_max": float(drop.max()),
             "softmax_rel_err_median": float(e_sm.median()), "softmax_rel_err_max": float(e_sm.max()),
-            "entmax_rel_err_median": float(e_ent.median()), "entmax_rel_err_max": float(e_ent.max())}
+            "entmax_rel_err_median": float(e_ent.median()), "entmax_rel_err_max": float(e_ent.max()),
+            "entmax_heads_exact_frac": float((e_ent <= 1e-5).float().mean())}
 
 
 def bench_e2e(args, wl, inp, eng, dev, flush, world):
@@ -490,21 +598,30 @@ def bench_e2e(args, wl, inp, eng, dev, flush, world):
 
 
 # ---------------------------------------------------------------- the oracle, timed
-def oracle_step_units(wl, host_units, k, alpha, budget_s):
+def cpu_threads():
+    """Host threads of the oracle's timed leg: one per core, at most 32 (each
+    holds its own copy of a unit's metadata)."""
+    return max(1, min(os.cpu_count() or 1, 32))
+
+
+def oracle_step_units(wl, host_units, k, alpha, budget_s, meta=None):
     """Run the oracle's decode step on host copies of some units until
-    budget_s of CPU time is spent; returns (unit-steps done, seconds)."""
+    budget_s of time is spent (at least one unit-step); returns (unit-steps
+    done, seconds).  meta: per-unit metadata dicts this caller owns (the
+    append refreshes their tail page)."""
     import oracle as O
 
     scale = float(np.float32(wl.scale))
     done, t0 = 0, time.perf_counter()
     while True:
-        for (kp, vp, n_valid, qg, meta) in host_units:
+        for i, (kp, vp, n_valid, qg, meta0) in enumerate(host_units):
+            md = meta0 if meta is None else meta[i]
             # append: refresh the tail page's metadata
             last = len(n_valid) - 1
             tail = O.page_metadata(kp[last:last + 1], n_valid[last:last + 1], wl.dtype)
-            for f in meta:
-                meta[f][last] = tail[f][0]
-            ub = O.bbox_upper_bound(qg, meta["kmax"], meta["kmin"], scale)
+            for f in md:
+                md[f][last] = tail[f][0]
+            ub = O.bbox_upper_bound(qg, md["kmax"], md["kmin"], scale)
             sel = O.select_topk(O.page_scores(ub), k)
             Ks = np.concatenate([kp[p, : n_valid[p]] for p in sel])
             Vs = np.concatenate([vp[p, : n_valid[p]] for p in sel])
@@ -532,19 +649,43 @@ def host_units_sample(wl, inp, n_units):
     return units
 
 
-def cpu_baseline(wl, inp, k, alpha, budget_s=15.0):
+def oracle_threaded(wl, units, k, alpha, pool, n_threads, budget_s):
+    """The oracle on n_threads host threads at once, each cycling over the
+    sampled units with its own metadata copies, for budget_s; returns
+    (unit-steps, wall seconds)."""
+    metas = [[{f: a.copy() for f, a in u[4].items()} for u in units] for _ in range(n_threads)]
+    t0 = time.perf_counter()
+    futs = [pool.submit(oracle_step_units, wl, units[i % len(units):] + units[:i % len(units)], k, alpha, budget_s,
+                        metas[i][i % len(units):] + metas[i][:i % len(units)]) for i in range(n_threads)]
+    done = sum(f.result()[0] for f in futs)
+    return done, time.perf_counter() - t0
+
+
+def cpu_baseline(wl, inp, k, alpha, pool, budget_s=15.0):
+    """The oracle as it stands, timed on this host: every thread of the pool
+    at once, and one thread alone (BLAS limited to one thread per worker)."""
     from threadpoolctl import threadpool_limits
 
-    units = host_units_sample(wl, inp, 2)
+    n_threads = pool._max_workers
+    units = host_units_sample(wl, inp, min(8, wl.units))
     with threadpool_limits(1):
-        done, secs = oracle_step_units(wl, units, k, alpha, budget_s)
-    return {"value": done / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"float64 numpy oracle, 1 thread: {done} unit-steps (append + scores + top-k + "
-                      f"entmax attention) cycling over units 0-1 of {wl.name}, {secs:.1f} s"}
+        done_n, secs_n = oracle_threaded(wl, units, k, alpha, pool, n_threads, budget_s)
+        done_1, secs_1 = oracle_step_units(wl, units[:1], k, alpha, budget_s / 2)
+    return {"value": done_n / secs_n, "unit": UNIT, "cores": n_threads, "kind": "oracle",
+            "host_cores": os.cpu_count(),
+            "sample": f"float64 numpy oracle on {n_threads} host threads at once (one BLAS thread each): "
+                      f"{done_n} unit-steps (append + scores + top-k + entmax attention) cycling over units "
+                      f"0-{len(units) - 1} of {wl.name}, {secs_n:.1f} s wall",
+            "single_thread": {"value": done_1 / secs_1, "cores": 1,
+                              "sample": f"{done_1} unit-steps of unit 0 in {secs_1:.1f} s"}}
 
 
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+
     from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs, scaled_down
 
     world, rank, local = dist_env()
@@ -552,37 +693,45 @@ def run_reference(args):
         return
     wl = WORKLOADS[args.workload]
     k = args.k or wl.topk
+    n_threads = cpu_threads()
+    pool = ThreadPoolExecutor(max_workers=n_threads)
     # inputs are drawn on the host here (the reference arm needs no GPU); the
-    # sampled units all live in sequence 0, so one sequence of the shape is drawn
-    inp = make_inputs(scaled_down(args.workload, batch=1), seed=3000, device="cpu")
-    units = host_units_sample(wl, inp, 2)
-    from threadpoolctl import threadpool_limits
-
-    # each step is a bounded sample of the workload: one unit-step of the
-    # oracle (append, scores, top-k, entmax attention), cycling over the units
+    # sampled units live in the first sequences, so only those are drawn
+    n_units = min(8, wl.units)
+    nb = -(-n_units // wl.num_kv_heads)
+    inp = make_inputs(scaled_down(args.workload, batch=nb), seed=3000, device="cpu")
+    units = host_units_sample(wl, inp, n_units)
     import oracle as O  # noqa: F401  (the reference arm runs the oracle)
 
+    # each step is a bounded sample of the workload: one unit-step of the
+    # oracle (append, scores, top-k, entmax attention) on every host thread
     done, secs = 0, 0.0
+    metas = [[{f: a.copy() for f, a in u[4].items()} for u in units] for _ in range(n_threads)]
     with threadpool_limits(1):
         for i in range(args.warmup + args.steps):
-            unit = [units[i % len(units)]]
-            d, s_ = oracle_step_units(wl, unit, k, args.alpha, 0.0)
+            t0 = time.perf_counter()
+            futs = [pool.submit(oracle_step_units, wl, [units[(i + j) % n_units]], k, args.alpha, 0.0,
+                                [metas[j][(i + j) % n_units]]) for j in range(n_threads)]
+            d = sum(f.result()[0] for f in futs)
             if i >= args.warmup:
                 done += d
-                secs += s_
+                secs += time.perf_counter() - t0
+    pool.shutdown()
     value = done / secs
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, done) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{wl.name}: batch {wl.batch}, {wl.num_q_heads} q / {wl.num_kv_heads} KV heads, "
                                f"d {wl.head_dim}, context {wl.context}, page size {wl.page_size}",
                    "policy": "topk", "k": k, "alpha": args.alpha, "global_batch": wl.batch,
-                   "seq_len": wl.context, "parallelism": "none (host oracle)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"float64 numpy oracle, 1 thread, one unit-step per step cycling "
-                                   f"over units 0-1 of {wl.name}: {done} unit-steps in {secs:.1f} s"},
+                   "seq_len": wl.context, "parallelism": f"none (host oracle, {n_threads} threads)",
+                   "l2": "not applicable (host)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_threads, "kind": "oracle",
+                         "sample": f"float64 numpy oracle, {n_threads} host threads, one unit-step per thread per "
+                                   f"step over units 0-{n_units - 1} of {wl.name}: {done} unit-steps in "
+                                   f"{secs:.1f} s"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out))

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libekv.so")
 BUILD = os.path.join(ROOT, "_build", "ekv")
-SOURCES = ["meta.cu", "score.cu", "topk.cu", "gauss.cu", "decode.cu", "decode_fused.cu", "softmax.cu", "certify.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["meta.cu", "score.cu", "topk.cu", "gauss.cu", "decode.cu", "decode_fused.cu", "decode_split.cu", "softmax.cu", "certify.cu", "api.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-Xcompiler", "-fPIC",
                 "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

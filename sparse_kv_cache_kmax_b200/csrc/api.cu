@@ -92,7 +92,7 @@ size_t decode_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
   const size_t S = static_cast<size_t>(c->page_size), D = static_cast<size_t>(c->head_dim);
   return a256(U * G * cap * S * sizeof(float)) + a256(U * G * cap * sizeof(float)) +
          a256(U * G * nqk * sizeof(float)) + a256(U * G * sizeof(float)) +
-         a256(U * npv * G * D * sizeof(float)) + a256(U * sizeof(int));
+         a256(U * npv * G * D * sizeof(float)) + a256(U * sizeof(int)) + a256(U * cap * sizeof(int));
 }
 
 DecodeWs carve_decode(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
@@ -108,6 +108,7 @@ DecodeWs carve_decode(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq,
   w.taus = cv.take<float>(U * G);
   w.part = cv.take<float>(U * static_cast<size_t>(npv) * G * D);
   w.counter = cv.take<int>(U);
+  w.sphys = cv.take<int>(U * static_cast<size_t>(cap));
   w.nqk = nqk;
   w.npv = npv;
   return w;
@@ -346,7 +347,7 @@ EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* se
     n += 1 + (topk_ws_bytes(seqs->batch * cache->num_kv_heads, seqs->max_pages, p->k) > 0 ? 2 : 1);
   else if (p->policy == EKV_POLICY_GAUSS) n += 3;
   else if (!full) return 0;
-  return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap);
+  return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap, p->dense_v);
 }
 
 EKV_API ekv_status ekv_selftest_wait_timeout(uint32_t polls, void* stream) {

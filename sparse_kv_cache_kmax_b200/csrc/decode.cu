@@ -631,11 +631,16 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
 
 }  // namespace
 
-int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap) {
+int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap, int dense_v) {
   const int G = Hq / c.num_kv_heads, U = s.batch * c.num_kv_heads;
   if (c.dtype != EKV_BF16 || U > 65535) return 3;
-#define EKV_CNT_CASE(DD, GG) \
-  if (c.head_dim == DD && G == GG) return fused_decode_fits<DD, GG>(U, cap, c.page_size) ? 1 : 3;
+#define EKV_CNT_CASE(DD, GG)                                                                 \
+  if (c.head_dim == DD && G == GG)                                                           \
+    switch (choose_decode_path<DD, GG>(U, cap, c.page_size, dense_v)) {                           \
+      case DecodePath::kFused: return 1;                                                            \
+      case DecodePath::kSplit: return 2;                                                            \
+      default: return 3;                                                                            \
+    }
   EKV_CNT_CASE(128, 1) EKV_CNT_CASE(128, 2) EKV_CNT_CASE(128, 4) EKV_CNT_CASE(128, 8) EKV_CNT_CASE(128, 16)
   EKV_CNT_CASE(64, 1) EKV_CNT_CASE(64, 2) EKV_CNT_CASE(64, 4) EKV_CNT_CASE(64, 8) EKV_CNT_CASE(64, 16)
 #undef EKV_CNT_CASE
@@ -681,9 +686,11 @@ cudaError_t launch_decode(const ekv_cache& c, const ekv_seqs& s, const void* q, 
   if (c.head_dim == DD && G == GG) return run_decode<TT, DD, GG>(a, U, st);
 #define EKV_DEC_BF16(DD, GG)                                                         \
   if (c.head_dim == DD && G == GG) {                                                 \
-    if (U <= 65535 && fused_decode_fits<DD, GG>(U, cap, c.page_size))                \
-      return run_fused_decode<DD, GG>(a, U, st);                                     \
-    return run_decode<bf16, DD, GG>(a, U, st);                                       \
+    switch (choose_decode_path<DD, GG>(U, cap, c.page_size, dense_v)) {              \
+      case DecodePath::kFused: return run_fused_decode<DD, GG>(a, U, st);            \
+      case DecodePath::kSplit: return run_split_decode<DD, GG>(a, U, st);            \
+      default: return run_decode<bf16, DD, GG>(a, U, st);                            \
+    }                                                                                \
   }
   if (c.dtype == EKV_BF16) {
     EKV_DEC_BF16(128, 1) EKV_DEC_BF16(128, 2) EKV_DEC_BF16(128, 4)

@@ -117,10 +117,36 @@ __device__ __forceinline__ void score_mtile(const uint4 (&va)[D / 32], const uin
   }
 }
 
+// Launch of the two-launch split decode (decode_split.cu): false when the
+// configuration does not fit it.
+template <int D, int G>
+bool split_decode_fits(int cap, int S);
+template <int D, int G>
+cudaError_t run_split_decode(DecodeArgs& a, int units, cudaStream_t st);
+
 // Launch of the fused path: false when the configuration does not fit it
 // (the caller then runs the three-kernel path).
 template <int D, int G>
 bool fused_decode_fits(int units, int cap, int S);
+// CTAs per unit of the fused path's cluster (0: it does not fit).
+template <int D, int G>
+int fused_decode_cluster(int units, int cap, int S);
+
+// The decode path of a bf16 selection: the one-cluster-per-unit kernel when
+// at least kFusedMinCluster CTAs can work on each unit at once (few units),
+// else the two-launch split decode when the selection fits it (many units),
+// else whichever fits, else the three-kernel path.
+constexpr int kFusedMinCluster = 4;
+enum class DecodePath { kFused, kSplit, kThree };
+template <int D, int G>
+DecodePath choose_decode_path(int units, int cap, int S, int dense_v) {
+  if (units > 65535) return DecodePath::kThree;
+  const int C = fused_decode_cluster<D, G>(units, cap, S);
+  const bool split = !dense_v && split_decode_fits<D, G>(cap, S);
+  if (C >= kFusedMinCluster) return DecodePath::kFused;
+  if (split) return DecodePath::kSplit;
+  return C > 0 ? DecodePath::kFused : DecodePath::kThree;
+}
 template <int D, int G>
 cudaError_t run_fused_decode(DecodeArgs& a, int units, cudaStream_t st);
 

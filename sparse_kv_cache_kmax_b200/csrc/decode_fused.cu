@@ -884,6 +884,13 @@ bool fused_decode_fits(int units, int cap, int S) {
 }
 
 template <int D, int G>
+int fused_decode_cluster(int units, int cap, int S) {
+  if (S % 16 != 0 || cap < 1) return 0;
+  const FusedGeom f = choose<D, G>(units, cap, S);
+  return f.smem > 0 ? f.C : 0;
+}
+
+template <int D, int G>
 cudaError_t run_fused_decode(DecodeArgs& a, int units, cudaStream_t st) {
   const FusedGeom f = choose<D, G>(units, a.cap, a.S);
   if (f.smem == 0) return cudaErrorInvalidConfiguration;
@@ -908,6 +915,7 @@ cudaError_t run_fused_decode(DecodeArgs& a, int units, cudaStream_t st) {
 
 #define EKV_FUSED_INST(DD, GG)                                            \
   template bool fused_decode_fits<DD, GG>(int, int, int);                 \
+  template int fused_decode_cluster<DD, GG>(int, int, int);               \
   template cudaError_t run_fused_decode<DD, GG>(DecodeArgs&, int, cudaStream_t);
 EKV_FUSED_INST(128, 1)
 EKV_FUSED_INST(128, 2)

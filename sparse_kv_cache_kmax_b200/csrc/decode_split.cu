@@ -1,0 +1,612 @@
+// Sparse α-entmax decode over the selected pages in two launches — EntmaxKV
+// summary page (gist.science/fr/paper/2605.21649) §2.C "Attention Entmax
+// Parcimonieuse", with the support-only V read that §2–§3 make exact.
+//
+//  1. k_score_kernel, grid (chunks, units): every CTA scores one chunk of 256
+//     selected tokens (8 warps × 32 rows, straight from global memory into
+//     tensor-core A fragments) for the G query heads of its unit, and writes
+//     the scores z, the chunk's per-head maxima and the physical page of each
+//     selected slot to an L2-resident scratch.
+//  2. head_decode_kernel, one CTA of 256 threads per query head: the head's
+//     scores u = (α−1)·z sit in registers (VPT per thread; above 16384
+//     selected tokens they are read again from L2 at each pass); a 256-bin
+//     histogram of u over (max u − 1, max u] brackets τ from the left (c
+//     values above an edge e force τ ≥ e − c^(−1/β): they alone would carry
+//     mass ≥ 1 below it); the values above the bracket are compacted; for
+//     β ∈ {1, 2} and few candidates the support is found by testing every
+//     candidate at once (u_j is in the support iff
+//     Σ_i (u_i − u_j)_+^β < 1) and τ is the float64 closed form on it,
+//     otherwise Newton's method from the left (f is convex and decreasing;
+//     one warp alone when the candidates are few) with a float64 finish.  The
+//     head's support tokens are then compacted and only their V rows are
+//     read, eight rows in flight per warp; warp partials are summed in warp
+//     order.
+// The heads of a unit read the same V rows at about the same time, so a row
+// they share comes from DRAM once.  Every sum has a fixed order, so results
+// are deterministic.
+#include "decode.cuh"
+
+namespace ekv {
+
+namespace {
+
+constexpr int kKsWarps = 8;
+constexpr int kKsThreads = 32 * kKsWarps;
+constexpr int kKsTokens = 32 * kKsWarps;   // selected tokens per CTA of the score launch
+constexpr int kHdThreads = 256;
+constexpr int kHdWarps = kHdThreads / 32;
+constexpr int kHdBins = 256;
+constexpr int kHdCand = 2048;              // candidates / support tokens held in shared memory at once
+constexpr int kHdPairMax = 256;            // candidates for the all-at-once support test
+constexpr int kHdRows = 8;                 // V rows in flight per warp
+constexpr int kHdMaxVpt = 64;              // values per thread held in registers (more: read per pass)
+constexpr int kSplitMaxTokens = 65536;     // selected tokens per unit on this path
+static_assert(kHdBins == kHdThreads, "one histogram bin per thread");
+
+// ------------------------------------------------------------------ 1. K scores
+template <int D, int G>
+__global__ void __launch_bounds__(kKsThreads, 2) k_score_kernel(DecodeArgs a) {
+  constexpr int KP = D / 32, NT = (G + 7) / 8;
+  __shared__ unsigned int cta_key[G];
+  grid_dep_enter();
+  const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int S = a.S;
+  int L;
+  const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
+  const int n_slots = unit_slots(a, unit, P);
+  const int ppc = kKsTokens / S;  // pages per CTA
+  const int s_begin = split * ppc;
+  if (s_begin >= n_slots) return;  // CTA-uniform
+  if (tid < G) cta_key[tid] = 0u;
+  const int row0 = warp * 32;
+  int phys[2], nv[2], slot[2];
+  bool live[2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const int r = row0 + mt * 16;
+    slot[mt] = s_begin + r / S;
+    live[mt] = slot[mt] < n_slots;
+    phys[mt] = -1;
+    nv[mt] = 0;
+    if (live[mt]) phys[mt] = slot_page(a, unit, b, slot[mt], P, L, &nv[mt]);
+  }
+  uint4 va[2][KP], vb[2][KP];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const int tok0 = (row0 + mt * 16) % S;
+    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+    const bf16* kb = static_cast<const bf16*>(a.k_pool) +
+                     ((static_cast<size_t>(phys[mt] < 0 ? 0 : phys[mt]) * a.Hkv + kvh) * S + tok0) * D;
+    const uint4* row_lo = reinterpret_cast<const uint4*>(kb + g * D) + t;
+    const uint4* row_hi = reinterpret_cast<const uint4*>(kb + (g + 8) * D) + t;
+#pragma unroll
+    for (int c = 0; c < KP; ++c) {
+      va[mt][c] = ok_lo ? __ldcs(row_lo + 4 * c) : make_uint4(0, 0, 0, 0);
+      vb[mt][c] = ok_hi ? __ldcs(row_hi + 4 * c) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // the physical page of each selected slot, for the V pass
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+    if (lane == 0 && live[mt] && (row0 + mt * 16) % S == 0)
+      a.ws.sphys[static_cast<size_t>(unit) * a.cap + slot[mt]] = phys[mt];
+  uint32_t bfrag[2 * KP][NT][2];
+  load_q_frags<D, G>(a, b, kvh, g, t, bfrag);
+  __syncthreads();  // cta_key initialised
+  const size_t zrow_len = static_cast<size_t>(a.cap) * S;
+  float wmax[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) wmax[nt][0] = wmax[nt][1] = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    float acc[NT][4];
+    score_mtile<D, G>(va[mt], vb[mt], bfrag, acc);
+    const int tok0 = (row0 + mt * 16) % S;
+    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int hd = nt * 8 + 2 * t + e;
+        const float zl = ok_lo ? a.scale * acc[nt][e] : -INFINITY;
+        const float zh = ok_hi ? a.scale * acc[nt][2 + e] : -INFINITY;
+        if (live[mt] && hd < G) {
+          float* zr = a.ws.zbuf + (static_cast<size_t>(unit) * G + hd) * zrow_len + static_cast<size_t>(slot[mt]) * S + tok0;
+          zr[g] = zl;
+          zr[g + 8] = zh;
+        }
+        wmax[nt][e] = fmaxf(wmax[nt][e], fmaxf(zl, zh));
+      }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float m = wmax[nt][e];
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      const int hd = nt * 8 + 2 * t + e;
+      if (g == 0 && hd < G && m > -INFINITY) atomicMax(&cta_key[hd], float_key(m));
+    }
+  __syncthreads();
+  if (tid < G) {
+    const unsigned int k = cta_key[tid];
+    a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
+  }
+}
+
+// ------------------------------------------------------------------ 2. τ and V per head
+struct HdShared {
+  int hist[kHdBins];
+  float cu[kHdCand];  // candidates above the bracket, then the support's weights
+  int ci[kHdCand];    // their token indices
+  float f[kHdWarps];
+  double d[3][kHdWarps];
+  int i[kHdWarps];
+};
+
+// Sums of (x, y, z) over the CTA in a fixed order; every thread gets them.
+__device__ __forceinline__ void hd_sum3(double& x, double& y, double& z, HdShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_sum(x);
+  y = warp_sum(y);
+  z = warp_sum(z);
+  __syncthreads();  // the previous sums' reads are done
+  if (lane == 0) {
+    sh.d[0][warp] = x;
+    sh.d[1][warp] = y;
+    sh.d[2][warp] = z;
+  }
+  __syncthreads();
+  x = y = z = 0.0;
+#pragma unroll
+  for (int w = 0; w < kHdWarps; ++w) {
+    x += sh.d[0][w];
+    y += sh.d[1][w];
+    z += sh.d[2][w];
+  }
+}
+
+__device__ __forceinline__ double hd_closed_tau(int ipow, double c, double s1, double s2) {
+  if (ipow == 1) return (s1 - 1.0) / c;
+  const double M = s1 / c, Q = s2 / c;
+  return M - sqrt(fmax(M * M - Q + 1.0 / c, 0.0));
+}
+
+// w^(β−1) for w > 0.
+template <typename V>
+__device__ __forceinline__ V hd_pow_bm1(V w, V beta, int ipow) {
+  switch (ipow) {
+    case 1: return V(1);
+    case 2: return w;
+    case 3: return w * w;
+    case 4: return w * w * w;
+    default:
+      if constexpr (sizeof(V) == 8) return pow(w, beta - 1.0);
+      else return exp2f((beta - 1.0f) * __log2f(w));
+  }
+}
+
+template <int D, int VPT>
+__global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, int G) {
+  constexpr int DPL = D / 32;
+  __shared__ HdShared sh;
+  __shared__ float red[kHdWarps][D];
+  grid_dep_enter();
+  const int row = blockIdx.x, unit = row / G, hg = row - unit * G, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = a.S;
+  int L;
+  const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
+  const int n = unit_slots(a, unit, P) * S;
+  const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + hg;
+  const float* z = a.ws.zbuf + static_cast<size_t>(row) * a.cap * S;
+  const float am1 = a.am1, beta = a.beta;
+  const int ipow = a.ipow;
+
+  // value k of this thread is token i = k·256 + tid: held in registers
+  // (VPT > 0), or read again from the scratch at every pass (VPT == 0)
+  constexpr bool kReg = VPT > 0;
+  const int NK = kReg ? VPT : (n + kHdThreads - 1) / kHdThreads;
+  float uv[kReg ? VPT : 1];
+  if constexpr (kReg) {
+#pragma unroll
+    for (int k = 0; k < (kReg ? VPT : NK); ++k) {
+      const int i = k * kHdThreads + tid;
+      uv[k] = i < n ? am1 * z[i] : -INFINITY;
+    }
+  }
+  auto val = [&](int k) -> float {
+    if constexpr (kReg) {
+      return uv[k];
+    } else {
+      const int i = k * kHdThreads + tid;
+      return i < n ? am1 * __ldcg(z + i) : -INFINITY;
+    }
+  };
+  // the head's maximum from the chunk maxima
+  const int nchunk = (n + kKsTokens - 1) / kKsTokens;
+  float m = -INFINITY;
+  for (int c = lane; c < nchunk; c += 32) m = fmaxf(m, a.ws.cmax[static_cast<size_t>(row) * a.ws.nqk + c]);
+  m = warp_max(m);  // every warp reads them all: no barrier
+  sh.hist[tid] = 0;
+  __syncthreads();
+
+  float tau = INFINITY;  // no finite score: no support, zero output
+  if (m > -INFINITY) {
+    const float um = am1 * m;
+    // 1. bracket from the histogram of u over (um − 1, um], bin 0 at the top
+#pragma unroll
+    for (int k = 0; k < (kReg ? VPT : NK); ++k)
+      if (val(k) > um - 1.0f) atomicAdd(&sh.hist[min(kHdBins - 1, static_cast<int>((um - val(k)) * kHdBins))], 1);
+    __syncthreads();
+    float cb = um - 1.0f;
+    {
+      const int h = sh.hist[tid];
+      int total;
+      const int c = block_exclusive_scan(h, sh.i, &total) + h;  // values in bins 0..tid
+      if (c > 0) {
+        const float fc = static_cast<float>(c);
+        const float inv = ipow == 1 ? 1.0f / fc : (ipow == 2 ? rsqrtf(fc) : exp2f(-__log2f(fc) / beta));
+        cb = fmaxf(cb, um - static_cast<float>(tid + 1) / kHdBins - inv);
+      }
+    }
+    cb = warp_max(cb);
+    if (lane == 0) sh.f[warp] = cb;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kHdWarps; ++w) cb = fmaxf(cb, sh.f[w]);
+    // slack for the fp32 rounding of the bound: τ_lo stays below τ
+    const double tau_lo = static_cast<double>(cb) - 4e-6 * (1.0 + fabs(static_cast<double>(um)));
+    float tlo = static_cast<float>(tau_lo);
+    if (static_cast<double>(tlo) > tau_lo) tlo = nextafterf(tlo, -INFINITY);
+
+    // 2. compaction of the values above τ_lo: thread after thread (a fixed
+    //    order, so every later sum is deterministic), one block scan
+    int nc;
+    {
+      int mine = 0;
+#pragma unroll
+      for (int k = 0; k < (kReg ? VPT : NK); ++k) mine += val(k) > tlo ? 1 : 0;
+      int p = block_exclusive_scan(mine, sh.i, &nc);
+#pragma unroll
+      for (int k = 0; k < (kReg ? VPT : NK); ++k)
+        if (val(k) > tlo) {
+          if (p < kHdCand) {
+            sh.cu[p] = val(k);
+            sh.ci[p] = k * kHdThreads + tid;
+          }
+          ++p;
+        }
+      __syncthreads();
+    }
+    const bool listed = nc <= kHdCand;
+
+    // 3. τ
+    const bool closed = ipow == 1 || ipow == 2;
+    double tt;
+    if (closed && nc <= kHdPairMax) {
+      // u_j is in the support iff Σ_i (u_i − u_j)_+^β < 1 (f decreases and f(τ) = 1)
+      double c = 0.0, s1 = 0.0, s2 = 0.0;
+      if (tid < nc) {
+        const float uj = sh.cu[tid];
+        float fs = 0.f;
+        for (int i = 0; i < nc; ++i) {
+          const float w = sh.cu[i] - uj;
+          if (w > 0.f) fs = fmaf(ipow == 1 ? 1.0f : w, w, fs);
+        }
+        if (fs < 1.0f) {
+          c = 1.0;
+          s1 = uj;
+          s2 = static_cast<double>(uj) * uj;
+        }
+      }
+      hd_sum3(c, s1, s2, sh);
+      tt = hd_closed_tau(ipow, c, s1, s2);
+      // the closed form must imply the support it was built on; if rounding
+      // at the edge says otherwise, repeat it on {u > τ} until it is stable
+      for (int rep = 0; rep < 8; ++rep) {
+        double c2 = 0.0, t1 = 0.0, t2 = 0.0;
+        if (tid < nc) {
+          const double u = sh.cu[tid];
+          if (u > tt) {
+            c2 = 1.0;
+            t1 = u;
+            t2 = u * u;
+          }
+        }
+        hd_sum3(c2, t1, t2, sh);
+        if (c2 == c || c2 < 1.0) break;
+        c = c2;
+        const double t_new = hd_closed_tau(ipow, c2, t1, t2);
+        if (t_new == tt) break;
+        tt = t_new;
+      }
+    } else {
+      // Newton from the left in fp32 over the candidates (or every value),
+      // then a float64 finish
+      auto sums = [&](auto t, auto& f, auto& df) {
+        using V = decltype(t);
+        V x = V(0), y = V(0);
+        auto term = [&](float u) {
+          const V w = static_cast<V>(u) - t;
+          if (w > V(0)) {
+            const V wb1 = hd_pow_bm1<V>(w, static_cast<V>(beta), ipow);
+            x += wb1 * w;
+            y += wb1;
+          }
+        };
+        if (listed) {
+          for (int j = tid; j < nc; j += kHdThreads) term(sh.cu[j]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < (kReg ? VPT : NK); ++k) term(val(k));
+        }
+        double dx = x, dy = y, dz = 0.0;
+        hd_sum3(dx, dy, dz, sh);
+        f = static_cast<V>(dx - 1.0);
+        df = static_cast<V>(dy);
+      };
+      // one warp alone over a short candidate list (no barriers per step)
+      auto warp_sums = [&](auto t, auto& f, auto& df) {
+        using V = decltype(t);
+        V x = V(0), y = V(0);
+        for (int j = lane; j < nc; j += 32) {
+          const V w = static_cast<V>(sh.cu[j]) - t;
+          if (w > V(0)) {
+            const V wb1 = hd_pow_bm1<V>(w, static_cast<V>(beta), ipow);
+            x += wb1 * w;
+            y += wb1;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          x += __shfl_xor_sync(0xffffffffu, x, o);
+          y += __shfl_xor_sync(0xffffffffu, y, o);
+        }
+        f = x - V(1);
+        df = y;
+      };
+      const bool solo = listed && nc <= 1024;
+      if (solo) {
+        if (warp == 0) {
+          float t = tlo;
+          for (int it = 0; it < 100; ++it) {
+            float f, df;
+            warp_sums(t, f, df);
+            if (it == 0 && f < 0.0f) {
+              t = um - 1.0f;
+              continue;
+            }
+            const float step = f / (beta * df);
+            if (!(step > 0.0f)) break;
+            t += step;
+            if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+          }
+          double d = t;
+          if (closed) {
+            for (int rep = 0; rep < 4; ++rep) {
+              double c3 = 0.0, t1 = 0.0, t2 = 0.0;
+              for (int j = lane; j < nc; j += 32) {
+                const double u = sh.cu[j];
+                if (u > d) {
+                  c3 += 1.0;
+                  t1 += u;
+                  t2 += u * u;
+                }
+              }
+              c3 = warp_sum(c3);
+              t1 = warp_sum(t1);
+              t2 = warp_sum(t2);
+              if (c3 < 1.0) break;
+              const double t_new = hd_closed_tau(ipow, c3, t1, t2);
+              if (t_new == d) break;
+              d = t_new;
+            }
+          } else {
+            double f, df;
+            warp_sums(d, f, df);
+            if (df > 0.0) d += f / (static_cast<double>(beta) * df);
+          }
+          if (lane == 0) sh.d[0][0] = d;
+        }
+        __syncthreads();
+        tt = sh.d[0][0];
+      } else {
+      float t = tlo;
+      for (int it = 0; it < 64; ++it) {
+        float f, df;
+        sums(t, f, df);
+        if (it == 0 && f < 0.0f) {  // bracket missed by rounding: restart from max u − 1
+          t = um - 1.0f;
+          continue;
+        }
+        const float step = f / (beta * df);
+        if (!(step > 0.0f)) break;
+        t += step;
+        if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+      }
+      tt = t;
+      if (closed) {
+        for (int rep = 0; rep < 4; ++rep) {
+          double c3 = 0.0, t1 = 0.0, t2 = 0.0;
+          auto add = [&](float uf) {
+            const double u = uf;
+            if (u > tt) {
+              c3 += 1.0;
+              t1 += u;
+              t2 += u * u;
+            }
+          };
+          if (listed) {
+            for (int j = tid; j < nc; j += kHdThreads) add(sh.cu[j]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < (kReg ? VPT : NK); ++k) add(val(k));
+          }
+          hd_sum3(c3, t1, t2, sh);
+          if (c3 < 1.0) break;
+          const double t_new = hd_closed_tau(ipow, c3, t1, t2);
+          if (t_new == tt) break;
+          tt = t_new;
+        }
+      } else {
+        double f, df;
+        sums(tt, f, df);
+        if (df > 0.0) tt += f / (static_cast<double>(beta) * df);
+      }
+      }
+    }
+    tau = static_cast<float>(tt);
+  }
+  __syncthreads();  // the candidate area is reused for the support list
+
+  // 4. support with the fp32 τ every later step uses: bits by ballots, and
+  //    compact(base) lists the support tokens at places base .. base +
+  //    kHdCand − 1 (thread after thread) with their weights p = (u − τ)^β;
+  //    it returns the support's size.
+  if (a.bits_out) {
+#pragma unroll
+    for (int k = 0; k < (kReg ? VPT : NK); ++k) {
+      const int i = k * kHdThreads + tid;
+      const unsigned int bal = __ballot_sync(0xffffffffu, i < n && val(k) > tau);
+      if (lane == 0 && (i >> 5) < a.words) a.bits_out[orow * a.words + (i >> 5)] = bal;
+    }
+  }
+  auto compact = [&](int base) {
+    int mine = 0;
+#pragma unroll
+    for (int k = 0; k < (kReg ? VPT : NK); ++k) mine += (k * kHdThreads + tid < n && val(k) > tau) ? 1 : 0;
+    int ns;
+    int p = block_exclusive_scan(mine, sh.i, &ns) - base;
+#pragma unroll
+    for (int k = 0; k < (kReg ? VPT : NK); ++k) {
+      const int i = k * kHdThreads + tid;
+      if (i < n && val(k) > tau) {
+        if (p >= 0 && p < kHdCand) {
+          sh.cu[p] = pow_beta_fast(val(k) - tau, beta, ipow);
+          sh.ci[p] = i;
+        }
+        ++p;
+      }
+    }
+    __syncthreads();
+    return ns;
+  };
+  const int ns = compact(0);
+  if (a.bits_out)
+    for (int w = (VPT * kHdThreads) / 32 + tid; w < a.words; w += kHdThreads) a.bits_out[orow * a.words + w] = 0u;
+  if (tid == 0) {
+    if (a.tau_out) a.tau_out[orow] = tau;
+    if (a.count_out) a.count_out[orow] = ns;
+  }
+
+  // 5. V of the support rows: warp w takes rows w·8 … w·8+7 of each block of 64
+  float acc[DPL];
+#pragma unroll
+  for (int x = 0; x < DPL; ++x) acc[x] = 0.f;
+  for (int base = 0; base < ns; base += kHdCand) {
+    if (base > 0) compact(base);
+    const int nl = min(ns - base, kHdCand);
+    for (int e0 = warp * kHdRows; e0 < nl; e0 += kHdWarps * kHdRows) {
+      float v[kHdRows][DPL];
+      float p[kHdRows];
+#pragma unroll
+      for (int r = 0; r < kHdRows; ++r) {
+        const int e = e0 + r;
+        p[r] = 0.f;
+#pragma unroll
+        for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
+        if (e < nl) {
+          const int tok = sh.ci[e];
+          const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
+          if (ph >= 0) {
+            p[r] = sh.cu[e];
+            const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                              ((static_cast<size_t>(ph) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
+            if constexpr (DPL == 4) {
+              const uint2 w2 = *reinterpret_cast<const uint2*>(src);
+              v[r][0] = __uint_as_float(w2.x << 16);
+              v[r][1] = __uint_as_float(w2.x & 0xffff0000u);
+              v[r][2] = __uint_as_float(w2.y << 16);
+              v[r][3] = __uint_as_float(w2.y & 0xffff0000u);
+            } else {
+              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
+              v[r][0] = __uint_as_float(w1 << 16);
+              v[r][1] = __uint_as_float(w1 & 0xffff0000u);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kHdRows; ++r)
+#pragma unroll
+        for (int x = 0; x < DPL; ++x) acc[x] = fmaf(p[r], v[r][x], acc[x]);
+    }
+    __syncthreads();  // the list is rewritten by the next round
+  }
+#pragma unroll
+  for (int x = 0; x < DPL; ++x) red[warp][lane * DPL + x] = acc[x];
+  __syncthreads();
+  for (int i = tid; i < D; i += kHdThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kHdWarps; ++w) s += red[w][i];
+    a.out[orow * D + i] = s;
+  }
+}
+
+template <int D>
+cudaError_t launch_head_decode(DecodeArgs& a, int rows, int G, cudaStream_t st) {
+  const int n_max = a.cap * a.S;
+#define EKV_HD_CASE(VV)                                                                                  \
+  if (n_max <= (VV) * kHdThreads) {                                                                      \
+    const cudaError_t e = launch_k(head_decode_kernel<D, VV>, dim3(rows), dim3(kHdThreads), 0, st, a, G); \
+    if (e != cudaSuccess) return e;                                                                      \
+    return cudaGetLastError();                                                                           \
+  }
+  EKV_HD_CASE(4) EKV_HD_CASE(16) EKV_HD_CASE(32) EKV_HD_CASE(kHdMaxVpt)
+#undef EKV_HD_CASE
+  const cudaError_t e = launch_k(head_decode_kernel<D, 0>, dim3(rows), dim3(kHdThreads), 0, st, a, G);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+template <int D, int G>
+bool split_decode_fits(int cap, int S) {
+  return S % 16 == 0 && cap >= 1 && static_cast<long long>(cap) * S <= kSplitMaxTokens;
+}
+
+template <int D, int G>
+cudaError_t run_split_decode(DecodeArgs& a, int units, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(a.ws.nqk), static_cast<unsigned>(units));
+  cudaError_t e = launch_k(k_score_kernel<D, G>, grid, dim3(kKsThreads), 0, st, a);
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_head_decode<D>(a, units * G, G, st);
+}
+
+#define EKV_SPLIT_INST(DD, GG)                               \
+  template bool split_decode_fits<DD, GG>(int, int);         \
+  template cudaError_t run_split_decode<DD, GG>(DecodeArgs&, int, cudaStream_t);
+EKV_SPLIT_INST(128, 1)
+EKV_SPLIT_INST(128, 2)
+EKV_SPLIT_INST(128, 4)
+EKV_SPLIT_INST(128, 8)
+EKV_SPLIT_INST(128, 16)
+EKV_SPLIT_INST(64, 1)
+EKV_SPLIT_INST(64, 2)
+EKV_SPLIT_INST(64, 4)
+EKV_SPLIT_INST(64, 8)
+EKV_SPLIT_INST(64, 16)
+#undef EKV_SPLIT_INST
+
+}  // namespace ekv

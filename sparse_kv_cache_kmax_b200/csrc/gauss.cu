@@ -16,8 +16,8 @@
 // n·σ^β·J_β(kPruneC) and stay negligible for every later τ (c only grows), so
 // only the survivors are iterated, from shared memory.  The recurrence
 // amplifies the rounding of Q and φ by about c^(2β)/β! for c > 0, so the fp32
-// iterations only approach the root; two final Newton steps evaluate every
-// term in float64.
+// iterations only approach the root (they stop once a step is below 1e-5);
+// the final Newton steps evaluate every term in float64.
 #include "kernels.cuh"
 
 namespace ekv {
@@ -85,9 +85,9 @@ __global__ void __launch_bounds__(kGaussThreads)
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
   __shared__ float c_mu[kGaussCand], c_sg[kGaussCand], c_n[kGaussCand];
-  __shared__ int s_count;
   __shared__ float f_scratch[32];
   __shared__ double d_scratch[32];
+  __shared__ int i_scratch[32];
 
   // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
   const size_t base = static_cast<size_t>(row) * max_pages;
@@ -106,23 +106,36 @@ __global__ void __launch_bounds__(kGaussThreads)
     return;
   }
 
-  if (tid == 0) s_count = 0;
-  __syncthreads();
-  for (int p = tid; p < P; p += blockDim.x) {
+  // candidates in page order: thread t owns the run of pages [t·R, t·R + R)
+  const int R = (P + kGaussThreads - 1) / kGaussThreads;
+  auto live = [&](int p) {
     const float mu = ws.mu[base + p], sg = ws.sig[base + p];
-    if (mu > -INFINITY && mu + kPruneC * sg > lo) {
-      const int slot = atomicAdd(&s_count, 1);
-      if (slot < kGaussCand) {
-        c_mu[slot] = mu;
-        c_sg[slot] = sg;
-        c_n[slot] = static_cast<float>(min(S, L - p * S));
+    return mu > -INFINITY && mu + kPruneC * sg > lo;
+  };
+  int mine = 0;
+  for (int j = 0; j < R; ++j) {
+    const int p = tid * R + j;
+    if (p < P && live(p)) ++mine;
+  }
+  int nc;
+  {
+    int pos = block_exclusive_scan(mine, i_scratch, &nc);
+    if (nc <= kGaussCand)
+      for (int j = 0; j < R; ++j) {
+        const int p = tid * R + j;
+        if (p < P && live(p)) {
+          c_mu[pos] = ws.mu[base + p];
+          c_sg[pos] = ws.sig[base + p];
+          c_n[pos] = static_cast<float>(min(S, L - p * S));
+          ++pos;
+        }
       }
-    }
   }
   __syncthreads();
-  const int nc = s_count;
   const bool cached = nc <= kGaussCand;
 
+  // F(τ) − 1 and F'(τ) over the candidates (or every page), summed in a
+  // fixed order
   auto evaluate = [&](double t, bool exact, double& F, double& dF) {
     F = 0.0;
     dF = 0.0;
@@ -142,23 +155,43 @@ __global__ void __launch_bounds__(kGaussThreads)
           gauss_terms<float>(ws.mu[base + p], ws.sig[base + p], n, t, beta, F, dF);
       }
     }
-    F = block_reduce(F, d_scratch, [](double x, double y) { return x + y; });
-    dF = block_reduce(dF, d_scratch, [](double x, double y) { return x + y; });
+    const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      F += __shfl_xor_sync(0xffffffffu, F, o);
+      dF += __shfl_xor_sync(0xffffffffu, dF, o);
+    }
+    __syncthreads();  // the previous evaluation's partials are read
+    if (lane == 0) {
+      d_scratch[warp] = F;
+      d_scratch[16 + warp] = dF;
+    }
+    __syncthreads();
+    F = 0.0;
+    dF = 0.0;
+    for (int w = 0; w < kGaussThreads / 32; ++w) {
+      F += d_scratch[w];
+      dF += d_scratch[16 + w];
+    }
   };
+  // fp32 terms: a monotone approach from the left while the steps are large;
+  // the float64 steps below converge quadratically from there
   double tau = static_cast<double>(lo);
-  for (int it = 0; it < 100; ++it) {  // fp32 terms: monotone approach from the left
+  for (int it = 0; it < 40; ++it) {
     double F, dF;
     evaluate(tau, false, F, dF);
     const double step = (F - 1.0) / dF;
     if (!(step > 0.0)) break;
     tau += step;
-    if (step <= 1e-7 * fmax(1.0, fabs(tau))) break;
+    if (step <= 1e-5 * fmax(1.0, fabs(tau))) break;
   }
-  for (int it = 0; it < 2; ++it) {    // float64 terms: quadratic polish (either side)
+  for (int it = 0; it < 6; ++it) {    // float64 terms: quadratic convergence (either side)
     double F, dF;
     evaluate(tau, true, F, dF);
     if (!(dF > 0.0)) break;
-    tau += (F - 1.0) / dF;
+    const double step = (F - 1.0) / dF;
+    tau += step;
+    if (fabs(step) <= 1e-12 * fmax(1.0, fabs(tau))) break;
   }
   if (tid == 0) {
     ws.tau_hat[row] = tau;
@@ -183,28 +216,43 @@ __global__ void __launch_bounds__(kGaussThreads)
   if (tid < G) s_thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
   __syncthreads();
   int32_t* out = sel + static_cast<size_t>(unit) * cap;
-  int carry = 0;
+  // thread t owns the run of pages [t·R, t·R + R): one pass counts the kept
+  // pages (and finds the best margin), one block scan places them, a second
+  // pass over the same run (now in L1) writes them in ascending page order
+  const int R = (P + kGaussThreads - 1) / kGaussThreads;
+  auto margin = [&](int p) {
+    double mg = -INFINITY;
+    for (int g = 0; g < G; ++g) {
+      const double m = static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - s_thr[g];
+      mg = fmax(mg, m);
+    }
+    return mg;
+  };
   double my_best = -INFINITY;
   int my_idx = 0x7fffffff;
-  for (int base = 0; base < P; base += blockDim.x) {
-    const int p = base + tid;
-    int keep = 0;
+  int mine = 0;
+  for (int j = 0; j < R; ++j) {
+    const int p = tid * R + j;
     if (p < P) {
-      double mg = -INFINITY;
-      for (int g = 0; g < G; ++g) {
-        const double m = static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - s_thr[g];
-        mg = fmax(mg, m);
-      }
-      keep = mg > 0.0 ? 1 : 0;
+      const double mg = margin(p);
+      mine += mg > 0.0 ? 1 : 0;
       if (mg > my_best) {
         my_best = mg;
         my_idx = p;
       }
     }
-    int total;
-    const int pos = block_exclusive_scan(keep, scan_scratch, &total) + carry;
-    if (keep && pos < cap) out[pos] = p;
-    carry += total;
+  }
+  int carry;
+  {
+    int pos = block_exclusive_scan(mine, scan_scratch, &carry);
+    if (mine > 0)
+      for (int j = 0; j < R; ++j) {
+        const int p = tid * R + j;
+        if (p < P && margin(p) > 0.0) {
+          if (pos < cap) out[pos] = p;
+          ++pos;
+        }
+      }
   }
   if (carry > 0) {
     if (tid == 0) {

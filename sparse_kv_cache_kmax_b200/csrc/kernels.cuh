@@ -19,8 +19,10 @@ struct DecodeWs {
   float* taus;      // [U, G]        thresholds τ (fp32)
   float* part;      // [U, npv, G, d] partial outputs of the V pass
   int* counter;     // [U]           finished V-pass CTAs
+  int* sphys;       // [U, cap]      physical page of each selected slot (−1: bad)
   int nqk, npv;     // score-pass and V-pass CTAs per unit
 };
+
 
 struct GaussWs {
   float* mu;        // [U, G, max_pages] (α−1)·m
@@ -72,8 +74,8 @@ cudaError_t launch_softmax_decode(const ekv_cache& c, const ekv_seqs& s, const v
                                   float scale, const int32_t* sel, const int32_t* n_sel, int cap,
                                   float* out, float* lse, void* ws, cudaStream_t st);
 
-// Kernels one launch_decode enqueues for these sizes (1 fused, or 3).
-int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap);
+// Kernels one launch_decode enqueues for these sizes (2: split decode, 1: cluster decode, 3: three-kernel decode).
+int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap, int dense_v);
 
 // Score-pass CTAs per unit: cap pages of S tokens, 256 tokens per CTA.
 inline int qk_splits(int cap, int S) {

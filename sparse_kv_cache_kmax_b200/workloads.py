@@ -221,5 +221,9 @@ def make_inputs(wl: Workload, seed: int, device="cpu", n_new: int = 1) -> dict:
 
 def gauss_cap(wl: Workload, max_pages: int) -> int:
     """Pages a unit may keep under the Gaussian policy (the ``cap`` of
-    ekv_select_gauss / ekv_decode_step): every page of the sequence."""
-    return int(max_pages)
+    ekv_select_gauss / ekv_decode_step, which sizes the selection buffer and
+    the decode's scratch): every page of the sequence, at most 65536 tokens'
+    worth (4096 pages of 16 tokens, 2048 of 32).  A selection past the cap keeps its
+    first cap pages and raises EKV_EFLAG_SEL_OVERFLOW, which the tests check
+    is never raised on these workloads."""
+    return int(min(max_pages, 65536 // wl.page_size))

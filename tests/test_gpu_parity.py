@@ -228,8 +228,9 @@ def test_decode_step_end_to_end(case, policy):
         G = wl.group
         err = row_rel_err(np64(out[b, h * G:(h + 1) * G]), orc["o"])
         assert np.all(err <= OUT_TOL[wl.dtype]), (policy, b, h, err.max())
-    # the step ran the kernels it says: bf16 top-k selections take the one-kernel
-    # cluster decode (append + score + top-k + decode); fp32 the three-kernel one
+    # the step ran the kernels it says: append + scores + one-stage top-k,
+    # then for bf16 the cluster decode (few units) or the two-launch split
+    # decode (many units), for fp32 the three-kernel decode
     n_kern = B.ekv_step_kernel_count(eng.cache, eng.seqs, eng.params, wl.num_q_heads)
     if policy == "topk":
-        assert n_kern == (4 if wl.dtype == "bf16" else 6), n_kern
+        assert n_kern - 3 in ((1, 2) if wl.dtype == "bf16" else (3,)), n_kern

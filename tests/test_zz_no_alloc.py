@@ -37,8 +37,8 @@ def _static_decode(gpu, alpha, sel, n_sel, cap):
 
 
 def _decode_kernels(gpu, cap):
-    """Kernels the decode of these sizes launches (a top-k step's count minus
-    its score and one-stage top-k kernels)."""
+    """Kernels the decode of these sizes launches: a top-k step's count minus
+    its page scores and one-stage top-k."""
     p = B.StepParams(B.EKV_POLICY_TOPK, cap, 0.0, cap, 1.5, gpu.scale, 0, 0)
     return B.ekv_step_kernel_count(gpu.cache, gpu.seqs, p, gpu.Hq) - 2
 
@@ -53,9 +53,10 @@ def _case(name, over, seed, k):
     return gpu, sel, n_sel
 
 
-# bf16 selection: the one-launch decode; fp32 cache: the three-kernel decode
+# many bf16 units: the two-launch split decode; fp32 cache: the three-kernel
+# decode; both keep their scores, maxima and page ids in the scratch
 CASES = {
-    "bf16_topk": ("clustered_128k", dict(batch=2, context=3005), 4242, 24),
+    "bf16_topk": ("short_scattered", dict(batch=10, context=900, context_min=300), 4242, 24),
     "f32_topk": ("tiny_fp32", dict(batch=2, context=4093), 4243, 32),
 }
 
@@ -64,11 +65,11 @@ CASES = {
 def test_static_scratch_decode_matches_workspace_decode_and_oracle_twice(case):
     name, over, seed, k = CASES[case]
     gpu, sel, n_sel = _case(name, over, seed, k)
-    other, osel, on = _case("gqa_32k", dict(batch=3, context=2500), 4244, 40)
+    other, osel, on = _case("short_scattered", dict(batch=12, context=1500, context_min=700), 4244, 40)
     wl = gpu.wl
     assert B.ekv_workspace_bytes(B.EKV_OP_ENTMAX_DECODE, gpu.cache, gpu.seqs, gpu.Hq, k) > 0
     kernels = _decode_kernels(gpu, k)
-    assert kernels == (3 if wl.dtype == "f32" else 1), kernels
+    assert kernels == (3 if wl.dtype == "f32" else 2), kernels
     ref = gpu.decode(1.5, sel, n_sel, k)
     torch.cuda.synchronize()
     orcs = {(b, h): oracle_unit(gpu.inp, b, h, sel=sel[b, h, : int(n_sel[b, h])].cpu().numpy())
