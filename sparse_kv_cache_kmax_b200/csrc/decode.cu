@@ -34,7 +34,9 @@ constexpr int kQkWarps = kQkTokensPerCta / 32;
 
 template <int D, int G>
 __global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) {
-  grid_dep_enter();
+  // the τ kernel that follows is let in only at the end: its CTAs, resident
+  // early, would take the SM slots of this launch's many short CTAs
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int KP = D / 32;          // 32-element chunks per K row
   constexpr int NT = (G + 7) / 8;     // 8-head tiles of the B operand
   __shared__ unsigned int cta_key[G];
@@ -140,12 +142,13 @@ __global__ void __launch_bounds__(32 * kQkWarps, 2) qk_mma_kernel(DecodeArgs a) 
     const unsigned int k = cta_key[tid];
     a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
   }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ 1'. qk (CUDA cores, fp32 caches)
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) qk_cc_kernel(DecodeArgs a) {
-  grid_dep_enter();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // dependents let in at the end, as qk_mma_kernel
   constexpr int PAD = 16 / sizeof(T);
   constexpr int RP = D + PAD;  // padded row pitch: rows start in different bank groups
   constexpr int TP = 4;        // pages staged per round
@@ -226,6 +229,7 @@ __global__ void __launch_bounds__(256) qk_cc_kernel(DecodeArgs a) {
     const unsigned int k = cta_key[tid];
     a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
   }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ 2. tau

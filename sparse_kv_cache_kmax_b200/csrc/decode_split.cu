@@ -39,6 +39,7 @@ constexpr int kHdBins = 256;
 constexpr int kHdCand = 2048;              // candidates / support tokens held in shared memory at once
 constexpr int kHdPairMax = 256;            // candidates for the all-at-once support test
 constexpr int kHdRows = 8;                 // V rows in flight per warp
+constexpr int kHdBatch = 8;                // score loads in flight per thread when streaming
 constexpr int kHdMaxVpt = 64;              // values per thread held in registers (more: read per pass)
 constexpr int kSplitMaxTokens = 65536;     // selected tokens per unit on this path
 static_assert(kHdBins == kHdThreads, "one histogram bin per thread");
@@ -48,7 +49,10 @@ template <int D, int G>
 __global__ void __launch_bounds__(kKsThreads, 2) k_score_kernel(DecodeArgs a) {
   constexpr int KP = D / 32, NT = (G + 7) / 8;
   __shared__ unsigned int cta_key[G];
-  grid_dep_enter();
+  // wait for the previous kernel; the per-head kernel that follows is let in
+  // only at the end (its CTAs hold many registers: resident early, they
+  // would crowd this launch's CTAs off the SMs)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(kKsThreads, 2) k_score_kernel(DecodeArgs a) {
     const unsigned int k = cta_key[tid];
     a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
   }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ 2. τ and V per head
@@ -221,12 +226,25 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
       uv[k] = i < n ? am1 * z[i] : -INFINITY;
     }
   }
-  auto val = [&](int k) -> float {
+  // fn(k, u) for every value of this thread in order of k; read from the
+  // scratch in batches of kHdBatch independent loads when not in registers
+  // (fn may hold warp collectives: k runs alike on every lane)
+  auto for_values = [&](auto fn) {
     if constexpr (kReg) {
-      return uv[k];
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) fn(k, uv[k]);
     } else {
-      const int i = k * kHdThreads + tid;
-      return i < n ? am1 * __ldcg(z + i) : -INFINITY;
+      for (int k0 = 0; k0 < NK; k0 += kHdBatch) {
+        float v[kHdBatch];
+#pragma unroll
+        for (int j = 0; j < kHdBatch; ++j) {
+          const int i = (k0 + j) * kHdThreads + tid;
+          v[j] = (k0 + j < NK && i < n) ? am1 * __ldcg(z + i) : -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < kHdBatch; ++j)
+          if (k0 + j < NK) fn(k0 + j, v[j]);
+      }
     }
   };
   // the head's maximum from the chunk maxima
@@ -241,9 +259,9 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   if (m > -INFINITY) {
     const float um = am1 * m;
     // 1. bracket from the histogram of u over (um − 1, um], bin 0 at the top
-#pragma unroll
-    for (int k = 0; k < (kReg ? VPT : NK); ++k)
-      if (val(k) > um - 1.0f) atomicAdd(&sh.hist[min(kHdBins - 1, static_cast<int>((um - val(k)) * kHdBins))], 1);
+    for_values([&](int, float u) {
+      if (u > um - 1.0f) atomicAdd(&sh.hist[min(kHdBins - 1, static_cast<int>((um - u) * kHdBins))], 1);
+    });
     __syncthreads();
     float cb = um - 1.0f;
     {
@@ -271,18 +289,16 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
     int nc;
     {
       int mine = 0;
-#pragma unroll
-      for (int k = 0; k < (kReg ? VPT : NK); ++k) mine += val(k) > tlo ? 1 : 0;
+      for_values([&](int, float u) { mine += u > tlo ? 1 : 0; });
       int p = block_exclusive_scan(mine, sh.i, &nc);
-#pragma unroll
-      for (int k = 0; k < (kReg ? VPT : NK); ++k)
-        if (val(k) > tlo) {
-          if (p < kHdCand) {
-            sh.cu[p] = val(k);
+      if (nc <= kHdCand)
+        for_values([&](int k, float u) {
+          if (u > tlo) {
+            sh.cu[p] = u;
             sh.ci[p] = k * kHdThreads + tid;
+            ++p;
           }
-          ++p;
-        }
+        });
       __syncthreads();
     }
     const bool listed = nc <= kHdCand;
@@ -344,8 +360,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
         if (listed) {
           for (int j = tid; j < nc; j += kHdThreads) term(sh.cu[j]);
         } else {
-#pragma unroll
-          for (int k = 0; k < (kReg ? VPT : NK); ++k) term(val(k));
+          for_values([&](int, float u) { term(u); });
         }
         double dx = x, dy = y, dz = 0.0;
         hd_sum3(dx, dy, dz, sh);
@@ -446,8 +461,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
           if (listed) {
             for (int j = tid; j < nc; j += kHdThreads) add(sh.cu[j]);
           } else {
-#pragma unroll
-            for (int k = 0; k < (kReg ? VPT : NK); ++k) add(val(k));
+            for_values([&](int, float u) { add(u); });
           }
           hd_sum3(c3, t1, t2, sh);
           if (c3 < 1.0) break;
@@ -470,37 +484,34 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   //    compact(base) lists the support tokens at places base .. base +
   //    kHdCand − 1 (thread after thread) with their weights p = (u − τ)^β;
   //    it returns the support's size.
-  if (a.bits_out) {
-#pragma unroll
-    for (int k = 0; k < (kReg ? VPT : NK); ++k) {
+  if (a.bits_out)
+    for_values([&](int k, float u) {
       const int i = k * kHdThreads + tid;
-      const unsigned int bal = __ballot_sync(0xffffffffu, i < n && val(k) > tau);
+      const unsigned int bal = __ballot_sync(0xffffffffu, i < n && u > tau);
       if (lane == 0 && (i >> 5) < a.words) a.bits_out[orow * a.words + (i >> 5)] = bal;
-    }
-  }
+    });
   auto compact = [&](int base) {
     int mine = 0;
-#pragma unroll
-    for (int k = 0; k < (kReg ? VPT : NK); ++k) mine += (k * kHdThreads + tid < n && val(k) > tau) ? 1 : 0;
+    for_values([&](int k, float u) { mine += (k * kHdThreads + tid < n && u > tau) ? 1 : 0; });
     int ns;
     int p = block_exclusive_scan(mine, sh.i, &ns) - base;
-#pragma unroll
-    for (int k = 0; k < (kReg ? VPT : NK); ++k) {
+    for_values([&](int k, float u) {
       const int i = k * kHdThreads + tid;
-      if (i < n && val(k) > tau) {
+      if (i < n && u > tau) {
         if (p >= 0 && p < kHdCand) {
-          sh.cu[p] = pow_beta_fast(val(k) - tau, beta, ipow);
+          sh.cu[p] = pow_beta_fast(u - tau, beta, ipow);
           sh.ci[p] = i;
         }
         ++p;
       }
-    }
+    });
     __syncthreads();
     return ns;
   };
   const int ns = compact(0);
   if (a.bits_out)
-    for (int w = (VPT * kHdThreads) / 32 + tid; w < a.words; w += kHdThreads) a.bits_out[orow * a.words + w] = 0u;
+    for (int w = ((kReg ? VPT : NK) * kHdThreads) / 32 + tid; w < a.words; w += kHdThreads)
+      a.bits_out[orow * a.words + w] = 0u;  // words past the ballots above
   if (tid == 0) {
     if (a.tau_out) a.tau_out[orow] = tau;
     if (a.count_out) a.count_out[orow] = ns;

@@ -26,7 +26,7 @@ namespace {
 
 constexpr int kGaussThreads = 256;
 constexpr int kGaussCand = 3072;
-constexpr float kPruneC = 7.0f;
+constexpr float kPruneC = 6.0f;
 
 template <typename R>
 __device__ __forceinline__ void normal_tail(R c, R& Q, R& phi);
@@ -106,36 +106,69 @@ __global__ void __launch_bounds__(kGaussThreads)
     return;
   }
 
-  // candidates in page order: thread t owns the run of pages [t·R, t·R + R)
-  const int R = (P + kGaussThreads - 1) / kGaussThreads;
-  auto live = [&](int p) {
+  // Candidates: the pages with μ + kPruneC·σ above the current τ.  τ only
+  // rises (Newton from the left), so a page dropped once stays negligible;
+  // the list is cut again as τ climbs.  Gathered thread after thread
+  // (thread t takes pages t, t + 256, …: coalesced loads; a fixed order, so
+  // the sums below are deterministic); while too many pages are left for
+  // shared memory, the steps read every page from global memory.
+  auto live = [&](int p, double t) {
     const float mu = ws.mu[base + p], sg = ws.sig[base + p];
-    return mu > -INFINITY && mu + kPruneC * sg > lo;
+    return mu > -INFINITY && static_cast<double>(mu) + kPruneC * static_cast<double>(sg) > t;
   };
-  int mine = 0;
-  for (int j = 0; j < R; ++j) {
-    const int p = tid * R + j;
-    if (p < P && live(p)) ++mine;
-  }
-  int nc;
-  {
+  int nc = 0;
+  bool cached = false;
+  auto gather = [&](double t) {  // every thread calls it
+    int mine = 0;
+    for (int p = tid; p < P; p += kGaussThreads) mine += live(p, t) ? 1 : 0;
     int pos = block_exclusive_scan(mine, i_scratch, &nc);
-    if (nc <= kGaussCand)
-      for (int j = 0; j < R; ++j) {
-        const int p = tid * R + j;
-        if (p < P && live(p)) {
+    cached = nc <= kGaussCand;
+    if (cached)
+      for (int p = tid; p < P; p += kGaussThreads)
+        if (live(p, t)) {
           c_mu[pos] = ws.mu[base + p];
           c_sg[pos] = ws.sig[base + p];
           c_n[pos] = static_cast<float>(min(S, L - p * S));
           ++pos;
         }
+    __syncthreads();
+  };
+  // cuts the cached list to the pages still above t, in place, order kept:
+  // thread t owns entries [t·R, t·R + R) (R ≤ 16), holds its survivors in
+  // registers across one barrier, then writes them at their new places
+  auto recut = [&](double t) {
+    constexpr int kMaxR = 16;
+    static_assert(kGaussCand <= kMaxR * kGaussThreads, "entries per thread");
+    const int R = (nc + kGaussThreads - 1) / kGaussThreads;
+    float m[kMaxR], sgm[kMaxR], nn[kMaxR];
+    unsigned int keep = 0u;
+#pragma unroll
+    for (int j = 0; j < kMaxR; ++j) {
+      const int i = tid * R + j;
+      m[j] = sgm[j] = nn[j] = 0.f;
+      if (j < R && i < nc) {
+        m[j] = c_mu[i];
+        sgm[j] = c_sg[i];
+        nn[j] = c_n[i];
+        if (static_cast<double>(m[j]) + kPruneC * static_cast<double>(sgm[j]) > t) keep |= 1u << j;
       }
-  }
-  __syncthreads();
-  const bool cached = nc <= kGaussCand;
+    }
+    int total;
+    int pos = block_exclusive_scan(__popc(keep), i_scratch, &total);  // its barriers order the reads before the writes
+#pragma unroll
+    for (int j = 0; j < kMaxR; ++j)
+      if ((keep >> j) & 1u) {
+        c_mu[pos] = m[j];
+        c_sg[pos] = sgm[j];
+        c_n[pos] = nn[j];
+        ++pos;
+      }
+    __syncthreads();
+    nc = total;
+  };
+  gather(static_cast<double>(lo));
 
-  // F(τ) − 1 and F'(τ) over the candidates (or every page), summed in a
-  // fixed order
+  // F(τ) and F'(τ) over the candidates (or every page), summed in a fixed order
   auto evaluate = [&](double t, bool exact, double& F, double& dF) {
     F = 0.0;
     dF = 0.0;
@@ -174,8 +207,9 @@ __global__ void __launch_bounds__(kGaussThreads)
       dF += d_scratch[16 + w];
     }
   };
-  // fp32 terms: a monotone approach from the left while the steps are large;
-  // the float64 steps below converge quadratically from there
+  // fp32 terms: a monotone approach from the left while the steps are large
+  // (the list cut every few steps); the float64 steps below converge
+  // quadratically from there
   double tau = static_cast<double>(lo);
   for (int it = 0; it < 40; ++it) {
     double F, dF;
@@ -184,7 +218,12 @@ __global__ void __launch_bounds__(kGaussThreads)
     if (!(step > 0.0)) break;
     tau += step;
     if (step <= 1e-5 * fmax(1.0, fabs(tau))) break;
+    if ((it & 3) == 3) {
+      if (cached) recut(tau);
+      else gather(tau);
+    }
   }
+  if (!cached) gather(tau);
   for (int it = 0; it < 6; ++it) {    // float64 terms: quadratic convergence (either side)
     double F, dF;
     evaluate(tau, true, F, dF);
@@ -216,10 +255,14 @@ __global__ void __launch_bounds__(kGaussThreads)
   if (tid < G) s_thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
   __syncthreads();
   int32_t* out = sel + static_cast<size_t>(unit) * cap;
-  // thread t owns the run of pages [t·R, t·R + R): one pass counts the kept
-  // pages (and finds the best margin), one block scan places them, a second
-  // pass over the same run (now in L1) writes them in ascending page order
-  const int R = (P + kGaussThreads - 1) / kGaussThreads;
+  // warp w owns the pages [w·C, (w + 1)·C), its lanes consecutive pages
+  // (coalesced loads): one pass counts the kept pages by ballots (and finds
+  // the best margin), the warp counts are scanned, a second pass writes the
+  // kept pages in ascending order
+  const int lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kGaussThreads / 32;
+  const int C = ((P + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int p0 = warp * C, p1 = min(P, p0 + C);
   auto margin = [&](int p) {
     double mg = -INFINITY;
     for (int g = 0; g < G; ++g) {
@@ -230,29 +273,37 @@ __global__ void __launch_bounds__(kGaussThreads)
   };
   double my_best = -INFINITY;
   int my_idx = 0x7fffffff;
-  int mine = 0;
-  for (int j = 0; j < R; ++j) {
-    const int p = tid * R + j;
-    if (p < P) {
+  int wcount = 0;
+  for (int q0 = p0; q0 < p1; q0 += 32) {
+    const int p = q0 + lane;
+    bool keep = false;
+    if (p < p1) {
       const double mg = margin(p);
-      mine += mg > 0.0 ? 1 : 0;
+      keep = mg > 0.0;
       if (mg > my_best) {
         my_best = mg;
         my_idx = p;
       }
     }
+    wcount += __popc(__ballot_sync(0xffffffffu, keep));
   }
-  int carry;
-  {
-    int pos = block_exclusive_scan(mine, scan_scratch, &carry);
-    if (mine > 0)
-      for (int j = 0; j < R; ++j) {
-        const int p = tid * R + j;
-        if (p < P && margin(p) > 0.0) {
-          if (pos < cap) out[pos] = p;
-          ++pos;
-        }
-      }
+  if (lane == 0) scan_scratch[warp] = wcount;
+  __syncthreads();
+  int before = 0, carry = 0;
+  for (int w = 0; w < kWarps; ++w) {
+    before += w < warp ? scan_scratch[w] : 0;
+    carry += scan_scratch[w];
+  }
+  if (wcount > 0) {
+    int pos = before;
+    for (int q0 = p0; q0 < p1; q0 += 32) {
+      const int p = q0 + lane;
+      const bool keep = p < p1 && margin(p) > 0.0;
+      const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+      const int at = pos + __popc(bal & ((1u << lane) - 1u));
+      if (keep && at < cap) out[at] = p;
+      pos += __popc(bal);
+    }
   }
   if (carry > 0) {
     if (tid == 0) {
@@ -262,7 +313,6 @@ __global__ void __launch_bounds__(kGaussThreads)
     return;
   }
   // fallback: the single page with the largest margin, lowest index on ties
-  const int lane = tid & 31, warp = tid >> 5;
   for (int o = 16; o > 0; o >>= 1) {
     const double om = __shfl_xor_sync(0xffffffffu, my_best, o);
     const int oi = __shfl_xor_sync(0xffffffffu, my_idx, o);
