@@ -44,10 +44,10 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture
 # of the clustered 128k shape, keyed by a hash of the kernel's sources (a
 # changed kernel has no measured traffic until it is captured again)
-SCORE_FILES = ("score.cu", "common.cuh", "kernels.cuh")
-DECODE_FILES = ("decode_split.cu", "decode.cuh", "common.cuh", "kernels.cuh")
-SCORE_TRAFFIC = {"d0d585139e2ad614": 137794048}
-DECODE_TRAFFIC = {}
+SCORE_FILES = ("score.cu", "common.cuh")
+DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh")
+SCORE_TRAFFIC = {}
+DECODE_TRAFFIC = {"851e2059314083b4": 35284480}
 
 
 def kernel_hash(files=SCORE_FILES):

@@ -223,6 +223,28 @@ EKV_API ekv_status ekv_exactness_certificate(const ekv_seqs* seqs, int32_t num_k
                                              const int32_t* n_sel, int32_t cap, const float* tau,
                                              int32_t* certified, void* stream);
 
+/*
+ * ekv_decode_adaptive — the top-k decode with a budget that grows until the
+ * output is provably the full-cache one ([EKV] §3 "Récupération du Support",
+ * through ekv_exactness_certificate): page scores once, then for
+ * k = k0, 2·k0, 4·k0, … (at most max_pages) the top-k selection, the sparse
+ * decode and the certificate of every query head; the first k at which every
+ * head of every unit is certified (or every page is selected) ends it.  The
+ * count of uncertified heads is kept on the device and read back once per
+ * round, so the call synchronises `stream` once per round.  Outputs are those
+ * of the last round: sel device [batch, Hkv, k] (row stride k = *k_used; the
+ * buffer must hold batch·Hkv·max_pages entries), n_sel [batch, Hkv], out
+ * fp32 [batch, Hq, d], tau fp32 [batch, Hq], certified int32 [batch, Hq]
+ * (all 1: a selection of every page is certified too); k_used: host int.  scale and
+ * alpha as ekv_entmax_decode.  ws: ekv_workspace_bytes(
+ * EKV_OP_DECODE_ADAPTIVE, ...) bytes (cap ignored).
+ */
+EKV_API ekv_status ekv_decode_adaptive(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                       int32_t num_q_heads, float scale, float alpha, int32_t k0,
+                                       int32_t* sel, int32_t* n_sel, float* out, float* tau,
+                                       int32_t* certified, int32_t* k_used, void* ws, size_t ws_bytes,
+                                       void* stream);
+
 /* Bytes of the library-owned scratch array of ekv_entmax_decode_static_ws. */
 #define EKV_STATIC_WS_BYTES (16u << 20)
 
@@ -236,12 +258,19 @@ EKV_API ekv_status ekv_exactness_certificate(const ekv_seqs* seqs, int32_t num_k
  * of EKV_STATIC_WS_BYTES bytes that every GPU loading the library holds until
  * the process exits.  A configuration whose scratch
  * (ekv_workspace_bytes(EKV_OP_ENTMAX_DECODE, ...)) exceeds that size returns
- * EKV_ERR_WORKSPACE before any device work.  All calls on a device share the
- * array: calls that overlap on the GPU race, so serialise them.  The array
- * keeps the previous call's contents; the only part that must start at zero
- * (the split counters) is reset by the call itself.  The first call on a
- * device looks up the array's device address, so make it before any stream
- * capture.  Allocates nothing.
+ * EKV_ERR_WORKSPACE before any device work (the limit is checked against
+ * the scratch of every decode path, although the one-cluster-per-unit path,
+ * taken for few units, keeps its scratch in shared memory and reads none of
+ * the array; the many-unit and fp32 paths keep their scores, maxima, page
+ * ids and split counters there).  All calls on a device share the array:
+ * calls that overlap on the GPU race, so serialise them.  The array keeps
+ * the previous call's contents; the only part that must start at zero (the
+ * split counters) is reset by the call itself.  The call looks up the
+ * array's device address with the device current: on the first call on a
+ * device, and again on every call made outside a stream capture (so a
+ * cudaDeviceReset, after which the address may change, is followed); a call
+ * inside a capture uses the address found before, so make one call on each
+ * device before capturing.  Allocates nothing.
  */
 EKV_API ekv_status ekv_entmax_decode_static_ws(const ekv_cache* cache, const ekv_seqs* seqs,
                                                const void* q, int32_t num_q_heads, float scale,
@@ -283,7 +312,8 @@ typedef enum {
   EKV_OP_ENTMAX_DECODE = 2,
   EKV_OP_DECODE_STEP = 3,
   EKV_OP_SOFTMAX_DECODE = 4,
-  EKV_OP_SELECT_TOPK = 5
+  EKV_OP_SELECT_TOPK = 5,
+  EKV_OP_DECODE_ADAPTIVE = 6
 } ekv_op;
 
 /*

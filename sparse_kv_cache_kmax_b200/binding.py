@@ -22,12 +22,14 @@ __all__ = [
     "ekv_decode_step", "ekv_workspace_bytes", "ekv_get_error", "ekv_status_string",
     "ekv_entmax_decode_static_ws", "ekv_step_kernel_count", "ekv_softmax_decode", "EKV_OP_SOFTMAX_DECODE",
     "ekv_exactness_certificate", "EKV_OP_SELECT_TOPK", "ekv_selftest_wait_timeout", "EKV_EFLAG_TIMEOUT",
+    "ekv_decode_adaptive", "EKV_OP_DECODE_ADAPTIVE",
 ]
 
 EKV_F32, EKV_BF16 = 0, 1
 EKV_POLICY_TOPK, EKV_POLICY_GAUSS, EKV_POLICY_FULL = 0, 1, 2
 EKV_OP_SELECT_GAUSS, EKV_OP_ENTMAX_DECODE, EKV_OP_DECODE_STEP, EKV_OP_SOFTMAX_DECODE = 1, 2, 3, 4
 EKV_OP_SELECT_TOPK = 5
+EKV_OP_DECODE_ADAPTIVE = 6
 EKV_EFLAG_BAD_PAGE, EKV_EFLAG_BAD_LEN, EKV_EFLAG_SEL_OVERFLOW, EKV_EFLAG_BAD_SEL = 1, 2, 4, 8
 EKV_EFLAG_TIMEOUT = 16
 
@@ -82,6 +84,8 @@ _SIGS = {
     "ekv_softmax_decode": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _P, _P, _I, _P, _P,
                            _P, _SZ, _P],
     "ekv_exactness_certificate": [ctypes.POINTER(Seqs), _I, _I, _I, _F, _P, _P, _P, _I, _P, _P, _P],
+    "ekv_decode_adaptive": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _I, _P, _P, _P, _P, _P,
+                            ctypes.POINTER(ctypes.c_int32), _P, _SZ, _P],
     "ekv_selftest_wait_timeout": [ctypes.c_uint32, _P],
     "ekv_step_kernel_count": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), ctypes.POINTER(StepParams), _I],
     "ekv_entmax_decode_static_ws": [ctypes.POINTER(Cache), ctypes.POINTER(Seqs), _P, _I, _F, _F, _P,
@@ -232,6 +236,17 @@ def ekv_exactness_certificate(seqs, num_kv_heads, page_size, alpha, ub, sel, n_s
     _check("ekv_exactness_certificate", lib().ekv_exactness_certificate(
         ctypes.byref(seqs), num_kv_heads, page_size, tau.shape[1], alpha, _ptr(ub), _ptr(sel), _ptr(n_sel),
         sel.shape[-1], _ptr(tau), _ptr(certified), _stream(stream)))
+
+
+def ekv_decode_adaptive(cache, seqs, q, scale, alpha, k0, sel, n_sel, out, tau, certified, ws, stream=None) -> int:
+    """Top-k decode whose budget doubles from k0 until every head is certified
+    exact; returns the final k (sel then holds [batch, Hkv, k])."""
+    k_used = ctypes.c_int32(0)
+    _check("ekv_decode_adaptive", lib().ekv_decode_adaptive(
+        ctypes.byref(cache), ctypes.byref(seqs), _ptr(q), q.shape[1], scale, alpha, int(k0), _ptr(sel), _ptr(n_sel),
+        _ptr(out), _ptr(tau), _ptr(certified), ctypes.byref(k_used), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+    return int(k_used.value)
 
 
 def ekv_selftest_wait_timeout(polls=1024, stream=None):

@@ -114,6 +114,15 @@ DecodeWs carve_decode(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq,
   return w;
 }
 
+// Scratch of ekv_decode_adaptive: page scores, a count, the decode's scratch
+// for every page, and the top-k scratch for any budget.
+size_t adaptive_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq) {
+  const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
+  return a256(U * static_cast<size_t>(s->max_pages) * sizeof(float)) + a256(sizeof(int32_t)) +
+         decode_ws_bytes(c, s, Hq, s->max_pages) +
+         a256(topk_ws_bytes_upto(static_cast<int>(U), s->max_pages, s->max_pages));
+}
+
 size_t step_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq, int cap) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   return a256(U * static_cast<size_t>(s->max_pages) * sizeof(float)) + gauss_ws_bytes(c, s, Hq) +
@@ -246,6 +255,52 @@ EKV_API ekv_status ekv_exactness_certificate(const ekv_seqs* seqs, int32_t num_k
                                         cap, tau, certified, static_cast<cudaStream_t>(stream)));
 }
 
+EKV_API ekv_status ekv_decode_adaptive(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
+                                       int32_t num_q_heads, float scale, float alpha, int32_t k0,
+                                       int32_t* sel, int32_t* n_sel, float* out, float* tau,
+                                       int32_t* certified, int32_t* k_used, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  EKV_TRY(validate_decode(cache, seqs, q, num_q_heads, 1.0f, alpha, sel, n_sel, seqs ? seqs->max_pages : 1, out));
+  EKV_TRY(check_cache(cache, true, true));
+  if (!finite_pos(scale) || sel == nullptr || tau == nullptr || certified == nullptr || k_used == nullptr || k0 < 1)
+    return EKV_ERR_INVALID_ARG;
+  if (!certificate_smem_ok(seqs->max_pages)) return EKV_ERR_UNSUPPORTED;
+  EKV_TRY(check_ws(ws, ws_bytes, adaptive_ws_bytes(cache, seqs, num_q_heads)));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t U = static_cast<size_t>(seqs->batch) * cache->num_kv_heads;
+  const int P = seqs->max_pages;
+  Carver cv{static_cast<char*>(ws)};
+  float* ub = cv.take<float>(U * static_cast<size_t>(P));
+  int32_t* count = cv.take<int32_t>(1);
+  const DecodeWs dw = carve_decode(cv, cache, seqs, num_q_heads, P);
+  void* tws = cv.base + cv.used;
+  EKV_TRY(cuda_status(launch_score(*cache, *seqs, q, num_q_heads, scale, ub, st)));
+  int k = k0 < P ? k0 : P;
+  for (;;) {
+    // sel holds [batch, Hkv, k] at this round's k
+    const size_t tk = topk_ws_bytes(static_cast<int>(U), P, k);
+    EKV_TRY(cuda_status(launch_topk(*seqs, cache->num_kv_heads, cache->page_size, ub, k, k, sel, n_sel,
+                                    tk > 0 ? tws : nullptr, st)));
+    Carver cv2{static_cast<char*>(ws)};
+    cv2.take<float>(U * static_cast<size_t>(P));
+    cv2.take<int32_t>(1);
+    const DecodeWs dk = carve_decode(cv2, cache, seqs, num_q_heads, k);
+    EKV_TRY(cuda_status(launch_decode(*cache, *seqs, q, num_q_heads, scale, alpha, sel, n_sel, k, 0, out, tau,
+                                      nullptr, nullptr, dk, st)));
+    EKV_TRY(cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), st)));
+    EKV_TRY(cuda_status(launch_certificate(*seqs, cache->num_kv_heads, cache->page_size, num_q_heads, alpha, ub,
+                                           sel, n_sel, k, tau, certified, st, count)));
+    int32_t left = 0;
+    EKV_TRY(cuda_status(cudaMemcpyAsync(&left, count, sizeof(int32_t), cudaMemcpyDeviceToHost, st)));
+    EKV_TRY(cuda_status(cudaStreamSynchronize(st)));
+    if (left == 0 || k >= P) break;
+    k = 2 * k < P ? 2 * k : P;
+  }
+  (void)dw;
+  *k_used = k;
+  return EKV_OK;
+}
+
 EKV_API ekv_status ekv_softmax_decode(const ekv_cache* cache, const ekv_seqs* seqs, const void* q,
                                       int32_t num_q_heads, float scale, const int32_t* sel,
                                       const int32_t* n_sel, int32_t cap, float* out, float* lse,
@@ -326,6 +381,8 @@ EKV_API size_t ekv_workspace_bytes(int32_t op, const ekv_cache* cache, const ekv
       return cap < 1 ? 0 : step_ws_bytes(cache, seqs, num_q_heads, cap);
     case EKV_OP_SELECT_TOPK:
       return cap < 1 ? 0 : topk_ws_bytes(seqs->batch * cache->num_kv_heads, seqs->max_pages, cap);
+    case EKV_OP_DECODE_ADAPTIVE:
+      return adaptive_ws_bytes(cache, seqs, num_q_heads);
     case EKV_OP_SOFTMAX_DECODE:
       return cap < 1 ? 0 : softmax_ws_bytes(seqs->batch * cache->num_kv_heads, num_q_heads,
                                             cache->num_kv_heads, cache->head_dim, cap);

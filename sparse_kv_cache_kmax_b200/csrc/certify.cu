@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(kCertThreads)
     certificate_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
                        int max_pages, int Hkv, int G, int Hq, const int32_t* __restrict__ sel,
                        const int32_t* __restrict__ n_sel, int cap, const float* __restrict__ tau,
-                       float am1, int32_t* __restrict__ cert) {
+                       float am1, int32_t* __restrict__ cert, int32_t* __restrict__ uncertified) {
   grid_dep_enter();
   extern __shared__ unsigned int selmask[];  // [⌈max_pages/32⌉]
   __shared__ float scratch[32];
@@ -47,7 +47,9 @@ __global__ void __launch_bounds__(kCertThreads)
     const float t = tau[orow];
     // nothing unselected can hold support; a head with no support in the
     // selection (τ = +inf) is exact only if nothing is left unselected
-    cert[orow] = (m == -INFINITY || (t < INFINITY && am1 * m <= t)) ? 1 : 0;
+    const int ok = (m == -INFINITY || (t < INFINITY && am1 * m <= t)) ? 1 : 0;
+    cert[orow] = ok;
+    if (!ok && uncertified) atomicAdd(uncertified, 1);
   }
 }
 
@@ -72,11 +74,11 @@ int certificate_smem_ok(int max_pages) { return (max_pages + 31) / 32 * 4 <= 48 
 
 cudaError_t launch_certificate(const ekv_seqs& s, int Hkv, int S, int Hq, float alpha, const float* ub,
                                const int32_t* sel, const int32_t* n_sel, int cap, const float* tau,
-                               int32_t* cert, cudaStream_t st) {
+                               int32_t* cert, cudaStream_t st, int32_t* uncertified) {
   const size_t smem = static_cast<size_t>((s.max_pages + 31) / 32) * sizeof(unsigned int);
   const cudaError_t e = launch_k(certificate_kernel, dim3(s.batch * Hkv), dim3(kCertThreads), smem, st, ub,
                                  s.seq_lens, S, s.max_pages, Hkv, Hq / Hkv, Hq, sel, n_sel, cap, tau,
-                                 alpha - 1.0f, cert);
+                                 alpha - 1.0f, cert, uncertified);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -11,20 +11,17 @@
 //     bulk async copies (one copy = one contiguous S×d K tile) and scores
 //     them on tensor cores (m16n8k16, rows of the tile loaded from shared
 //     memory straight into A fragments).  Scores z and page maxima stay in
-//     shared memory.  The CTA then pushes its per-head maxima to every CTA
-//     and, after the barrier, starts bulk copies of the V tiles of the pages
-//     that can hold support (a page maximum within 1 of the unit's maximum,
-//     in u = (α−1)·z units: τ ≥ max u − 1).
+//     shared memory.  The CTA then pushes its per-head maxima to every CTA.
 //  2. τ: query head h is solved by CTA h mod C on the head's scores of the
 //     whole unit, gathered from the cluster's shared memory (DSMEM) in token
 //     order: Σ[u − τ]_+^β = 1, β = 1/(α−1) (see cta_solve_tau).  The solver
 //     writes the head's support bits and count and sends τ to every CTA.
-//  3. V: each CTA lists the pages of its run holding a support token (some
-//     head's page maximum above τ) and its warps read only those V tiles,
-//     from shared memory when staged, else from global memory; p = [u − τ]^β
-//     comes from the scores in shared memory.  CTA r owns a 1/C slice of the
-//     unit's G×d outputs: every CTA pushes its partial of that slice to CTA
-//     r, which sums the C partials in rank order.
+//  3. V: each CTA lists the support tokens of its run (some head has
+//     u > τ) and reads only their V rows from global memory, eight rows in
+//     flight per warp; p = [u − τ]^β comes from the scores in shared memory.
+//     CTA r owns a 1/C slice of the unit's G×d outputs: every CTA pushes its
+//     partial of that slice to CTA r, which sums the C partials in rank
+//     order.
 // Every sum has a fixed order, so results are deterministic.
 #include <cooperative_groups.h>
 
@@ -43,7 +40,6 @@ constexpr int kFWarps = 16;
 constexpr int kFThreads = 32 * kFWarps;
 constexpr int kFMaxCluster = 16;
 constexpr int kFMaxSpw = 8;       // K ring slots per warp
-constexpr int kFMaxVSlots = 64;   // staged V tiles per CTA
 constexpr int kFMaxHeads = 16;    // query heads per KV head (G)
 constexpr int kTauBinsF = 256;
 constexpr int kPairwiseMax = 256; // candidates for the pairwise support test
@@ -56,8 +52,7 @@ struct FusedGeom {
   int tile_bytes; // bytes of one S×d K or V tile
   int chunk;      // outputs owned per CTA: ceil(G·d / C)
   int off_ints, off_pm, off_zs, off_inbox, off_ring;  // byte offsets in dynamic shared memory
-  int off_v;      // V staging area, from the start of the ring
-  int nvslots;    // staged V tiles
+  int off_v;      // bytes of the ring the τ scratch, the V token list and the partials need
   int smem;       // dynamic shared memory bytes
 };
 
@@ -378,11 +373,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   constexpr int KP = D / 32, NT = (G + 7) / 8, DPL = D / 32;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint64_t bars[kFWarps * kFMaxSpw];
-  __shared__ uint64_t vbars[kFMaxVSlots];
   __shared__ TauShared tsh;
   __shared__ float s_tau[G];
   __shared__ float mall[kFMaxHeads][kFMaxCluster];  // run maxima: [head][CTA rank]
-  __shared__ int s_vcount;
   __shared__ int scan_scratch[32];
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -393,19 +386,14 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   const int S = a.S, spc = f.spc, zp = f.zpitch, spw = f.spw;
   int* phys_s = reinterpret_cast<int*>(smem + f.off_ints);  // [spc]
   int* nv_s = phys_s + spc;                                  // [spc]
-  int* list_s = nv_s + spc;                                  // [spc]
-  int* vslot_s = list_s + spc;                               // [spc] staged V slot or −1
   float* pm = reinterpret_cast<float*>(smem + f.off_pm);     // [G][spc] page maxima of z
   float* zs = reinterpret_cast<float*>(smem + f.off_zs);     // [G][zpitch] scores z
   float* inbox = reinterpret_cast<float*>(smem + f.off_inbox);  // [C][chunk] partial outputs
   unsigned char* ring = smem + f.off_ring;
-  unsigned char* vtiles = ring + f.off_v;
 
   if (tid == 0) {
     for (int s = 0; s < kFWarps * spw; ++s) mbar_init(&bars[s], 1);
-    for (int s = 0; s < f.nvslots; ++s) mbar_init(&vbars[s], 1);
     fence_mbar_init();
-    s_vcount = 0;
   }
   for (int i = tid; i < kTauBinsF; i += kFThreads) tsh.hist[i] = 0;
   __syncthreads();
@@ -510,68 +498,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   }
   cluster.sync();
 
-  // V tiles of the pages that can hold support start moving into shared
-  // memory: τ ≥ max u − 1 over the unit, so a page whose maximum is not above
-  // that for some head holds no support.  When the candidates outnumber the
-  // slots, the slots go to the pages nearest their head's maximum (ties to
-  // the lower page), where the support lies.
-  {
-    float top[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float m = -INFINITY;
-      for (int r = 0; r < C; ++r) m = fmaxf(m, mall[h][r]);
-      top[h] = a.am1 * m;
-    }
-    float* dist = reinterpret_cast<float*>(list_s);  // [np], until the V list reuses it
-    int ncand = 0;
-    for (int j0 = 0; j0 < np; j0 += kFThreads) {
-      const int j = j0 + tid;
-      float d = -INFINITY;
-      if (j < np && phys_s[j] >= 0) {
-        if (a.dense_v) {
-          d = 0.f;
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pz = pm[h * spc + j];
-            if (pz > -INFINITY) d = fmaxf(d, a.am1 * pz - top[h]);
-          }
-          if (!(d > -1.0f)) d = -INFINITY;
-        }
-      }
-      if (j < np) dist[j] = d;
-      ncand += __syncthreads_count(d > -INFINITY);
-    }
-    const bool ranked = ncand > f.nvslots;
-    if (ranked && tid == 0) s_vcount = ncand;
-    for (int j = tid; j < np; j += kFThreads) {
-      const float d = dist[j];
-      int vs = -1;
-      if (d > -INFINITY) {
-        int slot;
-        if (ranked) {
-          slot = 0;
-          for (int i = 0; i < np; ++i) {
-            const float di = dist[i];
-            slot += (di > d || (di == d && i < j)) ? 1 : 0;
-          }
-        } else {
-          slot = atomicAdd(&s_vcount, 1);
-        }
-        if (slot < f.nvslots) {
-          vs = slot;
-          fence_proxy_async_smem();  // K tiles read from this area come before the copy
-          mbar_arrive_expect_tx(&vbars[vs], static_cast<unsigned int>(f.tile_bytes));
-          bulk_g2s(vtiles + static_cast<size_t>(vs) * f.tile_bytes,
-                   static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * tile_elems,
-                   static_cast<unsigned int>(f.tile_bytes), &vbars[vs]);
-        }
-      }
-      vslot_s[j] = vs;
-    }
-  }
-
   // ---------------------------------------------------------------- 2. τ
   const int tpc = spc * S;
   const int n_tok = n_slots * S;
@@ -623,87 +549,80 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   cluster.sync();
 
   // ---------------------------------------------------------------- 3. V
-  int nsup = 0;
-  for (int w0 = 0; w0 < np; w0 += kFThreads) {
-    const int j = w0 + tid;
+  // The run's support tokens (some head has u > τ; every valid token with
+  // dense_v), listed in token order over the free ring, then read row by row:
+  // warp w takes rows w·8 … w·8+7 of each block of 128, eight V rows in
+  // flight per warp, p = [u − τ]_+^β from the scores in shared memory.
+  int* tl = reinterpret_cast<int*>(ring);  // [np·S] token j·S + t of the run
+  int ntl = 0;
+  for (int x0 = 0; x0 < np * S; x0 += kFThreads) {
+    const int x = x0 + tid;
     int sup = 0;
-    if (j < np && phys_s[j] >= 0) {
-      if (a.dense_v) {
-        sup = 1;
-      } else {
+    if (x < np * S) {
+      const int j = x / S;
+      if (phys_s[j] >= 0 && x - j * S < nv_s[j]) {
+        if (a.dense_v) {
+          sup = 1;
+        } else {
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          if (a.am1 * pm[h * spc + j] > s_tau[h]) sup = 1;
+          for (int h = 0; h < G; ++h)
+            if (a.am1 * zs[h * zp + x] > s_tau[h]) sup = 1;
+        }
       }
     }
     int tot;
     const int pos = block_exclusive_scan(sup, scan_scratch, &tot);
-    if (sup) list_s[nsup + pos] = j;
-    nsup += tot;
+    if (sup) tl[ntl + pos] = x;
+    ntl += tot;
   }
   __syncthreads();
-
-  // Warps take whole support pages (page e goes to warp e mod 16).  Lane t
-  // computes p = [u − τ]_+^β of the page's token t for every head once; the
-  // row loop broadcasts them by shuffle and reads the V rows (staged in
-  // shared memory, else global), four at a time.
   float acc[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+  constexpr int kRowsInFlight = 8;
 #pragma unroll 1
-  for (int e = warp; e < nsup; e += kFWarps) {
-    const int j = list_s[e], nvv = nv_s[j], vs = vslot_s[j];
-    const bf16* vbase;
-    if (vs >= 0) {
-      if (!mbar_wait(&vbars[vs], 0u)) mbar_wait(&vbars[vs], 0u);
-      vbase = reinterpret_cast<const bf16*>(vtiles + static_cast<size_t>(vs) * f.tile_bytes);
-    } else {
-      vbase = static_cast<const bf16*>(a.v_pool) + (static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * tile_elems;
-    }
-#pragma unroll 1
-    for (int t0 = 0; t0 < nvv; t0 += 32) {
-      float p[G];
+  for (int e0 = warp * kRowsInFlight; e0 < ntl; e0 += kFWarps * kRowsInFlight) {
+    float v[kRowsInFlight][DPL];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        p[h] = 0.f;
-        if (t0 + lane < nvv) {
-          const float w = a.am1 * zs[h * zp + j * S + t0 + lane] - s_tau[h];
-          if (w > 0.f) p[h] = pow_beta_fast(w, a.beta, a.ipow);
-        }
-      }
-      const int nr = min(32, nvv - t0);
-#pragma unroll 4
-      for (int r = 0; r < nr; ++r) {
-        float v[DPL];
-        const bf16* src = vbase + static_cast<size_t>(t0 + r) * D + lane * DPL;
+    for (int r = 0; r < kRowsInFlight; ++r) {
+      const int e = e0 + r;
+#pragma unroll
+      for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
+      if (e < ntl) {
+        const int tok = tl[e], j = tok / S;
+        const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                          ((static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * S + (tok - j * S)) * D + lane * DPL;
         if constexpr (DPL == 4) {
           const uint2 w = *reinterpret_cast<const uint2*>(src);
-          v[0] = __uint_as_float(w.x << 16);
-          v[1] = __uint_as_float(w.x & 0xffff0000u);
-          v[2] = __uint_as_float(w.y << 16);
-          v[3] = __uint_as_float(w.y & 0xffff0000u);
+          v[r][0] = __uint_as_float(w.x << 16);
+          v[r][1] = __uint_as_float(w.x & 0xffff0000u);
+          v[r][2] = __uint_as_float(w.y << 16);
+          v[r][3] = __uint_as_float(w.y & 0xffff0000u);
         } else {
           const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
-          v[0] = __uint_as_float(w << 16);
-          v[1] = __uint_as_float(w & 0xffff0000u);
+          v[r][0] = __uint_as_float(w << 16);
+          v[r][1] = __uint_as_float(w & 0xffff0000u);
         }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsInFlight; ++r) {
+      const int e = e0 + r;
+      if (e < ntl) {
+        const int tok = tl[e];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float pt = __shfl_sync(0xffffffffu, p[h], r);
+          const float w = a.am1 * zs[h * zp + tok] - s_tau[h];
+          const float pt = w > 0.f ? pow_beta_fast(w, a.beta, a.ipow) : 0.f;
 #pragma unroll
-          for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(pt, v[e2], acc[h][e2]);
+          for (int x = 0; x < DPL; ++x) acc[h][x] = fmaf(pt, v[r][x], acc[h][x]);
         }
       }
     }
   }
-  // every staged copy has landed before its area is reused or the CTA exits
-  {
-    const int issued = min(s_vcount, f.nvslots);
-    for (int s = tid; s < issued; s += kFThreads)
-      if (!mbar_wait(&vbars[s], 0u)) mbar_wait(&vbars[s], 0u);
-  }
+  __syncthreads();  // the token list is read by every warp before the partials overwrite it
   // warp partials → CTA partial (warp order) → the owner's inbox
   float* red = reinterpret_cast<float*>(ring);  // [kFWarps][G][D], over the finished τ scratch
 #pragma unroll
@@ -784,13 +703,8 @@ FusedGeom plan(int C, int cap, int S, int smem_limit) {
   if (spw < 1) return FusedGeom{};
   f.spw = spw;
   const int ring_k = kFWarps * spw * f.tile_bytes;
-  int ring = std::max(ring_k, f.off_v);
-  // staged V tiles in what is left, up to one per page of the run
-  const int want = std::min(kFMaxVSlots, f.spc);
-  const int room = std::min(avail, f.off_v + want * f.tile_bytes);
-  ring = std::max(ring, room);
+  const int ring = std::max(ring_k, f.off_v);
   if (off + ring > smem_limit) return FusedGeom{};
-  f.nvslots = std::max(0, std::min(want, (ring - f.off_v) / f.tile_bytes));
   f.smem = off + ring;
   return f;
 }

@@ -63,9 +63,10 @@ int sm_count();
 
 // Exactness certificate per query head (certify.cu).
 int certificate_smem_ok(int max_pages);
+// uncertified (nullable): a device int the kernel adds the uncertified heads to.
 cudaError_t launch_certificate(const ekv_seqs& s, int Hkv, int S, int Hq, float alpha, const float* ub,
                                const int32_t* sel, const int32_t* n_sel, int cap, const float* tau,
-                               int32_t* cert, cudaStream_t st);
+                               int32_t* cert, cudaStream_t st, int32_t* uncertified = nullptr);
 
 // Softmax decode split over pages (softmax.cu).
 int softmax_splits(int units, int cap);

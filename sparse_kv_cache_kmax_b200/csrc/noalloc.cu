@@ -17,9 +17,12 @@
 //  * the array keeps whatever the previous call left in it.  The only scratch
 //    that must start at zero is the per-unit split counter, and the first
 //    decode kernel of every call sets it to zero;
-//  * the first call on a device looks up the array's device address (host
-//    code only sees a host-side stand-in for it), so make that first call
-//    before any stream capture.
+//  * host code only sees a host-side stand-in for the array: the call looks
+//    up its device address with the device current, the first time on a
+//    device and again whenever it is made outside a stream capture (so a
+//    cudaDeviceReset, which reloads the module, is followed correctly); a
+//    call inside a capture uses the address found before, so make one call
+//    on each device before capturing.
 #include <mutex>
 
 #include "kernels.cuh"
@@ -34,14 +37,22 @@ __device__ __align__(256) unsigned char g_static_decode_ws[EKV_STATIC_WS_BYTES];
 std::mutex g_ws_mutex;
 void* g_ws_addr[kMaxDevices] = {};
 
-// Device address of the array on the current device (set up once per device).
-cudaError_t static_ws_address(void** out) {
+// Device address of the array on the current device.  Looked up with the
+// device current on the first call, and again on every call made outside a
+// stream capture (a cudaDeviceReset reloads the module, which may move the
+// array); inside a capture the address found before is used, since the
+// lookup is not a call to make while capturing.
+cudaError_t static_ws_address(cudaStream_t stream, void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_ws_mutex);
-  if (g_ws_addr[dev] == nullptr) {
+  if (g_ws_addr[dev] == nullptr || cap == cudaStreamCaptureStatusNone) {
+    if (cap != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_decode_ws);
     if (e != cudaSuccess) return e;
@@ -64,7 +75,7 @@ extern "C" EKV_API ekv_status ekv_entmax_decode_static_ws(
                              out, tau, support_count, support_bits, nullptr, 0, stream);
   if (need > static_cast<size_t>(EKV_STATIC_WS_BYTES)) return EKV_ERR_WORKSPACE;
   void* ws = nullptr;
-  if (ekv::static_ws_address(&ws) != cudaSuccess) return EKV_ERR_CUDA;
+  if (ekv::static_ws_address(static_cast<cudaStream_t>(stream), &ws) != cudaSuccess) return EKV_ERR_CUDA;
   return ekv_entmax_decode(cache, seqs, q, num_q_heads, scale, alpha, sel, n_sel, cap, dense_v, out,
                            tau, support_count, support_bits, ws, EKV_STATIC_WS_BYTES, stream);
 }

@@ -59,15 +59,14 @@ class DecodeEngine:
 
     def decode_adaptive(self, q, k_new=None, v_new=None, k0=None, stream=None):
         """Top-k decode whose budget doubles until every query head is
-        certified exact (ekv_exactness_certificate: no unselected page can
+        certified exact (one ekv_decode_adaptive call: no unselected page can
         hold support, so the output is the full-cache one).  Appends first
         when k_new is given.  Returns (out [B, Hq, d], k used)."""
         Bsz, Hkv, P = self.batch, self.Hkv, self.max_pages
         dev = self.device
         if not hasattr(self, "_ad"):
-            ws = B.workspace(B.ekv_workspace_bytes(B.EKV_OP_ENTMAX_DECODE, self.cache, self.seqs, self.Hq, P), dev)
-            self._ad = dict(ub=torch.empty(Bsz, Hkv, P, device=dev),
-                            sel=torch.empty(Bsz * Hkv * P, dtype=torch.int32, device=dev),
+            ws = B.workspace(B.ekv_workspace_bytes(B.EKV_OP_DECODE_ADAPTIVE, self.cache, self.seqs, self.Hq, P), dev)
+            self._ad = dict(sel=torch.empty(Bsz * Hkv * P, dtype=torch.int32, device=dev),
                             n=torch.zeros(Bsz, Hkv, dtype=torch.int32, device=dev),
                             out=torch.zeros(Bsz, self.Hq, self.d, device=dev),
                             tau=torch.zeros(Bsz, self.Hq, device=dev),
@@ -75,19 +74,7 @@ class DecodeEngine:
         a = self._ad
         if k_new is not None:
             B.ekv_append(self.cache, self.seqs, k_new, v_new, stream)
-        scale, alpha = self.params.scale, self.params.alpha
-        B.ekv_score_pages(self.cache, self.seqs, q, scale, a["ub"], stream)
-        k = max(1, min(int(k0 or self.params.k or 1), P))
-        while True:
-            sel = a["sel"][: Bsz * Hkv * k].view(Bsz, Hkv, k)
-            if k not in a.setdefault("tk", {}):
-                n_tk = B.ekv_workspace_bytes(B.EKV_OP_SELECT_TOPK, self.cache, self.seqs, self.Hq, k)
-                a["tk"][k] = B.workspace(n_tk, dev) if n_tk else None
-            B.ekv_select_topk(self.seqs, Hkv, self.S, a["ub"], k, sel, a["n"], stream, ws=a["tk"][k])
-            B.ekv_entmax_decode(self.cache, self.seqs, q, scale, alpha, sel, a["n"], k, a["out"], a["ws"],
-                                tau=a["tau"], stream=stream)
-            B.ekv_exactness_certificate(self.seqs, Hkv, self.S, alpha, a["ub"], sel, a["n"], a["tau"], a["cert"],
-                                        stream=stream)
-            if k >= P or bool(a["cert"].all()):
-                return a["out"], k
-            k = min(2 * k, P)
+        k = B.ekv_decode_adaptive(self.cache, self.seqs, q, self.params.scale, self.params.alpha,
+                                  max(1, min(int(k0 or self.params.k or 1), P)), a["sel"], a["n"], a["out"],
+                                  a["tau"], a["cert"], a["ws"], stream)
+        return a["out"], k
