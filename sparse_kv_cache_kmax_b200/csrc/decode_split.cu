@@ -33,16 +33,17 @@ namespace {
 constexpr int kKsWarps = 8;
 constexpr int kKsThreads = 32 * kKsWarps;
 constexpr int kKsTokens = 32 * kKsWarps;   // selected tokens per CTA of the score launch
-constexpr int kHdThreads = 256;
-constexpr int kHdWarps = kHdThreads / 32;
+constexpr int kHdThreads = 256;           // per-head CTA when the scores sit in registers
+constexpr int kHdStreamThreads = 1024;    // per-head CTA when they are read from L2 at each pass
+constexpr int kHdMaxWarps = 32;
 constexpr int kHdBins = 256;
 constexpr int kHdCand = 2048;              // candidates / support tokens held in shared memory at once
 constexpr int kHdPairMax = 256;            // candidates for the all-at-once support test
 constexpr int kHdRows = 8;                 // V rows in flight per warp
 constexpr int kHdBatch = 8;                // score loads in flight per thread when streaming
 constexpr int kHdMaxVpt = 64;              // values per thread held in registers (more: read per pass)
-constexpr int kSplitMaxTokens = 65536;     // selected tokens per unit on this path
-static_assert(kHdBins == kHdThreads, "one histogram bin per thread");
+constexpr int kSplitMaxTokens = 1 << 20;   // selected tokens per unit on this path
+static_assert(kHdBins <= kHdThreads, "one histogram bin per thread");
 
 // ------------------------------------------------------------------ 1. K scores
 template <int D, int G>
@@ -150,14 +151,14 @@ struct HdShared {
   int hist[kHdBins];
   float cu[kHdCand];  // candidates above the bracket, then the support's weights
   int ci[kHdCand];    // their token indices
-  float f[kHdWarps];
-  double d[3][kHdWarps];
-  int i[kHdWarps];
+  float f[kHdMaxWarps];
+  double d[3][kHdMaxWarps];
+  int i[kHdMaxWarps];
 };
 
 // Sums of (x, y, z) over the CTA in a fixed order; every thread gets them.
 __device__ __forceinline__ void hd_sum3(double& x, double& y, double& z, HdShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   x = warp_sum(x);
   y = warp_sum(y);
   z = warp_sum(z);
@@ -169,8 +170,7 @@ __device__ __forceinline__ void hd_sum3(double& x, double& y, double& z, HdShare
   }
   __syncthreads();
   x = y = z = 0.0;
-#pragma unroll
-  for (int w = 0; w < kHdWarps; ++w) {
+  for (int w = 0; w < nw; ++w) {
     x += sh.d[0][w];
     y += sh.d[1][w];
     z += sh.d[2][w];
@@ -197,8 +197,9 @@ __device__ __forceinline__ V hd_pow_bm1(V w, V beta, int ipow) {
   }
 }
 
-template <int D, int VPT>
-__global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, int G) {
+template <int D, int VPT, int THREADS>
+__global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int G) {
+  constexpr int kHdWarps = THREADS / 32;
   constexpr int DPL = D / 32;
   __shared__ HdShared sh;
   __shared__ float red[kHdWarps][D];
@@ -217,12 +218,12 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   // value k of this thread is token i = k·256 + tid: held in registers
   // (VPT > 0), or read again from the scratch at every pass (VPT == 0)
   constexpr bool kReg = VPT > 0;
-  const int NK = kReg ? VPT : (n + kHdThreads - 1) / kHdThreads;
+  const int NK = kReg ? VPT : (n + THREADS - 1) / THREADS;
   float uv[kReg ? VPT : 1];
   if constexpr (kReg) {
 #pragma unroll
     for (int k = 0; k < (kReg ? VPT : NK); ++k) {
-      const int i = k * kHdThreads + tid;
+      const int i = k * THREADS + tid;
       uv[k] = i < n ? am1 * z[i] : -INFINITY;
     }
   }
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
         float v[kHdBatch];
 #pragma unroll
         for (int j = 0; j < kHdBatch; ++j) {
-          const int i = (k0 + j) * kHdThreads + tid;
+          const int i = (k0 + j) * THREADS + tid;
           v[j] = (k0 + j < NK && i < n) ? am1 * __ldcg(z + i) : -INFINITY;
         }
 #pragma unroll
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   float m = -INFINITY;
   for (int c = lane; c < nchunk; c += 32) m = fmaxf(m, a.ws.cmax[static_cast<size_t>(row) * a.ws.nqk + c]);
   m = warp_max(m);  // every warp reads them all: no barrier
-  sh.hist[tid] = 0;
+  if (tid < kHdBins) sh.hist[tid] = 0;
   __syncthreads();
 
   float tau = INFINITY;  // no finite score: no support, zero output
@@ -265,10 +266,10 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
     __syncthreads();
     float cb = um - 1.0f;
     {
-      const int h = sh.hist[tid];
+      const int h = tid < kHdBins ? sh.hist[tid] : 0;
       int total;
       const int c = block_exclusive_scan(h, sh.i, &total) + h;  // values in bins 0..tid
-      if (c > 0) {
+      if (tid < kHdBins && c > 0) {
         const float fc = static_cast<float>(c);
         const float inv = ipow == 1 ? 1.0f / fc : (ipow == 2 ? rsqrtf(fc) : exp2f(-__log2f(fc) / beta));
         cb = fmaxf(cb, um - static_cast<float>(tid + 1) / kHdBins - inv);
@@ -295,7 +296,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
         for_values([&](int k, float u) {
           if (u > tlo) {
             sh.cu[p] = u;
-            sh.ci[p] = k * kHdThreads + tid;
+            sh.ci[p] = k * THREADS + tid;
             ++p;
           }
         });
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
           }
         };
         if (listed) {
-          for (int j = tid; j < nc; j += kHdThreads) term(sh.cu[j]);
+          for (int j = tid; j < nc; j += THREADS) term(sh.cu[j]);
         } else {
           for_values([&](int, float u) { term(u); });
         }
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
             }
           };
           if (listed) {
-            for (int j = tid; j < nc; j += kHdThreads) add(sh.cu[j]);
+            for (int j = tid; j < nc; j += THREADS) add(sh.cu[j]);
           } else {
             for_values([&](int, float u) { add(u); });
           }
@@ -486,17 +487,17 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   //    it returns the support's size.
   if (a.bits_out)
     for_values([&](int k, float u) {
-      const int i = k * kHdThreads + tid;
+      const int i = k * THREADS + tid;
       const unsigned int bal = __ballot_sync(0xffffffffu, i < n && u > tau);
       if (lane == 0 && (i >> 5) < a.words) a.bits_out[orow * a.words + (i >> 5)] = bal;
     });
   auto compact = [&](int base) {
     int mine = 0;
-    for_values([&](int k, float u) { mine += (k * kHdThreads + tid < n && u > tau) ? 1 : 0; });
+    for_values([&](int k, float u) { mine += (k * THREADS + tid < n && u > tau) ? 1 : 0; });
     int ns;
     int p = block_exclusive_scan(mine, sh.i, &ns) - base;
     for_values([&](int k, float u) {
-      const int i = k * kHdThreads + tid;
+      const int i = k * THREADS + tid;
       if (i < n && u > tau) {
         if (p >= 0 && p < kHdCand) {
           sh.cu[p] = pow_beta_fast(u - tau, beta, ipow);
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
   };
   const int ns = compact(0);
   if (a.bits_out)
-    for (int w = ((kReg ? VPT : NK) * kHdThreads) / 32 + tid; w < a.words; w += kHdThreads)
+    for (int w = ((kReg ? VPT : NK) * THREADS) / 32 + tid; w < a.words; w += THREADS)
       a.bits_out[orow * a.words + w] = 0u;  // words past the ballots above
   if (tid == 0) {
     if (a.tau_out) a.tau_out[orow] = tau;
@@ -564,7 +565,7 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
 #pragma unroll
   for (int x = 0; x < DPL; ++x) red[warp][lane * DPL + x] = acc[x];
   __syncthreads();
-  for (int i = tid; i < D; i += kHdThreads) {
+  for (int i = tid; i < D; i += THREADS) {
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kHdWarps; ++w) s += red[w][i];
@@ -575,15 +576,16 @@ __global__ void __launch_bounds__(kHdThreads) head_decode_kernel(DecodeArgs a, i
 template <int D>
 cudaError_t launch_head_decode(DecodeArgs& a, int rows, int G, cudaStream_t st) {
   const int n_max = a.cap * a.S;
-#define EKV_HD_CASE(VV)                                                                                  \
-  if (n_max <= (VV) * kHdThreads) {                                                                      \
-    const cudaError_t e = launch_k(head_decode_kernel<D, VV>, dim3(rows), dim3(kHdThreads), 0, st, a, G); \
-    if (e != cudaSuccess) return e;                                                                      \
-    return cudaGetLastError();                                                                           \
+#define EKV_HD_CASE(VV)                                                                                      \
+  if (n_max <= (VV) * kHdThreads) {                                                                          \
+    const cudaError_t e = launch_k(head_decode_kernel<D, VV, kHdThreads>, dim3(rows), dim3(kHdThreads), 0, st, a, G); \
+    if (e != cudaSuccess) return e;                                                                          \
+    return cudaGetLastError();                                                                               \
   }
   EKV_HD_CASE(4) EKV_HD_CASE(16) EKV_HD_CASE(32) EKV_HD_CASE(kHdMaxVpt)
 #undef EKV_HD_CASE
-  const cudaError_t e = launch_k(head_decode_kernel<D, 0>, dim3(rows), dim3(kHdThreads), 0, st, a, G);
+  const cudaError_t e = launch_k(head_decode_kernel<D, 0, kHdStreamThreads>, dim3(rows), dim3(kHdStreamThreads), 0,
+                                 st, a, G);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

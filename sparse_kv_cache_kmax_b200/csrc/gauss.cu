@@ -24,7 +24,8 @@ namespace ekv {
 
 namespace {
 
-constexpr int kGaussThreads = 256;
+constexpr int kGaussThreads = 256;   // filter
+constexpr int kTauThreads = 1024;    // τ̂ solve: one CTA per query head, every thread on its pages
 constexpr int kGaussCand = 3072;
 constexpr float kPruneC = 6.0f;
 
@@ -76,7 +77,7 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
   dF += static_cast<double>(n) * beta * sb1 * static_cast<double>(jb1 > R(0) ? jb1 : R(0));
 }
 
-__global__ void __launch_bounds__(kGaussThreads)
+__global__ void __launch_bounds__(kTauThreads)
     gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
                      int Hkv, int G, int Hq, int beta, float* __restrict__ tau_out) {
   grid_dep_enter();
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kGaussThreads)
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
   __shared__ float c_mu[kGaussCand], c_sg[kGaussCand], c_n[kGaussCand];
   __shared__ float f_scratch[32];
-  __shared__ double d_scratch[32];
+  __shared__ double d_scratch[64];
   __shared__ int i_scratch[32];
 
   // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
@@ -120,11 +121,11 @@ __global__ void __launch_bounds__(kGaussThreads)
   bool cached = false;
   auto gather = [&](double t) {  // every thread calls it
     int mine = 0;
-    for (int p = tid; p < P; p += kGaussThreads) mine += live(p, t) ? 1 : 0;
+    for (int p = tid; p < P; p += kTauThreads) mine += live(p, t) ? 1 : 0;
     int pos = block_exclusive_scan(mine, i_scratch, &nc);
     cached = nc <= kGaussCand;
     if (cached)
-      for (int p = tid; p < P; p += kGaussThreads)
+      for (int p = tid; p < P; p += kTauThreads)
         if (live(p, t)) {
           c_mu[pos] = ws.mu[base + p];
           c_sg[pos] = ws.sig[base + p];
@@ -134,12 +135,12 @@ __global__ void __launch_bounds__(kGaussThreads)
     __syncthreads();
   };
   // cuts the cached list to the pages still above t, in place, order kept:
-  // thread t owns entries [t·R, t·R + R) (R ≤ 16), holds its survivors in
+  // thread t owns entries [t·R, t·R + R) (R ≤ 4), holds its survivors in
   // registers across one barrier, then writes them at their new places
   auto recut = [&](double t) {
-    constexpr int kMaxR = 16;
-    static_assert(kGaussCand <= kMaxR * kGaussThreads, "entries per thread");
-    const int R = (nc + kGaussThreads - 1) / kGaussThreads;
+    constexpr int kMaxR = 4;
+    static_assert(kGaussCand <= kMaxR * kTauThreads, "entries per thread");
+    const int R = (nc + kTauThreads - 1) / kTauThreads;
     float m[kMaxR], sgm[kMaxR], nn[kMaxR];
     unsigned int keep = 0u;
 #pragma unroll
@@ -197,14 +198,14 @@ __global__ void __launch_bounds__(kGaussThreads)
     __syncthreads();  // the previous evaluation's partials are read
     if (lane == 0) {
       d_scratch[warp] = F;
-      d_scratch[16 + warp] = dF;
+      d_scratch[32 + warp] = dF;
     }
     __syncthreads();
     F = 0.0;
     dF = 0.0;
-    for (int w = 0; w < kGaussThreads / 32; ++w) {
+    for (int w = 0; w < kTauThreads / 32; ++w) {
       F += d_scratch[w];
-      dF += d_scratch[16 + w];
+      dF += d_scratch[32 + w];
     }
   };
   // fp32 terms: a monotone approach from the left while the steps are large
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kGaussThreads)
     }
   }
   if (!cached) gather(tau);
-  for (int it = 0; it < 6; ++it) {    // float64 terms: quadratic convergence (either side)
+  for (int it = 0; it < 3; ++it) {    // float64 terms: quadratic convergence (either side)
     double F, dF;
     evaluate(tau, true, F, dF);
     if (!(dF > 0.0)) break;
@@ -352,7 +353,7 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
   const int Hkv = c.num_kv_heads, G = Hq / Hkv, U = s.batch * Hkv;
   const int beta = static_cast<int>(lrint(1.0 / (static_cast<double>(alpha) - 1.0)));
   {
-    const cudaError_t le_ = launch_k(gauss_tau_kernel, U * G, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
+    const cudaError_t le_ = launch_k(gauss_tau_kernel, U * G, kTauThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
                                                     G, Hq, beta, tau_hat);
     if (le_ != cudaSuccess) return le_;
   }

@@ -29,18 +29,22 @@ from gpu_helpers import (REL_TIE, assert_sel_matches, check_unit_decode, gen, np
 pytestmark = pytest.mark.gpu
 
 # (workload, policy, alpha, budget): the benchmark's headline line, its other
-# alphas and the Gaussian policy, and every other workload's own line
+# alphas, the Gaussian policy and the full-cache decode, and every other
+# workload's own line
 CASES = [
     ("clustered_128k", "topk", 1.5, 256),
     ("clustered_128k", "topk", 1.25, 256),
     ("clustered_128k", "topk", 2.0, 256),
     ("clustered_128k", "gauss", 1.5, 0.5),
+    ("clustered_128k", "full", 1.5, None),
     ("gqa_32k", "topk", 1.5, 64),
     ("short_scattered", "topk", 1.5, 32),
     ("long_512k", "topk", 1.5, 512),
     ("long_512k", "gauss", 1.5, 0.5),
+    ("long_512k", "full", 1.5, None),
     ("ctx_1m", "topk", 1.5, 512),
     ("ctx_1m", "gauss", 1.5, 0.5),
+    ("ctx_1m", "full", 1.5, None),
 ]
 
 _CACHE = {}
@@ -69,7 +73,8 @@ def test_fullsize_step_matches_oracle_on_sampled_units(name, policy, alpha, budg
     wl = inp["workload"]
     k = budget if policy == "topk" else None
     delta = budget if policy == "gauss" else None
-    cap = k if policy == "topk" else gauss_cap(wl, inp["max_pages"])
+    full = policy == "full"
+    cap = k if policy == "topk" else (inp["max_pages"] if full else gauss_cap(wl, inp["max_pages"]))
     eng = DecodeEngine(inp["k_pool"], inp["v_pool"], inp["page_table"], inp["seq_lens"], wl.num_q_heads,
                        policy=policy, k=k, delta=delta, alpha=alpha, cap=cap)
     eng.build_meta()
@@ -86,8 +91,8 @@ def test_fullsize_step_matches_oracle_on_sampled_units(name, policy, alpha, budg
     cnt = torch.full((wl.batch, Hq), -1, dtype=torch.int32, device="cuda")
     bits = torch.zeros(wl.batch, Hq, words, dtype=torch.int32, device="cuda")
     ws = B.workspace(B.ekv_workspace_bytes(B.EKV_OP_ENTMAX_DECODE, eng.cache, eng.seqs, Hq, cap), "cuda")
-    B.ekv_entmax_decode(eng.cache, eng.seqs, inp["q"], eng.params.scale, alpha, sel_all, n_all, cap, out_d, ws,
-                        tau=tau, support_count=cnt, support_bits=bits)
+    B.ekv_entmax_decode(eng.cache, eng.seqs, inp["q"], eng.params.scale, alpha, None if full else sel_all,
+                        None if full else n_all, cap, out_d, ws, tau=tau, support_count=cnt, support_bits=bits)
     torch.cuda.synchronize()
     assert torch.equal(out_d, out), "the step's decode and the standalone decode differ"
 
@@ -104,7 +109,7 @@ def test_fullsize_step_matches_oracle_on_sampled_units(name, policy, alpha, budg
                 want = O.select_topk(ub_h[b, h, :P], k)
                 assert int(n_h[b, h]) == min(k, P)
                 assert np.array_equal(sel_h[b, h, : n_h[b, h]], want), (b, h)
-    else:
+    elif policy == "gauss":
         tau_hat = torch.zeros(wl.batch, Hq, device="cuda")
         gsel = torch.zeros_like(sel_all)
         gn = torch.zeros_like(n_all)
@@ -121,6 +126,11 @@ def test_fullsize_step_matches_oracle_on_sampled_units(name, policy, alpha, budg
     G = wl.group
     n_units = 8 if wl.units >= 256 else 4
     for b, h in _sample_units(wl, n_units):
+        if full:
+            orc = oracle_unit(inp, b, h, policy="all", alpha=alpha)
+            check_unit_decode(orc, out_d, tau, cnt, bits, b, h, G, wl.dtype,
+                              what=f"{name} full cache alpha {alpha} unit {(b, h)}")
+            continue
         got = sel_all[b, h, : int(n_all[b, h])].cpu().numpy()
         orc = oracle_unit(inp, b, h, policy=policy, k=k, delta=delta, alpha=alpha)
         if policy == "topk":

@@ -234,3 +234,24 @@ def test_decode_step_end_to_end(case, policy):
     n_kern = B.ekv_step_kernel_count(eng.cache, eng.seqs, eng.params, wl.num_q_heads)
     if policy == "topk":
         assert n_kern - 3 in ((1, 2) if wl.dtype == "bf16" else (3,)), n_kern
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.7])
+def test_streaming_full_cache_decode_ragged_lengths(alpha):
+    """Full-cache decode of sequences longer than the scores one thread keeps
+    in registers (they are read again from L2 at every pass of the per-head
+    CTA), ragged lengths on a scattered pool, 64 units: the two-launch decode
+    with its streaming per-head kernel, against the oracle."""
+    wl = scaled_down("short_scattered", batch=8, context=40000, context_min=17000)
+    inp = gen(wl, 4242)
+    gpu = Gpu(inp)
+    gpu.build_meta()
+    p = B.StepParams(B.EKV_POLICY_FULL, 0, 0.0, inp["max_pages"], alpha, gpu.scale, 0, 0)
+    assert B.ekv_step_kernel_count(gpu.cache, gpu.seqs, p, wl.num_q_heads) == 2
+    out, tau, cnt, bits = gpu.decode(alpha)
+    torch.cuda.synchronize()
+    assert B.ekv_get_error() == 0
+    for b, h in _units(wl, 4):
+        orc = oracle_unit(inp, b, h, policy="all", alpha=alpha)
+        check_unit_decode(orc, out, tau, cnt, bits, b, h, wl.group, wl.dtype,
+                          what=f"alpha {alpha} unit {(b, h)}")
