@@ -526,6 +526,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     }
     if (tid < C) cluster.map_shared_rank(s_tau, tid)[h] = tau;
     if (tid == 0 && a.tau_out) a.tau_out[orow] = tau;
+    if (a.bits_out == nullptr && a.count_out == nullptr) {
+      __syncthreads();  // zh, cand and tsh are reused by the next head
+      continue;
+    }
     int cnt = 0;
     for (int base = 0; base < n_tok; base += kFThreads) {
       const int i = base + tid;
@@ -581,7 +585,13 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+  // Each batch: eight V rows in flight per warp; lane q computes the weight
+  // of (row q / G, head q mod G) once and the FMAs take it by shuffle, so the
+  // loop body stays small (it runs once per launch on every SM: its
+  // instructions are fetched cold).
   constexpr int kRowsInFlight = 8;
+  constexpr int kPairs = kRowsInFlight * G;
+  constexpr int kPerLane = (kPairs + 31) / 32;
 #pragma unroll 1
   for (int e0 = warp * kRowsInFlight; e0 < ntl; e0 += kFWarps * kRowsInFlight) {
     float v[kRowsInFlight][DPL];
@@ -607,20 +617,25 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
         }
       }
     }
+    float pl[kPerLane];
 #pragma unroll
-    for (int r = 0; r < kRowsInFlight; ++r) {
-      const int e = e0 + r;
-      if (e < ntl) {
-        const int tok = tl[e];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float w = a.am1 * zs[h * zp + tok] - s_tau[h];
-          const float pt = w > 0.f ? pow_beta_fast(w, a.beta, a.ipow) : 0.f;
-#pragma unroll
-          for (int x = 0; x < DPL; ++x) acc[h][x] = fmaf(pt, v[r][x], acc[h][x]);
-        }
+    for (int k = 0; k < kPerLane; ++k) {
+      const int q = k * 32 + lane, r = q / G, h = q - r * G;
+      float pt = 0.f;
+      if (q < kPairs && e0 + r < ntl) {
+        const float w = a.am1 * zs[h * zp + tl[e0 + r]] - s_tau[h];
+        if (w > 0.f) pt = pow_beta_fast(w, a.beta, a.ipow);
       }
+      pl[k] = pt;
     }
+#pragma unroll
+    for (int r = 0; r < kRowsInFlight; ++r)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pt = __shfl_sync(0xffffffffu, pl[(r * G + h) / 32], (r * G + h) % 32);
+#pragma unroll
+        for (int x = 0; x < DPL; ++x) acc[h][x] = fmaf(pt, v[r][x], acc[h][x]);
+      }
   }
   __syncthreads();  // the token list is read by every warp before the partials overwrite it
   // warp partials → CTA partial (warp order) → the owner's inbox
