@@ -19,13 +19,20 @@ extern __device__ unsigned int g_error_flags;
 
 __device__ __forceinline__ void raise_flag(unsigned int bit) { atomicOr(&g_error_flags, bit); }
 
+// A hint that brings the 128-byte line holding p into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------------------ launches
 // Every kernel is launched with programmatic stream serialization: its CTAs
 // may be dispatched while the previous kernel on the stream drains.  Each
 // kernel therefore opens with grid_dep_enter(): it waits until the previous
 // kernel has completed and its memory is visible (griddepcontrol.wait; a
 // no-op when launched without the attribute), then lets the next kernel be
-// dispatched early.  No global memory is read or written before the wait.
+// dispatched early.  No global memory is read or written before the wait
+// (the fused decode only hints L2 prefetches of its page-table row there,
+// which no kernel writes).
 __device__ __forceinline__ void grid_dep_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -453,9 +453,70 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
 
 // ------------------------------------------------------------------ 3. pv
 constexpr int kPvWarps = 8;
+constexpr int kPvRows = 32;  // V rows in flight per warp (a multiple of the page size)
 
+// One lane's share of a V row (DPL = D/32 consecutive elements), loaded in
+// its stored form with one aligned load and widened to fp32 when used.
+template <typename T, int DPL>
+struct PvRaw;
+template <>
+struct PvRaw<bf16, 4> {
+  using Row = uint2;
+  static __device__ __forceinline__ Row zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ Row load(const bf16* p) { return *reinterpret_cast<const uint2*>(p); }
+  static __device__ __forceinline__ void widen(Row w, float* v) {
+    v[0] = __uint_as_float(w.x << 16);
+    v[1] = __uint_as_float(w.x & 0xffff0000u);
+    v[2] = __uint_as_float(w.y << 16);
+    v[3] = __uint_as_float(w.y & 0xffff0000u);
+  }
+};
+template <>
+struct PvRaw<bf16, 2> {
+  using Row = uint32_t;
+  static __device__ __forceinline__ Row zero() { return 0u; }
+  static __device__ __forceinline__ Row load(const bf16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+  static __device__ __forceinline__ void widen(Row w, float* v) {
+    v[0] = __uint_as_float(w << 16);
+    v[1] = __uint_as_float(w & 0xffff0000u);
+  }
+};
+template <>
+struct PvRaw<float, 4> {
+  using Row = float4;
+  static __device__ __forceinline__ Row zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  static __device__ __forceinline__ Row load(const float* p) { return *reinterpret_cast<const float4*>(p); }
+  static __device__ __forceinline__ void widen(Row w, float* v) {
+    v[0] = w.x;
+    v[1] = w.y;
+    v[2] = w.z;
+    v[3] = w.w;
+  }
+};
+template <>
+struct PvRaw<float, 2> {
+  using Row = float2;
+  static __device__ __forceinline__ Row zero() { return make_float2(0.f, 0.f); }
+  static __device__ __forceinline__ Row load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+  static __device__ __forceinline__ void widen(Row w, float* v) {
+    v[0] = w.x;
+    v[1] = w.y;
+  }
+};
+
+// Two CTAs per SM where the batch of packed rows, the accumulators and the
+// weights fit in 128 registers a thread, one otherwise (no spills).
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
+constexpr int pv_min_blocks() {
+  constexpr int regs = kPvRows * static_cast<int>(sizeof(typename PvRaw<T, D / 32>::Row)) / 4 + G * (D / 32) + G + 24;
+  return regs <= 120 ? 2 : 1;
+}
+
+// PS: the page size (16 or 32), a template parameter so that every row of a
+// batch is addressed from its page's base with a constant offset.
+template <typename T, int D, int G, int PS>
+__global__ void __launch_bounds__(32 * kPvWarps, pv_min_blocks<T, D, G>()) pv_kernel(DecodeArgs a) {
+  static_assert(kPvRows % PS == 0, "a batch holds whole pages");
   grid_dep_enter();
   constexpr int DPL = D / 32;  // output columns per lane
   extern __shared__ __align__(16) float red[];  // [kPvWarps][G][D]
@@ -465,7 +526,8 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
   __shared__ int s_last;
 
   const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, S = a.S;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int S = PS;
   int L;
   const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
   const int n_slots = unit_slots(a, unit, P);
@@ -504,45 +566,48 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
       s_nv[pos] = nv;
     }
     __syncthreads();
-    for (int e = warp; e < nsup; e += kPvWarps) {
-      const int sl = s_list[e], ph = s_phys[e], nvv = s_nv[e];
-      // V rows and p of token `lane` for every head are independent loads
-      const T* vb = static_cast<const T*>(a.v_pool) + (static_cast<size_t>(ph) * a.Hkv + kvh) * S * D + lane * DPL;
-      float p[G];
+    // warp w takes PP consecutive listed pages per batch (PP·S = kPvRows
+    // rows: two 16-token pages or one 32-token page); row r of the batch is
+    // token r mod S of page r / S.  The rows stay packed until used, so a
+    // whole batch is in flight; lane r computes row r's weight per head.
+    constexpr int PP = kPvRows / S;
+    for (int e0 = warp * PP; e0 < nsup; e0 += kPvWarps * PP) {
+      const T* vbase[PP];
+      int nvp[PP];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        p[h] = 0.f;
-        if (lane < nvv) {
-          const float w = a.am1 * a.ws.zbuf[(static_cast<size_t>(unit) * G + h) * zrow + static_cast<size_t>(sl) * S + lane] - s_tau[h];
-          if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ipow);
+      for (int q = 0; q < PP; ++q) {
+        const bool ok = e0 + q < nsup;
+        nvp[q] = ok ? s_nv[e0 + q] : 0;
+        vbase[q] = static_cast<const T*>(a.v_pool) +
+                   ((static_cast<size_t>(ok ? s_phys[e0 + q] : 0) * a.Hkv + kvh) * S) * D + lane * DPL;
+      }
+      typename PvRaw<T, DPL>::Row raw[kPvRows];
+#pragma unroll
+      for (int r = 0; r < kPvRows; ++r)
+        raw[r] = (r % S) < nvp[r / S] ? PvRaw<T, DPL>::load(vbase[r / S] + (r % S) * D) : PvRaw<T, DPL>::zero();
+      float p[G];
+      {
+        const int e = e0 + lane / S, t = lane % S;
+        const bool ok = e < nsup && t < s_nv[e];
+        const size_t zi = ok ? static_cast<size_t>(s_list[e]) * S + t : 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          p[h] = 0.f;
+          if (ok) {
+            const float w = a.am1 * a.ws.zbuf[(static_cast<size_t>(unit) * G + h) * zrow + zi] - s_tau[h];
+            if (w > 0.f) p[h] = pow_beta(w, a.beta, a.ipow);
+          }
         }
       }
-      for (int t0 = 0; t0 < nvv; t0 += 8) {
-        float vv[8][DPL];
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-          const int t = t0 + tt;
-          if (t < nvv) {
-            if constexpr (DPL == 4) {
-              load4(vb + static_cast<size_t>(t) * D, vv[tt]);
-            } else {
-              const T* src = vb + static_cast<size_t>(t) * D;
-              vv[tt][0] = to_f32(src[0]);
-              vv[tt][1] = to_f32(src[1]);
-            }
-          } else {
+      for (int r = 0; r < kPvRows; ++r) {
+        float v[DPL];
+        PvRaw<T, DPL>::widen(raw[r], v);
 #pragma unroll
-            for (int e2 = 0; e2 < DPL; ++e2) vv[tt][e2] = 0.f;
-          }
-        }
+        for (int h = 0; h < G; ++h) {
+          const float ph_t = __shfl_sync(0xffffffffu, p[h], r);
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float ph_t = __shfl_sync(0xffffffffu, p[h], (t0 + tt) & 31);
-#pragma unroll
-            for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(ph_t, vv[tt][e2], acc[h][e2]);
-          }
+          for (int e2 = 0; e2 < DPL; ++e2) acc[h][e2] = fmaf(ph_t, v[e2], acc[h][e2]);
         }
       }
     }
@@ -578,6 +643,21 @@ __global__ void __launch_bounds__(32 * kPvWarps) pv_kernel(DecodeArgs a) {
     a.out[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + h) * D + j] = s;
   }
   if (tid == 0) a.ws.counter[unit] = 0;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_pv(DecodeArgs& a, int U, cudaStream_t st) {
+  void (*kernel)(DecodeArgs) = a.S == 16 ? pv_kernel<T, D, G, 16> : pv_kernel<T, D, G, 32>;
+  const size_t pv_smem = static_cast<size_t>(kPvWarps) * G * D * sizeof(float);
+  if (pv_smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pv_smem));
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 gp(static_cast<unsigned>(a.ws.npv), static_cast<unsigned>(U));
+  const cudaError_t e = launch_k(kernel, gp, 32 * kPvWarps, pv_smem, st, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 template <typename T, int D, int G>
@@ -620,20 +700,27 @@ cudaError_t run_decode(DecodeArgs& a, int U, cudaStream_t st) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t pv_smem = static_cast<size_t>(kPvWarps) * G * D * sizeof(float);
-  if (pv_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(pv_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pv_smem));
-    if (e != cudaSuccess) return e;
-  }
-  const dim3 gp(static_cast<unsigned>(a.ws.npv), static_cast<unsigned>(U));
-  {
-    const cudaError_t le_ = launch_k(pv_kernel<T, D, G>, gp, 32 * kPvWarps, pv_smem, st, a);
-    if (le_ != cudaSuccess) return le_;
-  }
-  return cudaGetLastError();
+  return launch_pv<T, D, G>(a, U, st);
 }
 
 }  // namespace
+
+template <int D, int G>
+cudaError_t run_dense_v_pass(DecodeArgs& a, int units, cudaStream_t st) {
+  return launch_pv<bf16, D, G>(a, units, st);
+}
+#define EKV_PV_INST(DD, GG) template cudaError_t run_dense_v_pass<DD, GG>(DecodeArgs&, int, cudaStream_t);
+EKV_PV_INST(128, 1)
+EKV_PV_INST(128, 2)
+EKV_PV_INST(128, 4)
+EKV_PV_INST(128, 8)
+EKV_PV_INST(128, 16)
+EKV_PV_INST(64, 1)
+EKV_PV_INST(64, 2)
+EKV_PV_INST(64, 4)
+EKV_PV_INST(64, 8)
+EKV_PV_INST(64, 16)
+#undef EKV_PV_INST
 
 int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap, int dense_v) {
   const int G = Hq / c.num_kv_heads, U = s.batch * c.num_kv_heads;
@@ -642,7 +729,7 @@ int decode_kernel_count(const ekv_cache& c, const ekv_seqs& s, int Hq, int cap, 
   if (c.head_dim == DD && G == GG)                                                           \
     switch (choose_decode_path<DD, GG>(U, cap, c.page_size, dense_v)) {                           \
       case DecodePath::kFused: return 1;                                                            \
-      case DecodePath::kSplit: return 2;                                                            \
+      case DecodePath::kSplit: return dense_v ? 3 : 2;                                              \
       default: return 3;                                                                            \
     }
   EKV_CNT_CASE(128, 1) EKV_CNT_CASE(128, 2) EKV_CNT_CASE(128, 4) EKV_CNT_CASE(128, 8) EKV_CNT_CASE(128, 16)

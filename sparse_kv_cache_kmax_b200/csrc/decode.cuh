@@ -123,6 +123,10 @@ template <int D, int G>
 bool split_decode_fits(int cap, int S);
 template <int D, int G>
 cudaError_t run_split_decode(DecodeArgs& a, int units, cudaStream_t st);
+// The three-kernel decode's V pass alone (decode.cu), over the scores and τ
+// the split decode left in the workspace: its dense-V variant.
+template <int D, int G>
+cudaError_t run_dense_v_pass(DecodeArgs& a, int units, cudaStream_t st);
 
 // Launch of the fused path: false when the configuration does not fit it
 // (the caller then runs the three-kernel path).
@@ -134,15 +138,16 @@ int fused_decode_cluster(int units, int cap, int S);
 
 // The decode path of a bf16 selection: the one-cluster-per-unit kernel when
 // at least kFusedMinCluster CTAs can work on each unit at once (few units),
-// else the two-launch split decode when the selection fits it (many units),
-// else whichever fits, else the three-kernel path.
+// else the split decode when the selection fits it (many units, or the full
+// cache: two launches, a third for dense V), else whichever fits, else the
+// three-kernel path.
 constexpr int kFusedMinCluster = 4;
 enum class DecodePath { kFused, kSplit, kThree };
 template <int D, int G>
 DecodePath choose_decode_path(int units, int cap, int S, int dense_v) {
   if (units > 65535) return DecodePath::kThree;
   const int C = fused_decode_cluster<D, G>(units, cap, S);
-  const bool split = !dense_v && split_decode_fits<D, G>(cap, S);
+  const bool split = split_decode_fits<D, G>(cap, S);
   if (C >= kFusedMinCluster) return DecodePath::kFused;
   if (split) return DecodePath::kSplit;
   return C > 0 ? DecodePath::kFused : DecodePath::kThree;

@@ -396,6 +396,15 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     fence_mbar_init();
   }
   for (int i = tid; i < kTauBinsF; i += kFThreads) tsh.hist[i] = 0;
+  // The page table is written by no kernel of the step: this CTA's share of
+  // the sequence's row is brought into L2 while the selection is still being
+  // made (a hint; the row is read again after the wait)
+  {
+    const int per = (a.max_pages + C - 1) / C;
+    const int p0 = rank * per, p1 = min(a.max_pages, p0 + per);
+    const int* row = a.page_table + static_cast<size_t>(b) * a.max_pages;
+    for (int p = p0 + 32 * tid; p < p1; p += 32 * kFThreads) prefetch_l2(row + p);
+  }
   __syncthreads();
   grid_dep_enter();
   int L;
@@ -497,6 +506,30 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     if (lane < C) cluster.map_shared_rank(&mall[0][0], lane)[h * kFMaxCluster + rank] = m;
   }
   cluster.sync();
+  // Every support token has u > max u − 1 for its head (its weight is at
+  // most 1): the V rows of those candidates are brought into L2 now, so the
+  // V pass after τ finds them there
+  if (!a.dense_v) {
+    float lo[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float m = -INFINITY;
+      for (int r = 0; r < C; ++r) m = fmaxf(m, mall[h][r]);
+      lo[h] = a.am1 * m - 1.0f;
+    }
+    for (int x = tid; x < np * S; x += kFThreads) {
+      const int j = x / S;
+      bool cand = false;
+#pragma unroll
+      for (int h = 0; h < G; ++h) cand |= a.am1 * zs[h * zp + x] > lo[h];
+      if (cand && phys_s[j] >= 0 && x - j * S < nv_s[j]) {
+        const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                          ((static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * S + (x - j * S)) * D;
+#pragma unroll
+        for (int c = 0; c < D * 2; c += 128) prefetch_l2(reinterpret_cast<const unsigned char*>(src) + c);
+      }
+    }
+  }
 
   // ---------------------------------------------------------------- 2. τ
   const int tpc = spc * S;

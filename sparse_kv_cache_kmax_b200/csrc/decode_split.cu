@@ -22,8 +22,10 @@
 //     read, eight rows in flight per warp; warp partials are summed in warp
 //     order.
 // The heads of a unit read the same V rows at about the same time, so a row
-// they share comes from DRAM once.  Every sum has a fixed order, so results
-// are deterministic.
+// they share comes from DRAM once.  With dense V, the per-head CTAs stop
+// after τ and the V pass of the three-kernel decode reads every valid row
+// once for all heads of the unit (pv_kernel, decode.cu).  Every sum has a
+// fixed order, so results are deterministic.
 #include "decode.cuh"
 
 namespace ekv {
@@ -63,6 +65,7 @@ __global__ void __launch_bounds__(kKsThreads, 2) k_score_kernel(DecodeArgs a) {
   const int n_slots = unit_slots(a, unit, P);
   const int ppc = kKsTokens / S;  // pages per CTA
   const int s_begin = split * ppc;
+  if (split == 0 && tid == 0) a.ws.counter[unit] = 0;  // the dense V pass's ticket
   if (s_begin >= n_slots) return;  // CTA-uniform
   if (tid < G) cta_key[tid] = 0u;
   const int row0 = warp * 32;
@@ -516,7 +519,9 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   if (tid == 0) {
     if (a.tau_out) a.tau_out[orow] = tau;
     if (a.count_out) a.count_out[orow] = ns;
+    if (a.dense_v) a.ws.taus[row] = tau;
   }
+  if (a.dense_v) return;  // every V row is read by the V pass that follows
 
   // 5. V of the support rows: warp w takes rows w·8 … w·8+7 of each block of 64
   float acc[DPL];
@@ -604,7 +609,9 @@ cudaError_t run_split_decode(DecodeArgs& a, int units, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_head_decode<D>(a, units * G, G, st);
+  e = launch_head_decode<D>(a, units * G, G, st);
+  if (e != cudaSuccess || !a.dense_v) return e;
+  return run_dense_v_pass<D, G>(a, units, st);
 }
 
 #define EKV_SPLIT_INST(DD, GG)                               \

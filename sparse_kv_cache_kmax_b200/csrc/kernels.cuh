@@ -7,9 +7,10 @@
 namespace ekv {
 
 // Decode work split.  The score pass over the selected K takes 256 tokens per
-// CTA (8 warps × 32 tokens); the V pass aims for two CTAs per SM of a B200.
+// CTA (8 warps × 32 tokens); the V pass aims for eight CTAs per SM of a B200
+// (two resident at a time), so that a dense V read keeps enough rows in flight.
 constexpr int kQkTokensPerCta = 256;
-constexpr int kPvTargetCtas = 296;
+constexpr int kPvTargetCtas = 1184;
 constexpr int kPvMaxSplits = 64;
 
 struct DecodeWs {

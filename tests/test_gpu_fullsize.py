@@ -24,7 +24,7 @@ from sparse_kv_cache_kmax_b200.engine import DecodeEngine
 from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, gauss_cap
 
 from gpu_helpers import (REL_TIE, assert_sel_matches, check_unit_decode, gen, np64, oracle_unit,
-                         topk_tie_band)
+                         row_rel_err, topk_tie_band)
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +95,15 @@ def test_fullsize_step_matches_oracle_on_sampled_units(name, policy, alpha, budg
                         None if full else n_all, cap, out_d, ws, tau=tau, support_count=cnt, support_bits=bits)
     torch.cuda.synchronize()
     assert torch.equal(out_d, out), "the step's decode and the standalone decode differ"
+    if full:
+        # the dense-V variant: same τ, every V row read, zero weights add nothing
+        out_v = torch.full_like(out, float("nan"))
+        tau_v = torch.full_like(tau, float("nan"))
+        B.ekv_entmax_decode(eng.cache, eng.seqs, inp["q"], eng.params.scale, alpha, None, None, cap, out_v, ws,
+                            dense_v=True, tau=tau_v)
+        torch.cuda.synchronize()
+        assert torch.equal(tau_v, tau)
+        assert np.all(row_rel_err(np64(out_v).reshape(-1, wl.head_dim), np64(out_d).reshape(-1, wl.head_dim)) <= 1e-5)
 
     scale = float(np.float32(wl.scale))
     if policy == "topk":

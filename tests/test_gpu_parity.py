@@ -255,3 +255,11 @@ def test_streaming_full_cache_decode_ragged_lengths(alpha):
         orc = oracle_unit(inp, b, h, policy="all", alpha=alpha)
         check_unit_decode(orc, out, tau, cnt, bits, b, h, wl.group, wl.dtype,
                           what=f"alpha {alpha} unit {(b, h)}")
+    # dense V: the same scores and τ, then every valid V row read once per
+    # unit by a third launch; zero weights add nothing
+    p.dense_v = 1
+    assert B.ekv_step_kernel_count(gpu.cache, gpu.seqs, p, wl.num_q_heads) == 3
+    out_d, tau_d, cnt_d, _ = gpu.decode(alpha, dense_v=True)
+    torch.cuda.synchronize()
+    assert torch.equal(tau_d, tau) and torch.equal(cnt_d, cnt)
+    assert np.all(row_rel_err(np64(out_d).reshape(-1, wl.head_dim), np64(out).reshape(-1, wl.head_dim)) <= 1e-5)
