@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   __syncthreads();
 
   float tau = INFINITY;  // no finite score: no support, zero output
+  int n_listed = -1;     // candidates listed in shared memory (−1: too many)
   if (m > -INFINITY) {
     const float um = am1 * m;
     // 1. bracket from the histogram of u over (um − 1, um], bin 0 at the top
@@ -306,6 +307,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
       __syncthreads();
     }
     const bool listed = nc <= kHdCand;
+    if (listed) n_listed = nc;
 
     // 3. τ
     const bool closed = ipow == 1 || ipow == 2;
@@ -484,16 +486,12 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   }
   __syncthreads();  // the candidate area is reused for the support list
 
-  // 4. support with the fp32 τ every later step uses: bits by ballots, and
-  //    compact(base) lists the support tokens at places base .. base +
-  //    kHdCand − 1 (thread after thread) with their weights p = (u − τ)^β;
-  //    it returns the support's size.
-  if (a.bits_out)
-    for_values([&](int k, float u) {
-      const int i = k * THREADS + tid;
-      const unsigned int bal = __ballot_sync(0xffffffffu, i < n && u > tau);
-      if (lane == 0 && (i >> 5) < a.words) a.bits_out[orow * a.words + (i >> 5)] = bal;
-    });
+  // 4. support with the fp32 τ every later step uses, listed at places
+  //    base .. base + kHdCand − 1 (thread after thread) with the weights
+  //    p = (u − τ)^β.  The support lies inside the candidates (u > τ ≥ τ_lo):
+  //    when they are listed, the support is cut from their list (same order)
+  //    and its bits are set one token at a time; otherwise compact(base)
+  //    passes over every value and the bits come from ballots.
   auto compact = [&](int base) {
     int mine = 0;
     for_values([&](int k, float u) { mine += (k * THREADS + tid < n && u > tau) ? 1 : 0; });
@@ -512,10 +510,51 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
     __syncthreads();
     return ns;
   };
-  const int ns = compact(0);
-  if (a.bits_out)
-    for (int w = ((kReg ? VPT : NK) * THREADS) / 32 + tid; w < a.words; w += THREADS)
-      a.bits_out[orow * a.words + w] = 0u;  // words past the ballots above
+  int ns;
+  if (n_listed >= 0) {
+    constexpr int kPer = (kHdCand + THREADS - 1) / THREADS;
+    float cu_r[kPer];
+    int ci_r[kPer];
+    int mine = 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int j = tid * kPer + q;
+      cu_r[q] = -INFINITY;
+      ci_r[q] = 0;
+      if (j < n_listed) {
+        cu_r[q] = sh.cu[j];
+        ci_r[q] = sh.ci[j];
+        mine += cu_r[q] > tau ? 1 : 0;
+      }
+    }
+    int p = block_exclusive_scan(mine, sh.i, &ns);  // every candidate is read before it returns
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (cu_r[q] > tau) {
+        sh.cu[p] = pow_beta_fast(cu_r[q] - tau, beta, ipow);
+        sh.ci[p] = ci_r[q];
+        ++p;
+      }
+    if (a.bits_out)
+      for (int w = tid; w < a.words; w += THREADS) a.bits_out[orow * a.words + w] = 0u;
+    __syncthreads();
+    if (a.bits_out)
+      for (int e = tid; e < ns; e += THREADS) {
+        const int i = sh.ci[e];
+        atomicOr(&a.bits_out[orow * a.words + (i >> 5)], 1u << (i & 31));
+      }
+  } else {
+    if (a.bits_out)
+      for_values([&](int k, float u) {
+        const int i = k * THREADS + tid;
+        const unsigned int bal = __ballot_sync(0xffffffffu, i < n && u > tau);
+        if (lane == 0 && (i >> 5) < a.words) a.bits_out[orow * a.words + (i >> 5)] = bal;
+      });
+    ns = compact(0);
+    if (a.bits_out)
+      for (int w = ((kReg ? VPT : NK) * THREADS) / 32 + tid; w < a.words; w += THREADS)
+        a.bits_out[orow * a.words + w] = 0u;  // words past the ballots above
+  }
   if (tid == 0) {
     if (a.tau_out) a.tau_out[orow] = tau;
     if (a.count_out) a.count_out[orow] = ns;
