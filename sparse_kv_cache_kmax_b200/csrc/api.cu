@@ -69,7 +69,9 @@ size_t gauss_ws_bytes(const ekv_cache* c, const ekv_seqs* s, int Hq) {
   const size_t U = static_cast<size_t>(s->batch) * c->num_kv_heads;
   const size_t G = static_cast<size_t>(Hq / c->num_kv_heads);
   const size_t rows = U * G * static_cast<size_t>(s->max_pages);
-  return 3 * a256(rows * sizeof(float)) + a256(U * G * sizeof(double));
+  const size_t nch = U * static_cast<size_t>(filter_chunks(s->max_pages));
+  return 3 * a256(rows * sizeof(float)) + a256(U * G * sizeof(double)) + a256(nch * sizeof(int)) +
+         a256(nch * sizeof(double)) + a256(nch * sizeof(int));
 }
 
 GaussWs carve_gauss(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq) {
@@ -81,6 +83,10 @@ GaussWs carve_gauss(Carver& cv, const ekv_cache* c, const ekv_seqs* s, int Hq) {
   w.sig = cv.take<float>(rows);
   w.hat = cv.take<float>(rows);
   w.tau_hat = cv.take<double>(U * G);
+  w.nchunk = filter_chunks(s->max_pages);
+  w.fcount = cv.take<int>(U * static_cast<size_t>(w.nchunk));
+  w.fbest = cv.take<double>(U * static_cast<size_t>(w.nchunk));
+  w.fbest_at = cv.take<int>(U * static_cast<size_t>(w.nchunk));
   return w;
 }
 
@@ -402,7 +408,7 @@ EKV_API int32_t ekv_step_kernel_count(const ekv_cache* cache, const ekv_seqs* se
   int n = p->append ? 1 : 0;
   if (p->policy == EKV_POLICY_TOPK)
     n += 1 + (topk_ws_bytes(seqs->batch * cache->num_kv_heads, seqs->max_pages, p->k) > 0 ? 2 : 1);
-  else if (p->policy == EKV_POLICY_GAUSS) n += 3;
+  else if (p->policy == EKV_POLICY_GAUSS) n += 4;
   else if (!full) return 0;
   return n + decode_kernel_count(*cache, *seqs, num_q_heads, cap, p->dense_v);
 }

@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kTauThreads) tau_kernel(DecodeArgs a, int G) {
           tau = static_cast<double>(um) - 1.0;
           continue;
         }
-        const double step = (f - 1.0) / (static_cast<double>(beta) * df);
+        const double step = norm_newton_step<double>(f - 1.0, df, static_cast<double>(beta));
         if (!(step > 0.0)) break;
         tau += step;
         if (step <= 1e-11 * fmax(1.0, fabs(tau))) break;

@@ -60,6 +60,24 @@ __device__ __forceinline__ float pow_beta(float w, float beta, int ipow) {
 // The same with a fast base-2 exp/log for non-integer β (relative error near
 // 1e-6, far inside the bf16 output tolerance): a few instructions instead of
 // an inlined powf, for code that runs once per CTA.
+// Newton step toward the root of Σ_i (u_i − τ)_+^β = 1, taken on
+// h(τ) = (Σ_i (u_i − τ)_+^β)^(1/β), the ℓ_β norm of (u − τ)_+: convex and
+// decreasing, so steps from the left never pass the root, and close to linear
+// far from it (Newton on the sum itself closes only a fraction 1/β of the gap
+// there).  With F = 1 + f the sum and s = Σ_i (u_i − τ)_+^(β−1), the step
+// (h − 1)/(−h') is F^(1−1/β)·(F^(1/β) − 1)/s, formed from f without
+// cancellation near the root; for β = 1 it is Newton's step f/s.
+template <typename V>
+__device__ __forceinline__ V norm_newton_step(V f, V s, V beta) {
+  if constexpr (sizeof(V) == 8) {
+    const double l = log1p(f);
+    return exp((1.0 - 1.0 / beta) * l) * expm1(l / beta) / s;
+  } else {
+    const float l = log1pf(f);
+    return expf((1.0f - 1.0f / beta) * l) * expm1f(l / beta) / s;
+  }
+}
+
 __device__ __forceinline__ float pow_beta_fast(float w, float beta, int ipow) {
   switch (ipow) {
     case 1: return w;

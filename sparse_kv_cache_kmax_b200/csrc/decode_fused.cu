@@ -212,7 +212,7 @@ __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_
         t = um - 1.0f;
         continue;
       }
-      const float step = f / (beta * df);
+      const float step = norm_newton_step<float>(f, df, beta);
       if (!(step > 0.0f)) break;
       t += step;
       if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;

@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
               t = um - 1.0f;
               continue;
             }
-            const float step = f / (beta * df);
+            const float step = norm_newton_step<float>(f, df, beta);
             if (!(step > 0.0f)) break;
             t += step;
             if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
           t = um - 1.0f;
           continue;
         }
-        const float step = f / (beta * df);
+        const float step = norm_newton_step<float>(f, df, beta);
         if (!(step > 0.0f)) break;
         t += step;
         if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;

@@ -9,24 +9,29 @@
 // c = (τ − μ)/σ and J_k(c) = ∫_c^∞ (x − c)^k φ(x) dx,
 //   E[(u − τ)_+^β] = σ^β J_β(c),   dE/dτ = −β σ^(β−1) J_(β−1)(c),
 //   J_0 = Q(c),  J_1 = φ(c) − c·Q(c),  J_k = (k−1)·J_(k−2) − c·J_(k−1)
-// (integration by parts with xφ = −φ').  F is convex and decreasing, so
-// Newton's method started left of the root (Jensen's bound
-// τ_lo = max_p μ_p − n_p^(−1/β), where F ≥ 1) climbs monotonically to it and
-// never overshoots.  Pages with c > kPruneC at τ_lo contribute below
+// (integration by parts with xφ = −φ').  F^(1/β) is convex and decreasing
+// (an L^β norm of (u − τ)_+), so Newton's method on it, started left of the
+// root (Jensen's bound τ_lo = max_p μ_p − n_p^(−1/β), where F ≥ 1), climbs
+// monotonically to the root and never overshoots.  Pages with c > kPruneC at τ_lo contribute below
 // n·σ^β·J_β(kPruneC) and stay negligible for every later τ (c only grows), so
 // only the survivors are iterated, from shared memory.  The recurrence
 // amplifies the rounding of Q and φ by about c^(2β)/β! for c > 0, so the fp32
 // iterations only approach the root (they stop once a step is below 1e-5);
 // the final Newton steps evaluate every term in float64.
+#include <cooperative_groups.h>
+
 #include "kernels.cuh"
 
 namespace ekv {
 
+namespace cg = cooperative_groups;
+
 namespace {
 
 constexpr int kGaussThreads = 256;   // filter
-constexpr int kTauThreads = 1024;    // τ̂ solve: one CTA per query head, every thread on its pages
-constexpr int kGaussCand = 3072;
+constexpr int kTauThreads = 512;     // τ̂ solve: a cluster of up to kTauMaxCluster CTAs per query head
+constexpr int kTauMaxCluster = 4;
+constexpr int kGaussCand = 4096;     // candidate pages per CTA in shared memory
 constexpr float kPruneC = 6.0f;
 
 template <typename R>
@@ -58,7 +63,10 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
     }
     return;
   }
-  const R c = static_cast<R>((tau - static_cast<double>(mu)) / static_cast<double>(sg));
+  // c in the precision of the terms (the fp32 steps only approach the root)
+  R c;
+  if constexpr (sizeof(R) == 8) c = (tau - static_cast<double>(mu)) / static_cast<double>(sg);
+  else c = __fdividef(static_cast<float>(tau) - mu, sg);
   if (c > static_cast<R>(kPruneC)) return;
   R Q, phi;
   normal_tail<R>(c, Q, phi);
@@ -77,42 +85,63 @@ __device__ __forceinline__ void gauss_terms(float mu, float sg, float n, double 
   dF += static_cast<double>(n) * beta * sb1 * static_cast<double>(jb1 > R(0) ? jb1 : R(0));
 }
 
+// Partial sums every CTA of a head's cluster pushes to every other one.
+struct TauExchange {
+  double part[2][kTauMaxCluster][2];  // [step parity][rank][F, F']
+  float lo[kTauMaxCluster];
+};
+
+// One cluster of C CTAs per query head; CTA r owns the r-th contiguous
+// share of the head's pages.  Every sum is a fixed tree inside a CTA, then
+// the C partials in rank order, so all CTAs hold the same value and take the
+// same steps.
 __global__ void __launch_bounds__(kTauThreads)
-    gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
-                     int Hkv, int G, int Hq, int beta, float* __restrict__ tau_out) {
+    gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages, int Hkv, int G,
+                     int Hq, int beta, float* __restrict__ tau_out) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks()), rank = static_cast<int>(cluster.block_rank());
   grid_dep_enter();
-  const int row = blockIdx.x, unit = row / G, g = row % G, b = unit / Hkv, kvh = unit % Hkv;
-  const int tid = threadIdx.x;
+  const int row = blockIdx.y, unit = row / G, g = row % G, b = unit / Hkv, kvh = unit % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
-  __shared__ float c_mu[kGaussCand], c_sg[kGaussCand], c_n[kGaussCand];
+  const int per = (P + C - 1) / C, pa = min(P, rank * per), pb = min(P, pa + per);
+  extern __shared__ float cand[];  // [3][kGaussCand]: μ, σ, n of the cached pages
+  float* c_mu = cand;
+  float* c_sg = cand + kGaussCand;
+  float* c_n = cand + 2 * kGaussCand;
+  __shared__ TauExchange tx;
   __shared__ float f_scratch[32];
   __shared__ double d_scratch[64];
   __shared__ int i_scratch[32];
+  int par = 0;
 
   // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
   const size_t base = static_cast<size_t>(row) * max_pages;
   const float inv_beta = 1.0f / static_cast<float>(beta);
   float lo = -INFINITY;
-  for (int p = tid; p < P; p += blockDim.x) {
+  for (int p = pa + tid; p < pb; p += kTauThreads) {
     const float mu = ws.mu[base + p];
     if (mu > -INFINITY) lo = fmaxf(lo, mu - powf(static_cast<float>(min(S, L - p * S)), -inv_beta));
   }
   lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
+  if (tid < C) cluster.map_shared_rank(&tx, tid)->lo[rank] = lo;
+  cluster.sync();
+  for (int r = 0; r < C; ++r) lo = fmaxf(lo, tx.lo[r]);
   if (P == 0 || !(lo > -INFINITY)) {
-    if (tid == 0) {
+    if (rank == 0 && tid == 0) {
       ws.tau_hat[row] = static_cast<double>(INFINITY);
       if (tau_out) tau_out[static_cast<size_t>(b) * Hq + kvh * G + g] = INFINITY;
     }
     return;
   }
 
-  // Candidates: the pages with μ + kPruneC·σ above the current τ.  τ only
-  // rises (Newton from the left), so a page dropped once stays negligible;
-  // the list is cut again as τ climbs.  Gathered thread after thread
-  // (thread t takes pages t, t + 256, …: coalesced loads; a fixed order, so
-  // the sums below are deterministic); while too many pages are left for
-  // shared memory, the steps read every page from global memory.
+  // Candidates: this CTA's pages with μ + kPruneC·σ above the current τ.  τ
+  // only rises (Newton from the left), so a page dropped once stays
+  // negligible; the list is cut again as τ climbs.  Gathered thread after
+  // thread (coalesced loads; a fixed order, so the sums are deterministic);
+  // while too many pages are left for shared memory, the steps read every
+  // page of the share from global memory.
   auto live = [&](int p, double t) {
     const float mu = ws.mu[base + p], sg = ws.sig[base + p];
     return mu > -INFINITY && static_cast<double>(mu) + kPruneC * static_cast<double>(sg) > t;
@@ -121,11 +150,11 @@ __global__ void __launch_bounds__(kTauThreads)
   bool cached = false;
   auto gather = [&](double t) {  // every thread calls it
     int mine = 0;
-    for (int p = tid; p < P; p += kTauThreads) mine += live(p, t) ? 1 : 0;
+    for (int p = pa + tid; p < pb; p += kTauThreads) mine += live(p, t) ? 1 : 0;
     int pos = block_exclusive_scan(mine, i_scratch, &nc);
     cached = nc <= kGaussCand;
     if (cached)
-      for (int p = tid; p < P; p += kTauThreads)
+      for (int p = pa + tid; p < pb; p += kTauThreads)
         if (live(p, t)) {
           c_mu[pos] = ws.mu[base + p];
           c_sg[pos] = ws.sig[base + p];
@@ -135,11 +164,10 @@ __global__ void __launch_bounds__(kTauThreads)
     __syncthreads();
   };
   // cuts the cached list to the pages still above t, in place, order kept:
-  // thread t owns entries [t·R, t·R + R) (R ≤ 4), holds its survivors in
-  // registers across one barrier, then writes them at their new places
+  // thread t owns entries [t·R, t·R + R), holds its survivors in registers
+  // across the scan's barriers, then writes them at their new places
   auto recut = [&](double t) {
-    constexpr int kMaxR = 4;
-    static_assert(kGaussCand <= kMaxR * kTauThreads, "entries per thread");
+    constexpr int kMaxR = kGaussCand / kTauThreads;
     const int R = (nc + kTauThreads - 1) / kTauThreads;
     float m[kMaxR], sgm[kMaxR], nn[kMaxR];
     unsigned int keep = 0u;
@@ -169,19 +197,20 @@ __global__ void __launch_bounds__(kTauThreads)
   };
   gather(static_cast<double>(lo));
 
-  // F(τ) and F'(τ) over the candidates (or every page), summed in a fixed order
+  // F(τ) and F'(τ) over the head's candidates: this CTA's terms in a fixed
+  // tree, then the cluster's partials in rank order
   auto evaluate = [&](double t, bool exact, double& F, double& dF) {
     F = 0.0;
     dF = 0.0;
     if (cached) {
-      for (int i = tid; i < nc; i += blockDim.x) {
+      for (int i = tid; i < nc; i += kTauThreads) {
         if (exact)
           gauss_terms<double>(c_mu[i], c_sg[i], c_n[i], t, beta, F, dF);
         else
           gauss_terms<float>(c_mu[i], c_sg[i], c_n[i], t, beta, F, dF);
       }
     } else {
-      for (int p = tid; p < P; p += blockDim.x) {
+      for (int p = pa + tid; p < pb; p += kTauThreads) {
         const float n = static_cast<float>(min(S, L - p * S));
         if (exact)
           gauss_terms<double>(ws.mu[base + p], ws.sig[base + p], n, t, beta, F, dF);
@@ -189,33 +218,54 @@ __global__ void __launch_bounds__(kTauThreads)
           gauss_terms<float>(ws.mu[base + p], ws.sig[base + p], n, t, beta, F, dF);
       }
     }
-    const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       F += __shfl_xor_sync(0xffffffffu, F, o);
       dF += __shfl_xor_sync(0xffffffffu, dF, o);
     }
-    __syncthreads();  // the previous evaluation's partials are read
     if (lane == 0) {
       d_scratch[warp] = F;
       d_scratch[32 + warp] = dF;
     }
     __syncthreads();
+    if (tid < C) {
+      double sf = 0.0, sd = 0.0;
+      for (int w = 0; w < kTauThreads / 32; ++w) {
+        sf += d_scratch[w];
+        sd += d_scratch[32 + w];
+      }
+      TauExchange* dst = cluster.map_shared_rank(&tx, tid);
+      dst->part[par][rank][0] = sf;
+      dst->part[par][rank][1] = sd;
+    }
+    cluster.sync();  // also orders this step's reads of d_scratch before the next step's writes
     F = 0.0;
     dF = 0.0;
-    for (int w = 0; w < kTauThreads / 32; ++w) {
-      F += d_scratch[w];
-      dF += d_scratch[32 + w];
+    for (int r = 0; r < C; ++r) {
+      F += tx.part[par][r][0];
+      dF += tx.part[par][r][1];
     }
+    par ^= 1;  // the next step writes the other half: a slow CTA may still read this one
   };
   // fp32 terms: a monotone approach from the left while the steps are large
-  // (the list cut every few steps); the float64 steps below converge
+  // (the lists cut every few steps); the float64 steps below converge
   // quadratically from there
+  // Newton's method on h(τ) = F(τ)^(1/β), the L^β norm of (u − τ)_+ under the
+  // pages' mixture: convex and decreasing like F, so the steps from the left
+  // never pass the root, and close to linear far from it (Newton on F itself
+  // only closes a fraction 1/β of the gap per step there).  The step
+  // (h − 1)/(−h') is β·(F − F^(1−1/β))/(−F') = β·F^(1−1/β)·(F^(1/β) − 1)/(−F'),
+  // evaluated from F − 1 without cancellation near the root.
+  const double omb = 1.0 - 1.0 / beta;
+  auto newton_step = [&](double F, double dF) {
+    const double l = log1p(F - 1.0);
+    return beta * exp(omb * l) * expm1(l / beta) / dF;
+  };
   double tau = static_cast<double>(lo);
   for (int it = 0; it < 40; ++it) {
     double F, dF;
     evaluate(tau, false, F, dF);
-    const double step = (F - 1.0) / dF;
+    const double step = newton_step(F, dF);
     if (!(step > 0.0)) break;
     tau += step;
     if (step <= 1e-5 * fmax(1.0, fabs(tau))) break;
@@ -225,95 +275,74 @@ __global__ void __launch_bounds__(kTauThreads)
     }
   }
   if (!cached) gather(tau);
-  for (int it = 0; it < 3; ++it) {    // float64 terms: quadratic convergence (either side)
+  for (int it = 0; it < 3; ++it) {  // float64 terms: quadratic convergence (either side)
     double F, dF;
     evaluate(tau, true, F, dF);
-    if (!(dF > 0.0)) break;
-    const double step = (F - 1.0) / dF;
+    if (!(dF > 0.0) || !(F > 0.0)) break;
+    const double step = newton_step(F, dF);
     tau += step;
-    if (fabs(step) <= 1e-12 * fmax(1.0, fabs(tau))) break;
+    // the error left after a step of size e is of order e², so a step below
+    // 1e-7 leaves τ̂ within ~1e-14: no further evaluation is needed
+    if (fabs(step) <= 1e-7 * fmax(1.0, fabs(tau))) break;
   }
-  if (tid == 0) {
+  if (rank == 0 && tid == 0) {
     ws.tau_hat[row] = tau;
     if (tau_out) tau_out[static_cast<size_t>(b) * Hq + kvh * G + g] = static_cast<float>(tau);
   }
 }
 
-// Keep page p when (α−1)·ŝ_{p,h} > τ̂_h − Δ for some query head h of the unit;
-// compaction in ascending page order; fallback to the largest margin.
+// Keep page p when (α−1)·ŝ_{p,h} > τ̂_h − Δ for some query head h of the unit,
+// in ascending page order; when no page passes, keep the page of largest
+// margin (lowest index on ties).  Two launches over chunks of kFilterChunk
+// pages: the first counts each chunk's kept pages and finds its best margin,
+// the second writes the kept pages at the place the counts of the earlier
+// chunks give (chunk 0 also writes n_sel, and the fallback page).
+struct FilterCtx {
+  double thr[16];  // τ̂_h − Δ
+  int scan[32];
+  double best_m[32];
+  int best_i[32];
+};
+
+__device__ __forceinline__ double page_margin(const GaussWs& ws, const FilterCtx& fc, int unit, int G, int max_pages,
+                                              int p) {
+  double mg = -INFINITY;
+  for (int g = 0; g < G; ++g)
+    mg = fmax(mg, static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - fc.thr[g]);
+  return mg;
+}
+
+// The chunk's pages [c0, c1): warp w takes [c0 + w·kPer, …), its lanes
+// consecutive pages (coalesced loads).
+constexpr int kFilterPerWarp = kFilterChunk / (kGaussThreads / 32);
+
 __global__ void __launch_bounds__(kGaussThreads)
-    gauss_filter_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages,
-                        int Hkv, int G, double delta, int cap, int32_t* __restrict__ sel,
-                        int32_t* __restrict__ n_sel) {
+    gauss_count_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages, int Hkv, int G,
+                       double delta) {
   grid_dep_enter();
-  const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
+  const int chunk = blockIdx.x, unit = blockIdx.y, b = unit / Hkv, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
-  __shared__ double s_thr[16];
-  __shared__ int scan_scratch[32];
-  __shared__ double best_m[32];
-  __shared__ int best_i[32];
-  if (tid < G) s_thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
+  __shared__ FilterCtx fc;
+  if (tid < G) fc.thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
   __syncthreads();
-  int32_t* out = sel + static_cast<size_t>(unit) * cap;
-  // warp w owns the pages [w·C, (w + 1)·C), its lanes consecutive pages
-  // (coalesced loads): one pass counts the kept pages by ballots (and finds
-  // the best margin), the warp counts are scanned, a second pass writes the
-  // kept pages in ascending order
-  const int lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kGaussThreads / 32;
-  const int C = ((P + kWarps - 1) / kWarps + 31) / 32 * 32;
-  const int p0 = warp * C, p1 = min(P, p0 + C);
-  auto margin = [&](int p) {
-    double mg = -INFINITY;
-    for (int g = 0; g < G; ++g) {
-      const double m = static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - s_thr[g];
-      mg = fmax(mg, m);
-    }
-    return mg;
-  };
+  const int p0 = chunk * kFilterChunk + warp * kFilterPerWarp, p1 = min(P, p0 + kFilterPerWarp);
   double my_best = -INFINITY;
-  int my_idx = 0x7fffffff;
-  int wcount = 0;
+  int my_idx = 0x7fffffff, cnt = 0;
   for (int q0 = p0; q0 < p1; q0 += 32) {
     const int p = q0 + lane;
     bool keep = false;
     if (p < p1) {
-      const double mg = margin(p);
+      const double mg = page_margin(ws, fc, unit, G, max_pages, p);
       keep = mg > 0.0;
       if (mg > my_best) {
         my_best = mg;
         my_idx = p;
       }
     }
-    wcount += __popc(__ballot_sync(0xffffffffu, keep));
+    cnt += __popc(__ballot_sync(0xffffffffu, keep));
   }
-  if (lane == 0) scan_scratch[warp] = wcount;
-  __syncthreads();
-  int before = 0, carry = 0;
-  for (int w = 0; w < kWarps; ++w) {
-    before += w < warp ? scan_scratch[w] : 0;
-    carry += scan_scratch[w];
-  }
-  if (wcount > 0) {
-    int pos = before;
-    for (int q0 = p0; q0 < p1; q0 += 32) {
-      const int p = q0 + lane;
-      const bool keep = p < p1 && margin(p) > 0.0;
-      const unsigned int bal = __ballot_sync(0xffffffffu, keep);
-      const int at = pos + __popc(bal & ((1u << lane) - 1u));
-      if (keep && at < cap) out[at] = p;
-      pos += __popc(bal);
-    }
-  }
-  if (carry > 0) {
-    if (tid == 0) {
-      n_sel[unit] = min(carry, cap);
-      if (carry > cap) raise_flag(EKV_EFLAG_SEL_OVERFLOW);
-    }
-    return;
-  }
-  // fallback: the single page with the largest margin, lowest index on ties
   for (int o = 16; o > 0; o >>= 1) {
     const double om = __shfl_xor_sync(0xffffffffu, my_best, o);
     const int oi = __shfl_xor_sync(0xffffffffu, my_idx, o);
@@ -323,25 +352,101 @@ __global__ void __launch_bounds__(kGaussThreads)
     }
   }
   if (lane == 0) {
-    best_m[warp] = my_best;
-    best_i[warp] = my_idx;
+    fc.scan[warp] = cnt;
+    fc.best_m[warp] = my_best;
+    fc.best_i[warp] = my_idx;
   }
   __syncthreads();
   if (tid == 0) {
+    int total = 0;
     double bm = -INFINITY;
     int bi = 0x7fffffff;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-      if (best_m[w] > bm || (best_m[w] == bm && best_i[w] < bi)) {
-        bm = best_m[w];
-        bi = best_i[w];
+    for (int w = 0; w < kGaussThreads / 32; ++w) {
+      total += fc.scan[w];
+      if (fc.best_m[w] > bm || (fc.best_m[w] == bm && fc.best_i[w] < bi)) {
+        bm = fc.best_m[w];
+        bi = fc.best_i[w];
       }
     }
-    if (P > 0 && bi < P) {
-      out[0] = bi;
-      n_sel[unit] = 1;
-    } else {
-      n_sel[unit] = 0;
+    const size_t at = static_cast<size_t>(unit) * ws.nchunk + chunk;
+    ws.fcount[at] = total;
+    ws.fbest[at] = bm;
+    ws.fbest_at[at] = bi;
+  }
+}
+
+__global__ void __launch_bounds__(kGaussThreads)
+    gauss_write_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages, int Hkv, int G,
+                       double delta, int cap, int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
+  grid_dep_enter();
+  const int chunk = blockIdx.x, unit = blockIdx.y, b = unit / Hkv, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  int L;
+  const int P = seq_pages(seq_lens, b, S, max_pages, &L);
+  __shared__ FilterCtx fc;
+  __shared__ int s_before, s_total;
+  if (tid < G) fc.thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
+  if (warp == 0) {
+    // kept pages of the earlier chunks, and of all chunks
+    int before = 0, total = 0;
+    for (int c = lane; c < ws.nchunk; c += 32) {
+      const int n = ws.fcount[static_cast<size_t>(unit) * ws.nchunk + c];
+      before += c < chunk ? n : 0;
+      total += n;
     }
+    before = warp_sum(before);
+    total = warp_sum(total);
+    if (lane == 0) {
+      s_before = before;
+      s_total = total;
+    }
+  }
+  __syncthreads();
+  int32_t* out = sel + static_cast<size_t>(unit) * cap;
+  const int total = s_total;
+  if (total == 0) {
+    // fallback: the page of largest margin over every chunk, lowest index on ties
+    if (chunk == 0 && tid == 0) {
+      double bm = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int c = 0; c < ws.nchunk; ++c) {
+        const size_t at = static_cast<size_t>(unit) * ws.nchunk + c;
+        if (ws.fbest[at] > bm || (ws.fbest[at] == bm && ws.fbest_at[at] < bi)) {
+          bm = ws.fbest[at];
+          bi = ws.fbest_at[at];
+        }
+      }
+      if (P > 0 && bi < P) {
+        out[0] = bi;
+        n_sel[unit] = 1;
+      } else {
+        n_sel[unit] = 0;
+      }
+    }
+    return;
+  }
+  if (chunk == 0 && tid == 0) {
+    n_sel[unit] = min(total, cap);
+    if (total > cap) raise_flag(EKV_EFLAG_SEL_OVERFLOW);
+  }
+  const int p0 = chunk * kFilterChunk + warp * kFilterPerWarp, p1 = min(P, p0 + kFilterPerWarp);
+  int cnt = 0;
+  for (int q0 = p0; q0 < p1; q0 += 32) {
+    const int p = q0 + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, p < p1 && page_margin(ws, fc, unit, G, max_pages, p) > 0.0));
+  }
+  if (lane == 0) fc.scan[warp] = cnt;
+  __syncthreads();
+  int pos = s_before;
+  for (int w = 0; w < warp; ++w) pos += fc.scan[w];
+  if (cnt == 0) return;
+  for (int q0 = p0; q0 < p1; q0 += 32) {
+    const int p = q0 + lane;
+    const bool keep = p < p1 && page_margin(ws, fc, unit, G, max_pages, p) > 0.0;
+    const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+    const int at = pos + __popc(bal & ((1u << lane) - 1u));
+    if (keep && at < cap) out[at] = p;
+    pos += __popc(bal);
   }
 }
 
@@ -352,18 +457,45 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
                                 int32_t* n_sel, float* tau_hat, cudaStream_t st) {
   const int Hkv = c.num_kv_heads, G = Hq / Hkv, U = s.batch * Hkv;
   const int beta = static_cast<int>(lrint(1.0 / (static_cast<double>(alpha) - 1.0)));
-  {
-    const cudaError_t le_ = launch_k(gauss_tau_kernel, U * G, kTauThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
-                                                    G, Hq, beta, tau_hat);
-    if (le_ != cudaSuccess) return le_;
-  }
-  cudaError_t e = cudaGetLastError();
+  // CTAs per head: one up to 8192 pages (a cluster's barrier per step costs
+  // more than it saves there), else enough to give the B200's SMs two CTAs
+  // each, at most kTauMaxCluster
+  const int rows = U * G;
+  int C = 1;
+  while (C < kTauMaxCluster && s.max_pages > 8192 && rows * C * 2 <= 2 * 148) C *= 2;
+  const size_t smem = 3 * kGaussCand * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(gauss_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   {
-    const cudaError_t le_ = launch_k(gauss_filter_kernel, U, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv,
-                                                   G, static_cast<double>(delta), cap, sel, n_sel);
-    if (le_ != cudaSuccess) return le_;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(C), static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(kTauThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, gauss_tau_kernel, ws, s.seq_lens, c.page_size, s.max_pages, Hkv, G, Hq, beta,
+                           tau_hat);
+    if (e != cudaSuccess) return e;
   }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 fgrid(static_cast<unsigned>(ws.nchunk), static_cast<unsigned>(U));
+  e = launch_k(gauss_count_kernel, fgrid, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv, G,
+               static_cast<double>(delta));
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_k(gauss_write_kernel, fgrid, kGaussThreads, 0, st, ws, s.seq_lens, c.page_size, s.max_pages, Hkv, G,
+               static_cast<double>(delta), cap, sel, n_sel);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

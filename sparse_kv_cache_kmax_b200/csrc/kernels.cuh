@@ -25,11 +25,19 @@ struct DecodeWs {
 };
 
 
+// Pages per CTA of the Gaussian filter.
+constexpr int kFilterChunk = 1024;
+inline int filter_chunks(int max_pages) { return (max_pages + kFilterChunk - 1) / kFilterChunk; }
+
 struct GaussWs {
   float* mu;        // [U, G, max_pages] (α−1)·m
   float* sig;       // [U, G, max_pages] (α−1)·s
   float* hat;       // [U, G, max_pages] (α−1)·ŝ
   double* tau_hat;  // [U, G]
+  int* fcount;      // [U, nchunk] pages kept per filter chunk
+  double* fbest;    // [U, nchunk] the chunk's largest margin
+  int* fbest_at;    // [U, nchunk] its page (lowest on ties)
+  int nchunk;
 };
 
 cudaError_t launch_build_meta(const ekv_cache& c, const ekv_seqs& s, cudaStream_t st);

@@ -128,3 +128,6 @@ def test_step_kernel_count_host_side():
     assert L.ekv_step_kernel_count(ctypes.byref(f32), ctypes.byref(s), ctypes.byref(topk), 32) == 6
     full = B.StepParams(B.EKV_POLICY_FULL, 0, 0.5, 4, 1.5, 0.1, 0, 0)
     assert L.ekv_step_kernel_count(ctypes.byref(f32), ctypes.byref(s), ctypes.byref(full), 32) == 3
+    # Gaussian policy: page statistics, τ̂, filter count and filter write
+    gauss = B.StepParams(B.EKV_POLICY_GAUSS, 0, 0.5, 4, 1.5, 0.1, 0, 1)
+    assert L.ekv_step_kernel_count(ctypes.byref(f32), ctypes.byref(s), ctypes.byref(gauss), 32) == 1 + 4 + 3
