@@ -192,8 +192,9 @@ __device__ __noinline__ double repair_closed_tau(const float* cand, int nc, int 
   return tau;
 }
 
-// Newton's method from the left in fp32 (f is convex and decreasing), then a
-// float64 finish: the closed form for β ∈ {1,2}, one Newton step otherwise.
+// Newton's method from the left in fp32 on the ℓ_β norm of (u − τ)_+ (convex
+// and decreasing), then a float64 finish: the closed form for β ∈ {1,2}, one
+// Newton step otherwise.
 __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_lo, float um,
                                           float beta, int ipow, TauShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -266,8 +267,8 @@ __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_
 //     every candidate at once; τ is the float64 closed form on that support,
 //     kept if the support it implies is the same, else refined by repeating
 //     the closed form on {u > τ}.  Otherwise Newton's method from the left in
-//     fp32 (f is convex and decreasing) and a float64 finish: the closed form
-//     for β ∈ {1,2}, one float64 Newton step otherwise.
+//     fp32 on the ℓ_β norm of (u − τ)_+ (convex and decreasing) and a float64
+//     finish: the closed form for β ∈ {1,2}, one float64 Newton step otherwise.
 // Returns the fp32 τ every later step uses.
 __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, float am1, float beta,
                                int ipow, TauShared& sh) {
@@ -506,31 +507,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     if (lane < C) cluster.map_shared_rank(&mall[0][0], lane)[h * kFMaxCluster + rank] = m;
   }
   cluster.sync();
-  // Every support token has u > max u − 1 for its head (its weight is at
-  // most 1): the V rows of those candidates are brought into L2 now, so the
-  // V pass after τ finds them there
-  if (!a.dense_v) {
-    float lo[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float m = -INFINITY;
-      for (int r = 0; r < C; ++r) m = fmaxf(m, mall[h][r]);
-      lo[h] = a.am1 * m - 1.0f;
-    }
-    for (int x = tid; x < np * S; x += kFThreads) {
-      const int j = x / S;
-      bool cand = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) cand |= a.am1 * zs[h * zp + x] > lo[h];
-      if (cand && phys_s[j] >= 0 && x - j * S < nv_s[j]) {
-        const bf16* src = static_cast<const bf16*>(a.v_pool) +
-                          ((static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * S + (x - j * S)) * D;
-#pragma unroll
-        for (int c = 0; c < D * 2; c += 128) prefetch_l2(reinterpret_cast<const unsigned char*>(src) + c);
-      }
-    }
-  }
-
   // ---------------------------------------------------------------- 2. τ
   const int tpc = spc * S;
   const int n_tok = n_slots * S;

@@ -7,7 +7,9 @@
 //     tensor-core A fragments) for the G query heads of its unit, and writes
 //     the scores z, the chunk's per-head maxima and the physical page of each
 //     selected slot to an L2-resident scratch.
-//  2. head_decode_kernel, one CTA of 256 threads per query head: the head's
+//  2. head_warp_kernel, one warp per query head, when the selection holds at
+//     most 512 tokens (below); otherwise head_decode_kernel, one CTA of 256
+//     threads per query head (1024 when streaming): the head's
 //     scores u = (α−1)·z sit in registers (VPT per thread; above 16384
 //     selected tokens they are read again from L2 at each pass); a 256-bin
 //     histogram of u over (max u − 1, max u] brackets τ from the left (c
@@ -16,8 +18,9 @@
 //     β ∈ {1, 2} and few candidates the support is found by testing every
 //     candidate at once (u_j is in the support iff
 //     Σ_i (u_i − u_j)_+^β < 1) and τ is the float64 closed form on it,
-//     otherwise Newton's method from the left (f is convex and decreasing;
-//     one warp alone when the candidates are few) with a float64 finish.  The
+//     otherwise Newton's method from the left on the ℓ_β norm of (u − τ)_+
+//     (convex and decreasing; one warp alone when the candidates are few)
+//     with a float64 finish.  The
 //     head's support tokens are then compacted and only their V rows are
 //     read, eight rows in flight per warp; warp partials are summed in warp
 //     order.
@@ -617,9 +620,190 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   }
 }
 
+// ------------------------------------------------------------------ 2'. one warp per head
+// For selections of at most 32·VPL tokens a whole query head fits one warp
+// (VPL values per lane, token k·32 + lane), and the head needs no block
+// barrier at all: Newton's method on the ℓ_β norm over every value from
+// max u − 1 (where the sum is ≥ 1), the float64 closed form on the support
+// for β ∈ {1, 2} (one float64 Newton step otherwise), the support's bits by
+// ballots, its tokens and weights listed in token order in the warp's
+// shared memory, then its V rows, eight in flight, each lane summing its own
+// output columns.
+template <int VPL>
+constexpr int head_warps() {
+  return 8;
+}
+
+template <int D, int VPL>
+__global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(DecodeArgs a, int G, int rows) {
+  constexpr int kWarps = head_warps<VPL>();
+  constexpr int DPL = D / 32;
+  __shared__ float s_p[kWarps][32 * VPL];
+  __shared__ int s_i[kWarps][32 * VPL];
+  grid_dep_enter();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * kWarps + warp;
+  if (row >= rows) return;  // warp-uniform, and no block barrier follows
+  const int unit = row / G, hg = row - unit * G, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int S = a.S;
+  int L;
+  const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
+  const int n = unit_slots(a, unit, P) * S;
+  const size_t orow = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * G + hg;
+  const float* z = a.ws.zbuf + static_cast<size_t>(row) * a.cap * S;
+  const float am1 = a.am1, beta = a.beta;
+  const int ipow = a.ipow;
+  float u[VPL];
+  float m = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int i = k * 32 + lane;
+    u[k] = i < n ? am1 * __ldcg(z + i) : -INFINITY;
+    m = fmaxf(m, u[k]);
+  }
+  m = warp_max(m);
+
+  float tau = INFINITY;  // no finite score: no support, zero output
+  if (m > -INFINITY) {
+    float t = m - 1.0f;
+    for (int it = 0; it < 100; ++it) {
+      float x = 0.f, y = 0.f;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const float w = u[k] - t;
+        if (w > 0.f) {
+          const float wb1 = hd_pow_bm1<float>(w, beta, ipow);
+          x += wb1 * w;
+          y += wb1;
+        }
+      }
+      x = warp_sum(x);
+      y = warp_sum(y);
+      const float step = norm_newton_step<float>(x - 1.0f, y, beta);
+      if (!(step > 0.0f)) break;
+      t += step;
+      if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+    }
+    double d = t;
+    if (ipow == 1 || ipow == 2) {
+      // the closed form on {u > τ}, repeated while the support it implies moves
+      for (int rep = 0; rep < 4; ++rep) {
+        double c = 0.0, s1 = 0.0, s2 = 0.0;
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+          const double uu = u[k];
+          if (uu > d) {
+            c += 1.0;
+            s1 += uu;
+            s2 += uu * uu;
+          }
+        }
+        c = warp_sum(c);
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (c < 1.0) break;
+        const double t_new = hd_closed_tau(ipow, c, s1, s2);
+        if (t_new == d) break;
+        d = t_new;
+      }
+    } else {
+      double x = 0.0, y = 0.0;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const double w = static_cast<double>(u[k]) - d;
+        if (w > 0.0) {
+          const double wb1 = hd_pow_bm1<double>(w, static_cast<double>(beta), ipow);
+          x += wb1 * w;
+          y += wb1;
+        }
+      }
+      x = warp_sum(x);
+      y = warp_sum(y);
+      if (y > 0.0) d += (x - 1.0) / (static_cast<double>(beta) * y);
+    }
+    tau = static_cast<float>(d);
+  }
+
+  // support: bits by ballots (word k holds tokens k·32 …), list in token order
+  int ns = 0;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int i = k * 32 + lane;
+    const bool in = i < n && u[k] > tau;
+    const unsigned int bal = __ballot_sync(0xffffffffu, in);
+    if (a.bits_out && lane == 0 && k < a.words) a.bits_out[orow * a.words + k] = bal;
+    if (in) {
+      const int at = ns + __popc(bal & ((1u << lane) - 1u));
+      s_p[warp][at] = pow_beta_fast(u[k] - tau, beta, ipow);
+      s_i[warp][at] = i;
+    }
+    ns += __popc(bal);
+  }
+  if (a.bits_out)
+    for (int w = VPL + lane; w < a.words; w += 32) a.bits_out[orow * a.words + w] = 0u;
+  if (lane == 0) {
+    if (a.tau_out) a.tau_out[orow] = tau;
+    if (a.count_out) a.count_out[orow] = ns;
+    if (a.dense_v) a.ws.taus[row] = tau;
+  }
+  if (a.dense_v) return;  // every V row is read by the V pass that follows
+  __syncwarp();
+
+  float acc[DPL];
+#pragma unroll
+  for (int x = 0; x < DPL; ++x) acc[x] = 0.f;
+  for (int e0 = 0; e0 < ns; e0 += kHdRows) {
+    float v[kHdRows][DPL];
+    float p[kHdRows];
+#pragma unroll
+    for (int r = 0; r < kHdRows; ++r) {
+      const int e = e0 + r;
+      p[r] = 0.f;
+#pragma unroll
+      for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
+      if (e < ns) {
+        const int tok = s_i[warp][e];
+        const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
+        if (ph >= 0) {
+          p[r] = s_p[warp][e];
+          const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                            ((static_cast<size_t>(ph) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(src);
+            v[r][0] = __uint_as_float(w2.x << 16);
+            v[r][1] = __uint_as_float(w2.x & 0xffff0000u);
+            v[r][2] = __uint_as_float(w2.y << 16);
+            v[r][3] = __uint_as_float(w2.y & 0xffff0000u);
+          } else {
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
+            v[r][0] = __uint_as_float(w1 << 16);
+            v[r][1] = __uint_as_float(w1 & 0xffff0000u);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kHdRows; ++r)
+#pragma unroll
+      for (int x = 0; x < DPL; ++x) acc[x] = fmaf(p[r], v[r][x], acc[x]);
+  }
+#pragma unroll
+  for (int x = 0; x < DPL; ++x) a.out[orow * D + lane * DPL + x] = acc[x];
+}
+
 template <int D>
 cudaError_t launch_head_decode(DecodeArgs& a, int rows, int G, cudaStream_t st) {
   const int n_max = a.cap * a.S;
+#define EKV_HW_CASE(VV)                                                                                    \
+  if (n_max <= 32 * (VV)) {                                                                                \
+    constexpr int W = head_warps<VV>();                                                                    \
+    const cudaError_t e =                                                                                  \
+        launch_k(head_warp_kernel<D, VV>, dim3((rows + W - 1) / W), dim3(32 * W), 0, st, a, G, rows);      \
+    if (e != cudaSuccess) return e;                                                                        \
+    return cudaGetLastError();                                                                             \
+  }
+  EKV_HW_CASE(4) EKV_HW_CASE(8) EKV_HW_CASE(16)
+#undef EKV_HW_CASE
 #define EKV_HD_CASE(VV)                                                                                      \
   if (n_max <= (VV) * kHdThreads) {                                                                          \
     const cudaError_t e = launch_k(head_decode_kernel<D, VV, kHdThreads>, dim3(rows), dim3(kHdThreads), 0, st, a, G); \

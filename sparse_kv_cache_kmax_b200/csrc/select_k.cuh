@@ -57,17 +57,17 @@ struct ListKeys {
 };
 
 
-template <int THREADS, int BINS>
+template <int THREADS, int BINS, int LIST = 8192>
 struct Select {
   static constexpr int kTopkThreads = THREADS;
   static constexpr int kTopkWarps = THREADS / 32;
-  static constexpr int kKeysPerThread = 8192 / THREADS;            // registers per thread for lists ≤ 8192
+  static constexpr int kKeysPerThread = LIST / THREADS;            // registers per thread for lists ≤ LIST
   static constexpr int kRegKeys = 2 * kKeysPerThread * THREADS;    // longest list held in registers
   static constexpr int kBins = BINS;
   static constexpr int kDigitBits = BINS == 4096 ? 12 : (BINS == 2048 ? 11 : 10);
   static constexpr int kRankMax = 256;  // keys of the k-th key's bin ranked directly
   static_assert(THREADS >= kRankMax && THREADS <= 1024 && THREADS % 32 == 0, "block size");
-  static_assert(BINS % THREADS == 0 && 8192 % THREADS == 0 && (1 << kDigitBits) == BINS, "bins and keys per thread");
+  static_assert(BINS % THREADS == 0 && LIST % THREADS == 0 && (1 << kDigitBits) == BINS, "bins and keys per thread");
 
 struct SelectShared {
   unsigned int hist[2][kBins];

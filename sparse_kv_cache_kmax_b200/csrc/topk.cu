@@ -31,24 +31,30 @@ constexpr int kTopkThreads = Sel::kTopkThreads;
 constexpr int kRegKeys = Sel::kRegKeys;
 constexpr int kChunk = 8192;                  // pages per first-stage chunk of a long unit
 
+// Short lists (at most kShortList pages per sequence): 256 threads, 4 keys
+// each, 1024 bins, so that many units' CTAs are resident at once.
+using SelShort = Select<256, 1024, 1024>;
+constexpr int kShortList = SelShort::kKeysPerThread * SelShort::kTopkThreads;
+
 // One unit per CTA.
-__global__ void __launch_bounds__(kTopkThreads)
+template <class SelT>
+__global__ void __launch_bounds__(SelT::kTopkThreads)
     topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int S,
                 int max_pages, int Hkv, int k, int stride, int32_t* __restrict__ sel,
                 int32_t* __restrict__ n_sel) {
   grid_dep_enter();
-  __shared__ SelectShared sh;
+  __shared__ typename SelT::SelectShared sh;
   const int unit = blockIdx.x, b = unit / Hkv, tid = threadIdx.x;
   int L;
   const int P = seq_pages(seq_lens, b, S, max_pages, &L);
   int32_t* out = sel + static_cast<size_t>(unit) * stride;
   const float* row = ub + static_cast<size_t>(unit) * max_pages;
   if (P <= k) {
-    for (int i = tid; i < P; i += kTopkThreads) out[i] = i;
+    for (int i = tid; i < P; i += SelT::kTopkThreads) out[i] = i;
     if (tid == 0) n_sel[unit] = P;
     return;
   }
-  Sel::select_k(sh, P, k, RowKeys{row}, [](int i) { return i; }, out, n_sel + unit);
+  SelT::select_k(sh, P, k, RowKeys{row}, [](int i) { return i; }, out, n_sel + unit);
 }
 
 // First stage of a long unit: chunk c keeps its k best pages.
@@ -171,8 +177,12 @@ cudaError_t launch_topk(const ekv_seqs& s, int Hkv, int S, const float* ub, int 
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  const cudaError_t le = launch_k(topk_kernel, dim3(U), dim3(kTopkThreads), 0, st, ub,
-                                  s.seq_lens, S, s.max_pages, Hkv, k, stride, sel, n_sel);
+  const cudaError_t le =
+      s.max_pages <= kShortList
+          ? launch_k(topk_kernel<SelShort>, dim3(U), dim3(SelShort::kTopkThreads), 0, st, ub, s.seq_lens, S,
+                     s.max_pages, Hkv, k, stride, sel, n_sel)
+          : launch_k(topk_kernel<Sel>, dim3(U), dim3(kTopkThreads), 0, st, ub, s.seq_lens, S, s.max_pages, Hkv, k,
+                     stride, sel, n_sel);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
