@@ -46,8 +46,8 @@ FALLBACK_HBM_GBS = 6650.0
 # changed kernel has no measured traffic until it is captured again)
 SCORE_FILES = ("score.cu", "common.cuh")
 DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh")
-SCORE_TRAFFIC = {"9d59cbe25c63e9dc": 137794048}
-DECODE_TRAFFIC = {"851e2059314083b4": 35284480}
+SCORE_TRAFFIC = {"2ac4280b73b40cfc": 135471616}
+DECODE_TRAFFIC = {"946920e13b39ee83": 35248384}
 
 
 def kernel_hash(files=SCORE_FILES):
@@ -442,6 +442,27 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(result))
+
+
+def run_line(args):
+    """One line of the default run alone (one policy on one workload), on the
+    workload's own inputs: the command the per-line ncu summaries use."""
+    from sparse_kv_cache_kmax_b200 import binding as Bd
+    from sparse_kv_cache_kmax_b200.workloads import WORKLOADS, make_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Bd.lib()
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, seed=3000, device=dev, n_new=1)
+    flush = L2Flush(dev)
+    peak, _ = hbm_peak()
+    policy = {"topk": "topk", "gauss": "gauss", "full": "full", "dense": "full"}[args.line]
+    kw = {"k": args.k or wl.topk} if policy == "topk" else (
+        {"delta": wl.delta if wl.delta is not None else 0.5} if policy == "gauss" else {"dense_v": args.line == "dense"})
+    ln = Line(wl, inp, policy, args.alpha, dev, flush, **kw)
+    m = ln.measure(args.steps, args.warmup, peak)
+    print(json.dumps(dict(short_line(m), line=args.line, workload=wl.name, alpha=args.alpha)))
 
 
 # (workload, policy, alpha, budget) of the other lines in the default run
@@ -839,6 +860,8 @@ def main(argv=None):
                    help="time one stage alone on inputs holding only what it reads ('copy': a plain "
                         "device copy of the stage's bytes, for reference)")
     p.add_argument("--shape", default="", help="kernel mode: override 'batch,q_heads,kv_heads'")
+    p.add_argument("--line", choices=["topk", "gauss", "full", "dense"],
+                   help="run one line of the default output alone: this policy on --workload")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")
@@ -846,6 +869,8 @@ def main(argv=None):
         run_reference(args)
     elif args.kernel:
         run_kernel(args)
+    elif args.line:
+        run_line(args)
     else:
         run_ours(args)
 

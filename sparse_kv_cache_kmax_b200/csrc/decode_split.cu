@@ -45,7 +45,7 @@ constexpr int kHdBins = 256;
 constexpr int kHdCand = 2048;              // candidates / support tokens held in shared memory at once
 constexpr int kHdPairMax = 256;            // candidates for the all-at-once support test
 constexpr int kHdRows = 8;                 // V rows in flight per warp
-constexpr int kHdBatch = 8;                // score loads in flight per thread when streaming
+constexpr int kHdBatch = 4;                // 16-byte score loads in flight per thread when streaming
 constexpr int kHdMaxVpt = 64;              // values per thread held in registers (more: read per pass)
 constexpr int kSplitMaxTokens = 1 << 20;   // selected tokens per unit on this path
 static_assert(kHdBins <= kHdThreads, "one histogram bin per thread");
@@ -221,10 +221,13 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   const float am1 = a.am1, beta = a.beta;
   const int ipow = a.ipow;
 
-  // value k of this thread is token i = k·256 + tid: held in registers
-  // (VPT > 0), or read again from the scratch at every pass (VPT == 0)
+  // value k of this thread: held in registers (VPT > 0) as token
+  // k·THREADS + tid, or read again from the scratch at every pass (VPT == 0)
+  // four consecutive tokens per 16-byte load: token 4·((k/4)·THREADS + tid) +
+  // k mod 4 (tok(k) gives it)
   constexpr bool kReg = VPT > 0;
-  const int NK = kReg ? VPT : (n + THREADS - 1) / THREADS;
+  const int NK = kReg ? VPT : 4 * ((n + 4 * THREADS - 1) / (4 * THREADS));
+  auto tok = [&](int k) { return kReg ? k * THREADS + tid : 4 * ((k >> 2) * THREADS + tid) + (k & 3); };
   float uv[kReg ? VPT : 1];
   if constexpr (kReg) {
 #pragma unroll
@@ -234,23 +237,31 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
     }
   }
   // fn(k, u) for every value of this thread in order of k; read from the
-  // scratch in batches of kHdBatch independent loads when not in registers
-  // (fn may hold warp collectives: k runs alike on every lane)
+  // scratch in batches of kHdBatch independent 16-byte loads when not in
+  // registers (n is a multiple of 4, so a load starting below n stays in
+  // the row; fn may hold warp collectives: k runs alike on every lane)
   auto for_values = [&](auto fn) {
     if constexpr (kReg) {
 #pragma unroll
       for (int k = 0; k < VPT; ++k) fn(k, uv[k]);
     } else {
-      for (int k0 = 0; k0 < NK; k0 += kHdBatch) {
-        float v[kHdBatch];
+      for (int q0 = 0; q0 < NK / 4; q0 += kHdBatch) {
+        float4 v[kHdBatch];
 #pragma unroll
         for (int j = 0; j < kHdBatch; ++j) {
-          const int i = (k0 + j) * THREADS + tid;
-          v[j] = (k0 + j < NK && i < n) ? am1 * __ldcg(z + i) : -INFINITY;
+          const int i = 4 * ((q0 + j) * THREADS + tid);
+          v[j] = (q0 + j < NK / 4 && i < n) ? __ldcg(reinterpret_cast<const float4*>(z + i))
+                                            : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         }
 #pragma unroll
         for (int j = 0; j < kHdBatch; ++j)
-          if (k0 + j < NK) fn(k0 + j, v[j]);
+          if (q0 + j < NK / 4) {
+            const int k = 4 * (q0 + j);
+            fn(k, am1 * v[j].x);
+            fn(k + 1, am1 * v[j].y);
+            fn(k + 2, am1 * v[j].z);
+            fn(k + 3, am1 * v[j].w);
+          }
       }
     }
   };
@@ -303,7 +314,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
         for_values([&](int k, float u) {
           if (u > tlo) {
             sh.cu[p] = u;
-            sh.ci[p] = k * THREADS + tid;
+            sh.ci[p] = tok(k);
             ++p;
           }
         });
@@ -497,11 +508,11 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   //    passes over every value and the bits come from ballots.
   auto compact = [&](int base) {
     int mine = 0;
-    for_values([&](int k, float u) { mine += (k * THREADS + tid < n && u > tau) ? 1 : 0; });
+    for_values([&](int k, float u) { mine += (tok(k) < n && u > tau) ? 1 : 0; });
     int ns;
     int p = block_exclusive_scan(mine, sh.i, &ns) - base;
     for_values([&](int k, float u) {
-      const int i = k * THREADS + tid;
+      const int i = tok(k);
       if (i < n && u > tau) {
         if (p >= 0 && p < kHdCand) {
           sh.cu[p] = pow_beta_fast(u - tau, beta, ipow);
@@ -546,7 +557,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
         const int i = sh.ci[e];
         atomicOr(&a.bits_out[orow * a.words + (i >> 5)], 1u << (i & 31));
       }
-  } else {
+  } else if (kReg) {
     if (a.bits_out)
       for_values([&](int k, float u) {
         const int i = k * THREADS + tid;
@@ -555,8 +566,20 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
       });
     ns = compact(0);
     if (a.bits_out)
-      for (int w = ((kReg ? VPT : NK) * THREADS) / 32 + tid; w < a.words; w += THREADS)
+      for (int w = (VPT * THREADS) / 32 + tid; w < a.words; w += THREADS)
         a.bits_out[orow * a.words + w] = 0u;  // words past the ballots above
+  } else {
+    // streamed values: a warp's lanes hold tokens four apart, so the bits
+    // are set one token at a time after the row is cleared
+    if (a.bits_out) {
+      for (int w = tid; w < a.words; w += THREADS) a.bits_out[orow * a.words + w] = 0u;
+      __syncthreads();
+      for_values([&](int k, float u) {
+        const int i = tok(k);
+        if (i < n && u > tau) atomicOr(&a.bits_out[orow * a.words + (i >> 5)], 1u << (i & 31));
+      });
+    }
+    ns = compact(0);
   }
   if (tid == 0) {
     if (a.tau_out) a.tau_out[orow] = tau;
