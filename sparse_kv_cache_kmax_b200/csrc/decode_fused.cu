@@ -194,13 +194,15 @@ __device__ __noinline__ double repair_closed_tau(const float* cand, int nc, int 
 
 // Newton's method from the left in fp32 on the ℓ_β norm of (u − τ)_+ (convex
 // and decreasing), then a float64 finish: the closed form for β ∈ {1,2}, one
-// Newton step otherwise.
+// Newton step otherwise.  Up to kSoloMax candidates one warp iterates alone
+// (no barrier per step); above that the CTA does, one barrier per step.
+constexpr int kSoloMax = 128;
 __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_lo, float um,
                                           float beta, int ipow, TauShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool closed = ipow == 1 || ipow == 2;
   double tau;
-  const bool solo = nc <= 1024;
+  const bool solo = nc <= kSoloMax;
   if (!solo || warp == 0) {
     float t = static_cast<float>(tau_lo);
     if (static_cast<double>(t) > tau_lo) t = nextafterf(t, -INFINITY);
@@ -255,10 +257,33 @@ __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_
   return tau;
 }
 
-// τ of one query head: Σ_i [u_i − τ]_+^β = 1, u_i = (α−1)·z_i, over the n
-// scores z[0..n) in shared memory whose histogram over (um − 1, um] (um =
-// (α−1)·max z, 256 bins from the top) is in sh.hist.  The whole CTA calls it;
-// it leaves sh.hist zeroed.  cand: shared scratch of n floats.
+// τ of one query head without a closed form (β ∉ {1, 2}): Newton's method
+// from the left on the ℓ_β norm of (u − τ)_+ over all n values u in shared
+// memory, from max u − 1 (where the sum is ≥ 1: the maximum alone gives 1),
+// one pass and one barrier per step, then one float64 Newton step.  The
+// whole CTA calls it; it returns the fp32 τ every later step uses.
+__device__ float cta_newton_tau(const float* u, int n, float um, float beta, int ipow, TauShared& sh) {
+  float t = um - 1.0f;
+  int par = 1;
+  for (int it = 0; it < 64; ++it) {
+    float f, df;
+    par ^= 1;
+    f_df<float>(u, n, t, beta, ipow, false, sh, par, f, df);
+    const float step = norm_newton_step<float>(f, df, beta);
+    if (!(step > 0.0f)) break;
+    t += step;
+    if (step <= 2e-7f * fmaxf(1.0f, fabsf(t))) break;
+  }
+  double tau = t, f, df;
+  f_df<double>(u, n, tau, static_cast<double>(beta), ipow, false, sh, 0, f, df);
+  if (df > 0.0) tau += f / (static_cast<double>(beta) * df);
+  return static_cast<float>(tau);
+}
+
+// τ of one query head: Σ_i [u_i − τ]_+^β = 1 over the n values u[0..n) in
+// shared memory (argument z), whose histogram over (um − 1, um] (um = max u,
+// 256 bins from the top) is in sh.hist.  The whole CTA calls it; it leaves
+// sh.hist zeroed.  cand: shared scratch of n floats.
 //  1. Bracket: c values above an edge e force τ ≥ e − c^(−1/β) (c of them
 //     would already carry mass ≥ 1); the best edge gives τ_lo.
 //  2. The values above τ_lo are compacted (warp order, then scan order).
@@ -270,8 +295,8 @@ __device__ __noinline__ double newton_tau(const float* cand, int nc, double tau_
 //     fp32 on the ℓ_β norm of (u − τ)_+ (convex and decreasing) and a float64
 //     finish: the closed form for β ∈ {1,2}, one float64 Newton step otherwise.
 // Returns the fp32 τ every later step uses.
-__device__ float cta_solve_tau(const float* z, int n, float um, float* cand, float am1, float beta,
-                               int ipow, TauShared& sh) {
+__device__ float cta_solve_tau(const float* z, int n, float um, float* cand, float beta, int ipow,
+                               TauShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // 1. bracket, computed by every warp from the histogram (no barrier)
   float cb = um - 1.0f;
@@ -313,7 +338,7 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     int mine = 0;
     for (int base = 0; base < n; base += kFThreads) {
       const int i = base + tid;
-      const bool in = i < n && am1 * z[i] > tau_lo_f;
+      const bool in = i < n && z[i] > tau_lo_f;
       mine += __popc(__ballot_sync(0xffffffffu, in));
     }
     if (lane == 0) sh.i[warp] = mine;
@@ -328,7 +353,7 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
     }
     for (int base = 0; base < n; base += kFThreads) {
       const int i = base + tid;
-      const float u = i < n ? am1 * z[i] : -INFINITY;
+      const float u = i < n ? z[i] : -INFINITY;
       const bool in = i < n && u > tau_lo_f;
       const unsigned int bal = __ballot_sync(0xffffffffu, in);
       if (in) cand[pos + __popc(bal & ((1u << lane) - 1u))] = u;
@@ -339,8 +364,7 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
   }
   // 3. τ
   double tau;
-  const bool closed = ipow == 1 || ipow == 2;
-  if (closed && nc <= kPairwiseMax) {
+  if ((ipow == 1 || ipow == 2) && nc <= kPairwiseMax) {
     bool in = false;
     float ut = 0.f;
     double c = 0.0, s1 = 0.0, s2 = 0.0;
@@ -510,7 +534,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   // ---------------------------------------------------------------- 2. τ
   const int tpc = spc * S;
   const int n_tok = n_slots * S;
-  float* zh = reinterpret_cast<float*>(ring);
+  float* zh = reinterpret_cast<float*>(ring);  // u = (α−1)·z of the head being solved
+  const bool closed = a.ipow == 1 || a.ipow == 2;
   float* cand = zh + ((n_tok + 31) & ~31);
   const size_t words = static_cast<size_t>(a.words);
   for (int h = rank; h < G; h += C) {
@@ -523,15 +548,20 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
       for (int i = 4 * tid; i < n_tok; i += 4 * kFThreads) {
         const int r = i / tpc;
         const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(zs, r) + h * zp + (i - r * tpc));
-        *reinterpret_cast<float4*>(zh + i) = v;
         const float uu[4] = {a.am1 * v.x, a.am1 * v.y, a.am1 * v.z, a.am1 * v.w};
+        *reinterpret_cast<float4*>(zh + i) = make_float4(uu[0], uu[1], uu[2], uu[3]);
+        if (!closed) continue;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           if (uu[k] > um - 1.0f)
             atomicAdd(&tsh.hist[min(kTauBinsF - 1, static_cast<int>((um - uu[k]) * kTauBinsF))], 1);
       }
       __syncthreads();
-      tau = cta_solve_tau(zh, n_tok, um, cand, a.am1, a.beta, a.ipow, tsh);
+      // β ∈ {1, 2}: bracket, candidates, pairwise support test and closed
+      // form; otherwise Newton over every value from max u − 1 (f ≥ 0 there:
+      // the maximum alone gives 1), one barrier per step, without a bracket
+      tau = closed ? cta_solve_tau(zh, n_tok, um, cand, a.beta, a.ipow, tsh)
+                   : cta_newton_tau(zh, n_tok, um, a.beta, a.ipow, tsh);
     }
     if (tid < C) cluster.map_shared_rank(s_tau, tid)[h] = tau;
     if (tid == 0 && a.tau_out) a.tau_out[orow] = tau;
@@ -542,7 +572,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
     int cnt = 0;
     for (int base = 0; base < n_tok; base += kFThreads) {
       const int i = base + tid;
-      const bool in = i < n_tok && tau < INFINITY && a.am1 * zh[i] > tau;
+      const bool in = i < n_tok && tau < INFINITY && zh[i] > tau;
       cnt += in ? 1 : 0;
       const unsigned int bal = __ballot_sync(0xffffffffu, in);
       if (a.bits_out && lane == 0 && i < n_tok) a.bits_out[orow * words + i / 32] = bal;

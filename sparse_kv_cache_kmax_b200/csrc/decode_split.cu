@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
         f = x - V(1);
         df = y;
       };
-      const bool solo = listed && nc <= 1024;
+      const bool solo = listed && nc <= 128;  // one warp alone only when the candidates are few
       if (solo) {
         if (warp == 0) {
           float t = tlo;
