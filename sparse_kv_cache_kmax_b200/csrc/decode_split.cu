@@ -2,9 +2,10 @@
 // summary page (gist.science/fr/paper/2605.21649) §2.C "Attention Entmax
 // Parcimonieuse", with the support-only V read that §2–§3 make exact.
 //
-//  1. k_score_kernel, grid (chunks, units): every CTA scores one chunk of 256
-//     selected tokens (8 warps × 32 rows, straight from global memory into
-//     tensor-core A fragments) for the G query heads of its unit, and writes
+//  1. k_score_kernel, grid (CTAs per unit, units): every CTA scores chunks of
+//     256 selected tokens (8 warps × 32 rows, straight from global memory into
+//     tensor-core A fragments) for the G query heads of its unit, chunk after
+//     chunk up to the unit's own selection, and writes
 //     the scores z, the chunk's per-head maxima and the physical page of each
 //     selected slot to an L2-resident scratch.
 //  2. head_warp_kernel, one warp per query head, when the selection holds at
@@ -29,6 +30,8 @@
 // after τ and the V pass of the three-kernel decode reads every valid row
 // once for all heads of the unit (pv_kernel, decode.cu).  Every sum has a
 // fixed order, so results are deterministic.
+#include <algorithm>
+
 #include "decode.cuh"
 
 namespace ekv {
@@ -59,95 +62,99 @@ __global__ void __launch_bounds__(kKsThreads, 2) k_score_kernel(DecodeArgs a) {
   // only at the end (its CTAs hold many registers: resident early, they
   // would crowd this launch's CTAs off the SMs)
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int split = blockIdx.x, unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int unit = blockIdx.y, b = unit / a.Hkv, kvh = unit % a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int S = a.S;
   int L;
   const int P = seq_pages(a.seq_lens, b, S, a.max_pages, &L);
   const int n_slots = unit_slots(a, unit, P);
-  const int ppc = kKsTokens / S;  // pages per CTA
-  const int s_begin = split * ppc;
-  if (split == 0 && tid == 0) a.ws.counter[unit] = 0;  // the dense V pass's ticket
-  if (s_begin >= n_slots) return;  // CTA-uniform
-  if (tid < G) cta_key[tid] = 0u;
-  const int row0 = warp * 32;
-  int phys[2], nv[2], slot[2];
-  bool live[2];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-    const int r = row0 + mt * 16;
-    slot[mt] = s_begin + r / S;
-    live[mt] = slot[mt] < n_slots;
-    phys[mt] = -1;
-    nv[mt] = 0;
-    if (live[mt]) phys[mt] = slot_page(a, unit, b, slot[mt], P, L, &nv[mt]);
-  }
-  uint4 va[2][KP], vb[2][KP];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-    const int tok0 = (row0 + mt * 16) % S;
-    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
-    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
-    const bf16* kb = static_cast<const bf16*>(a.k_pool) +
-                     ((static_cast<size_t>(phys[mt] < 0 ? 0 : phys[mt]) * a.Hkv + kvh) * S + tok0) * D;
-    const uint4* row_lo = reinterpret_cast<const uint4*>(kb + g * D) + t;
-    const uint4* row_hi = reinterpret_cast<const uint4*>(kb + (g + 8) * D) + t;
-#pragma unroll
-    for (int c = 0; c < KP; ++c) {
-      va[mt][c] = ok_lo ? __ldcs(row_lo + 4 * c) : make_uint4(0, 0, 0, 0);
-      vb[mt][c] = ok_hi ? __ldcs(row_hi + 4 * c) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  // the physical page of each selected slot, for the V pass
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-    if (lane == 0 && live[mt] && (row0 + mt * 16) % S == 0)
-      a.ws.sphys[static_cast<size_t>(unit) * a.cap + slot[mt]] = phys[mt];
+  const int ppc = kKsTokens / S;  // pages per chunk
+  if (blockIdx.x == 0 && tid == 0) a.ws.counter[unit] = 0;  // the dense V pass's ticket
   uint32_t bfrag[2 * KP][NT][2];
   load_q_frags<D, G>(a, b, kvh, g, t, bfrag);
-  __syncthreads();  // cta_key initialised
   const size_t zrow_len = static_cast<size_t>(a.cap) * S;
-  float wmax[NT][2];
+  // CTA x takes chunks x, x + gridDim.x, …: the grid is sized for the cap,
+  // the loop stops at the unit's own selection
+  for (int split = blockIdx.x; split * ppc < n_slots; split += gridDim.x) {
+    const int s_begin = split * ppc;
+    if (tid < G) cta_key[tid] = 0u;
+    const int row0 = warp * 32;
+    int phys[2], nv[2], slot[2];
+    bool live[2];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) wmax[nt][0] = wmax[nt][1] = -INFINITY;
+    for (int mt = 0; mt < 2; ++mt) {
+      const int r = row0 + mt * 16;
+      slot[mt] = s_begin + r / S;
+      live[mt] = slot[mt] < n_slots;
+      phys[mt] = -1;
+      nv[mt] = 0;
+      if (live[mt]) phys[mt] = slot_page(a, unit, b, slot[mt], P, L, &nv[mt]);
+    }
+    uint4 va[2][KP], vb[2][KP];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-    float acc[NT][4];
-    score_mtile<D, G>(va[mt], vb[mt], bfrag, acc);
-    const int tok0 = (row0 + mt * 16) % S;
-    const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
-    const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+    for (int mt = 0; mt < 2; ++mt) {
+      const int tok0 = (row0 + mt * 16) % S;
+      const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+      const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+      const bf16* kb = static_cast<const bf16*>(a.k_pool) +
+                       ((static_cast<size_t>(phys[mt] < 0 ? 0 : phys[mt]) * a.Hkv + kvh) * S + tok0) * D;
+      const uint4* row_lo = reinterpret_cast<const uint4*>(kb + g * D) + t;
+      const uint4* row_hi = reinterpret_cast<const uint4*>(kb + (g + 8) * D) + t;
+#pragma unroll
+      for (int c = 0; c < KP; ++c) {
+        va[mt][c] = ok_lo ? __ldcs(row_lo + 4 * c) : make_uint4(0, 0, 0, 0);
+        vb[mt][c] = ok_hi ? __ldcs(row_hi + 4 * c) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    // the physical page of each selected slot, for the V pass
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+      if (lane == 0 && live[mt] && (row0 + mt * 16) % S == 0)
+        a.ws.sphys[static_cast<size_t>(unit) * a.cap + slot[mt]] = phys[mt];
+    __syncthreads();  // cta_key initialised
+    float wmax[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) wmax[nt][0] = wmax[nt][1] = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      float acc[NT][4];
+      score_mtile<D, G>(va[mt], vb[mt], bfrag, acc);
+      const int tok0 = (row0 + mt * 16) % S;
+      const bool ok_lo = phys[mt] >= 0 && tok0 + g < nv[mt];
+      const bool ok_hi = phys[mt] >= 0 && tok0 + g + 8 < nv[mt];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hd = nt * 8 + 2 * t + e;
+          const float zl = ok_lo ? a.scale * acc[nt][e] : -INFINITY;
+          const float zh = ok_hi ? a.scale * acc[nt][2 + e] : -INFINITY;
+          if (live[mt] && hd < G) {
+            float* zr = a.ws.zbuf + (static_cast<size_t>(unit) * G + hd) * zrow_len + static_cast<size_t>(slot[mt]) * S + tok0;
+            zr[g] = zl;
+            zr[g + 8] = zh;
+          }
+          wmax[nt][e] = fmaxf(wmax[nt][e], fmaxf(zl, zh));
+        }
+    }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
+        float m = wmax[nt][e];
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
         const int hd = nt * 8 + 2 * t + e;
-        const float zl = ok_lo ? a.scale * acc[nt][e] : -INFINITY;
-        const float zh = ok_hi ? a.scale * acc[nt][2 + e] : -INFINITY;
-        if (live[mt] && hd < G) {
-          float* zr = a.ws.zbuf + (static_cast<size_t>(unit) * G + hd) * zrow_len + static_cast<size_t>(slot[mt]) * S + tok0;
-          zr[g] = zl;
-          zr[g + 8] = zh;
-        }
-        wmax[nt][e] = fmaxf(wmax[nt][e], fmaxf(zl, zh));
+        if (g == 0 && hd < G && m > -INFINITY) atomicMax(&cta_key[hd], float_key(m));
       }
-  }
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float m = wmax[nt][e];
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-      const int hd = nt * 8 + 2 * t + e;
-      if (g == 0 && hd < G && m > -INFINITY) atomicMax(&cta_key[hd], float_key(m));
+    __syncthreads();
+    if (tid < G) {
+      const unsigned int k = cta_key[tid];
+      a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
     }
-  __syncthreads();
-  if (tid < G) {
-    const unsigned int k = cta_key[tid];
-    a.ws.cmax[(static_cast<size_t>(unit) * G + tid) * a.ws.nqk + split] = k == 0u ? -INFINITY : key_float(k);
+    __syncthreads();  // cta_key is reset by the next chunk
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -850,7 +857,9 @@ bool split_decode_fits(int cap, int S) {
 
 template <int D, int G>
 cudaError_t run_split_decode(DecodeArgs& a, int units, cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>(a.ws.nqk), static_cast<unsigned>(units));
+  // about eight CTAs per SM of a B200 in all; each loops over its chunks
+  const int per_unit = std::max(1, std::min(a.ws.nqk, (8 * 148) / std::max(1, units)));
+  const dim3 grid(static_cast<unsigned>(per_unit), static_cast<unsigned>(units));
   cudaError_t e = launch_k(k_score_kernel<D, G>, grid, dim3(kKsThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
