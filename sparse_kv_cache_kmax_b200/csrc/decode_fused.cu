@@ -393,8 +393,11 @@ __device__ float cta_solve_tau(const float* z, int n, float um, float* cand, flo
   return static_cast<float>(tau);
 }
 
-template <int D, int G>
+// IPOW: β when it is 1 or 2 (α = 2 or 1.5), fixed at compile time so that
+// those kernels carry no code for other exponents; 0: β read at run time.
+template <int D, int G, int IPOW>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a, FusedGeom f) {
+  const int ipow = IPOW != 0 ? IPOW : a.ipow;
   constexpr int KP = D / 32, NT = (G + 7) / 8, DPL = D / 32;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint64_t bars[kFWarps * kFMaxSpw];
@@ -535,7 +538,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   const int tpc = spc * S;
   const int n_tok = n_slots * S;
   float* zh = reinterpret_cast<float*>(ring);  // u = (α−1)·z of the head being solved
-  const bool closed = a.ipow == 1 || a.ipow == 2;
+  const bool closed = ipow == 1 || ipow == 2;
   float* cand = zh + ((n_tok + 31) & ~31);
   const size_t words = static_cast<size_t>(a.words);
   for (int h = rank; h < G; h += C) {
@@ -560,8 +563,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
       // β ∈ {1, 2}: bracket, candidates, pairwise support test and closed
       // form; otherwise Newton over every value from max u − 1 (f ≥ 0 there:
       // the maximum alone gives 1), one barrier per step, without a bracket
-      tau = closed ? cta_solve_tau(zh, n_tok, um, cand, a.beta, a.ipow, tsh)
-                   : cta_newton_tau(zh, n_tok, um, a.beta, a.ipow, tsh);
+      tau = closed ? cta_solve_tau(zh, n_tok, um, cand, a.beta, ipow, tsh)
+                   : cta_newton_tau(zh, n_tok, um, a.beta, ipow, tsh);
     }
     if (tid < C) cluster.map_shared_rank(s_tau, tid)[h] = tau;
     if (tid == 0 && a.tau_out) a.tau_out[orow] = tau;
@@ -663,7 +666,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
       float pt = 0.f;
       if (q < kPairs && e0 + r < ntl) {
         const float w = a.am1 * zs[h * zp + tl[e0 + r]] - s_tau[h];
-        if (w > 0.f) pt = pow_beta_fast(w, a.beta, a.ipow);
+        if (w > 0.f) pt = pow_beta_fast(w, a.beta, ipow);
       }
       pl[k] = pt;
     }
@@ -777,7 +780,7 @@ int max_active_clusters(int C, int smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fused_decode_kernel<D, G>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, fused_decode_kernel<D, G, 0>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -793,10 +796,12 @@ cudaError_t prepare_kernel(int smem_limit) {
   std::lock_guard<std::mutex> lock(mu);
   if (static_cast<int>(done.size()) <= dev) done.resize(dev + 1, 0);
   if (done[dev]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_limit);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(fused_decode_kernel<D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
+  for (auto kern : {fused_decode_kernel<D, G, 0>, fused_decode_kernel<D, G, 1>, fused_decode_kernel<D, G, 2>}) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_limit);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   done[dev] = 1;
   return cudaSuccess;
 }
@@ -821,7 +826,7 @@ FusedGeom choose(int units, int cap, int S) {
   const DeviceLimits lim = device_limits();
   cudaFuncAttributes fa{};
   FusedGeom best{};
-  const bool have_attr = cudaFuncGetAttributes(&fa, fused_decode_kernel<D, G>) == cudaSuccess;
+  const bool have_attr = cudaFuncGetAttributes(&fa, fused_decode_kernel<D, G, 0>) == cudaSuccess;
   const int smem_limit = lim.smem_optin - static_cast<int>(fa.sharedSizeBytes);
   if (have_attr && prepare_kernel<D, G>(smem_limit) == cudaSuccess) {
     for (int C = kFMaxCluster; C >= 1; C >>= 1) {
@@ -876,7 +881,9 @@ cudaError_t run_fused_decode(DecodeArgs& a, int units, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_decode_kernel<D, G>, a, f);
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, a.ipow == 1 ? fused_decode_kernel<D, G, 1> : (a.ipow == 2 ? fused_decode_kernel<D, G, 2> : fused_decode_kernel<D, G, 0>),
+      a, f);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
