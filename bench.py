@@ -160,8 +160,8 @@ class L2Flush:
 
 # ---------------------------------------------------------------- bytes
 def step_bytes(inp, policy, n_sel, support_pages, support_tokens):
-    """Bytes one step must move, and each kernel's share (SURVEY §8(d)'s
-    per-unit figures × the units of the step): the metadata rows the
+    """Bytes one step must move, and each kernel's share (per-unit bytes ×
+    the units of the step): the metadata rows the
     selection reads (box for top-k, mean/var for the Gaussian policy; none
     for the full cache), q, the page scores, the selected K, the V rows of the
     support (token by token for the decode kernel, as the method needs them;

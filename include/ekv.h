@@ -188,8 +188,8 @@ EKV_API ekv_status ekv_entmax_decode(const ekv_cache* cache, const ekv_seqs* seq
 
 /*
  * ekv_softmax_decode — softmax attention decode over the paged cache: the
- * full-cache baseline of [EKV] §4 ("the full cache read dominates"), split
- * over pages.  For every query head h, o_h = Σ_i e^{z_i − m}·v_i / Σ_i e^{z_i − m}
+ * full-cache baseline of [EKV] §4 (reading the whole cache is what sparse
+ * decoding avoids), split over pages.  For every query head h, o_h = Σ_i e^{z_i − m}·v_i / Σ_i e^{z_i − m}
  * with z_i = scale·q_h·k_i over every valid token of the selected pages
  * (sel = NULL with n_sel NULL: every page of the sequence; cap ≥ max_pages).
  * sel: device [batch, Hkv, cap] logical page indices with n_sel entries per

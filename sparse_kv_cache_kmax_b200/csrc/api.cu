@@ -283,7 +283,7 @@ EKV_API ekv_status ekv_decode_adaptive(const ekv_cache* cache, const ekv_seqs* s
   EKV_TRY(cuda_status(launch_score(*cache, *seqs, q, num_q_heads, scale, ub, st)));
   int k = k0 < P ? k0 : P;
   for (;;) {
-    // sel holds [batch, Hkv, k] at this round's k
+    // sel holds [batch, Hkv, k] for the current budget k
     const size_t tk = topk_ws_bytes(static_cast<int>(U), P, k);
     EKV_TRY(cuda_status(launch_topk(*seqs, cache->num_kv_heads, cache->page_size, ub, k, k, sel, n_sel,
                                     tk > 0 ? tws : nullptr, st)));

@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
 #pragma unroll
         for (int x = 0; x < DPL; ++x) acc[x] = fmaf(p[r], v[r][x], acc[x]);
     }
-    __syncthreads();  // the list is rewritten by the next round
+    __syncthreads();  // the list is rewritten for the next kHdCand support tokens
   }
 #pragma unroll
   for (int x = 0; x < DPL; ++x) red[warp][lane * DPL + x] = acc[x];
