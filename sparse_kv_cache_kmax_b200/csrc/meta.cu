@@ -54,24 +54,22 @@ struct Pair<float> {
   }
 };
 
-// Metadata of one coordinate pair over tokens 0..n-1 of a page (n ≤ 32).
+// Metadata of one coordinate pair over tokens 0..n-1 of a page (1 ≤ n ≤ 32).
 // When `inject` ≥ 0, token `inject` takes the values (xa, xb) instead of the
-// pool.  The page's values are loaded first as one batch of independent loads.
+// pool.  The page's values are loaded first as one batch of independent,
+// unconditional loads (a token past n reads token 0 again and is dropped):
+// loads behind per-token branches were issued one after another.
 template <typename T>
 __device__ void page_pair_meta(const T* page_k, int D, int n, int j, int inject, float xa,
                                float xb, T* box_row, T* mom_row) {
   float va[32], vb[32];
 #pragma unroll
   for (int t = 0; t < 32; ++t) {
-    va[t] = vb[t] = 0.f;
-    if (t < n) {
-      if (t == inject) {
-        va[t] = xa;
-        vb[t] = xb;
-      } else {
-        Pair<T>::load(page_k + static_cast<size_t>(t) * D + j, va[t], vb[t]);
-      }
-    }
+    const int tt = t < n ? t : 0;
+    float a, b;
+    Pair<T>::load(page_k + static_cast<size_t>(tt) * D + j, a, b);
+    va[t] = t < n ? (t == inject ? xa : a) : 0.f;
+    vb[t] = t < n ? (t == inject ? xb : b) : 0.f;
   }
   float mx0 = -INFINITY, mx1 = -INFINITY, mn0 = INFINITY, mn1 = INFINITY;
   double s0 = 0.0, s1 = 0.0;
