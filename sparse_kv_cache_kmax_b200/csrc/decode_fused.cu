@@ -636,27 +636,27 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(DecodeArgs a
   constexpr int kPerLane = (kPairs + 31) / 32;
 #pragma unroll 1
   for (int e0 = warp * kRowsInFlight; e0 < ntl; e0 += kFWarps * kRowsInFlight) {
+    // every row is loaded unconditionally (a row past the list reads list
+    // entry e0, which exists, and is zeroed after): loads behind per-row
+    // branches are issued one after another
     float v[kRowsInFlight][DPL];
 #pragma unroll
     for (int r = 0; r < kRowsInFlight; ++r) {
       const int e = e0 + r;
-#pragma unroll
-      for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
-      if (e < ntl) {
-        const int tok = tl[e], j = tok / S;
-        const bf16* src = static_cast<const bf16*>(a.v_pool) +
-                          ((static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * S + (tok - j * S)) * D + lane * DPL;
-        if constexpr (DPL == 4) {
-          const uint2 w = *reinterpret_cast<const uint2*>(src);
-          v[r][0] = __uint_as_float(w.x << 16);
-          v[r][1] = __uint_as_float(w.x & 0xffff0000u);
-          v[r][2] = __uint_as_float(w.y << 16);
-          v[r][3] = __uint_as_float(w.y & 0xffff0000u);
-        } else {
-          const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
-          v[r][0] = __uint_as_float(w << 16);
-          v[r][1] = __uint_as_float(w & 0xffff0000u);
-        }
+      const bool in = e < ntl;
+      const int tok = tl[in ? e : e0], j = tok / S;
+      const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                        ((static_cast<size_t>(phys_s[j]) * a.Hkv + kvh) * S + (tok - j * S)) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        v[r][0] = in ? __uint_as_float(w.x << 16) : 0.f;
+        v[r][1] = in ? __uint_as_float(w.x & 0xffff0000u) : 0.f;
+        v[r][2] = in ? __uint_as_float(w.y << 16) : 0.f;
+        v[r][3] = in ? __uint_as_float(w.y & 0xffff0000u) : 0.f;
+      } else {
+        const uint32_t w = *reinterpret_cast<const unsigned int*>(src);
+        v[r][0] = in ? __uint_as_float(w << 16) : 0.f;
+        v[r][1] = in ? __uint_as_float(w & 0xffff0000u) : 0.f;
       }
     }
     float pl[kPerLane];
