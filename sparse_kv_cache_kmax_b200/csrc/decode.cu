@@ -584,7 +584,11 @@ __global__ void __launch_bounds__(32 * kPvWarps, pv_min_blocks<T, D, G>()) pv_ke
       typename PvRaw<T, DPL>::Row raw[kPvRows];
 #pragma unroll
       for (int r = 0; r < kPvRows; ++r)
-        raw[r] = (r % S) < nvp[r / S] ? PvRaw<T, DPL>::load(vbase[r / S] + (r % S) * D) : PvRaw<T, DPL>::zero();
+      {
+        // unconditional load of a row inside the page tile, zeroed after
+        const auto x = PvRaw<T, DPL>::load(vbase[r / S] + (r % S) * D);
+        raw[r] = (r % S) < nvp[r / S] ? x : PvRaw<T, DPL>::zero();
+      }
       float p[G];
       {
         const int e = e0 + lane / S, t = lane % S;

@@ -257,8 +257,9 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
 #pragma unroll
         for (int j = 0; j < kHdBatch; ++j) {
           const int i = 4 * ((q0 + j) * THREADS + tid);
-          v[j] = (q0 + j < NK / 4 && i < n) ? __ldcg(reinterpret_cast<const float4*>(z + i))
-                                            : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+          const bool in = q0 + j < NK / 4 && i < n;
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(z + (in ? i : 0)));  // n ≥ 4 here
+          v[j] = in ? x : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         }
 #pragma unroll
         for (int j = 0; j < kHdBatch; ++j)
@@ -608,28 +609,26 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
 #pragma unroll
       for (int r = 0; r < kHdRows; ++r) {
         const int e = e0 + r;
-        p[r] = 0.f;
-#pragma unroll
-        for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
-        if (e < nl) {
-          const int tok = sh.ci[e];
-          const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
-          if (ph >= 0) {
-            p[r] = sh.cu[e];
-            const bf16* src = static_cast<const bf16*>(a.v_pool) +
-                              ((static_cast<size_t>(ph) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
-            if constexpr (DPL == 4) {
-              const uint2 w2 = *reinterpret_cast<const uint2*>(src);
-              v[r][0] = __uint_as_float(w2.x << 16);
-              v[r][1] = __uint_as_float(w2.x & 0xffff0000u);
-              v[r][2] = __uint_as_float(w2.y << 16);
-              v[r][3] = __uint_as_float(w2.y & 0xffff0000u);
-            } else {
-              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
-              v[r][0] = __uint_as_float(w1 << 16);
-              v[r][1] = __uint_as_float(w1 & 0xffff0000u);
-            }
-          }
+        // unconditional load (a row past the list reads entry e0, which
+        // exists; an invalid page reads page 0) zeroed after: loads behind
+        // per-row branches are issued one after another
+        const bool in_list = e < nl;
+        const int tok = sh.ci[in_list ? e : e0];
+        const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
+        const bool in = in_list && ph >= 0;
+        p[r] = in ? sh.cu[in_list ? e : e0] : 0.f;
+        const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                          ((static_cast<size_t>(ph >= 0 ? ph : 0) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const uint2 w2 = *reinterpret_cast<const uint2*>(src);
+          v[r][0] = in ? __uint_as_float(w2.x << 16) : 0.f;
+          v[r][1] = in ? __uint_as_float(w2.x & 0xffff0000u) : 0.f;
+          v[r][2] = in ? __uint_as_float(w2.y << 16) : 0.f;
+          v[r][3] = in ? __uint_as_float(w2.y & 0xffff0000u) : 0.f;
+        } else {
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
+          v[r][0] = in ? __uint_as_float(w1 << 16) : 0.f;
+          v[r][1] = in ? __uint_as_float(w1 & 0xffff0000u) : 0.f;
         }
       }
 #pragma unroll
@@ -788,28 +787,26 @@ __global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(Decod
 #pragma unroll
     for (int r = 0; r < kHdRows; ++r) {
       const int e = e0 + r;
-      p[r] = 0.f;
-#pragma unroll
-      for (int x = 0; x < DPL; ++x) v[r][x] = 0.f;
-      if (e < ns) {
-        const int tok = s_i[warp][e];
-        const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
-        if (ph >= 0) {
-          p[r] = s_p[warp][e];
-          const bf16* src = static_cast<const bf16*>(a.v_pool) +
-                            ((static_cast<size_t>(ph) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
-          if constexpr (DPL == 4) {
-            const uint2 w2 = *reinterpret_cast<const uint2*>(src);
-            v[r][0] = __uint_as_float(w2.x << 16);
-            v[r][1] = __uint_as_float(w2.x & 0xffff0000u);
-            v[r][2] = __uint_as_float(w2.y << 16);
-            v[r][3] = __uint_as_float(w2.y & 0xffff0000u);
-          } else {
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
-            v[r][0] = __uint_as_float(w1 << 16);
-            v[r][1] = __uint_as_float(w1 & 0xffff0000u);
-          }
-        }
+      // unconditional load (a row past the list reads entry e0, which
+      // exists; an invalid page reads page 0) zeroed after: loads behind
+      // per-row branches are issued one after another
+      const bool in_list = e < ns;
+      const int tok = s_i[warp][in_list ? e : e0];
+      const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
+      const bool in = in_list && ph >= 0;
+      p[r] = in ? s_p[warp][in_list ? e : e0] : 0.f;
+      const bf16* src = static_cast<const bf16*>(a.v_pool) +
+                        ((static_cast<size_t>(ph >= 0 ? ph : 0) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const uint2 w2 = *reinterpret_cast<const uint2*>(src);
+        v[r][0] = in ? __uint_as_float(w2.x << 16) : 0.f;
+        v[r][1] = in ? __uint_as_float(w2.x & 0xffff0000u) : 0.f;
+        v[r][2] = in ? __uint_as_float(w2.y << 16) : 0.f;
+        v[r][3] = in ? __uint_as_float(w2.y & 0xffff0000u) : 0.f;
+      } else {
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(src);
+        v[r][0] = in ? __uint_as_float(w1 << 16) : 0.f;
+        v[r][1] = in ? __uint_as_float(w1 & 0xffff0000u) : 0.f;
       }
     }
 #pragma unroll
