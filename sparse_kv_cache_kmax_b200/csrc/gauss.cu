@@ -116,14 +116,33 @@ __global__ void __launch_bounds__(kTauThreads)
   __shared__ int i_scratch[32];
   int par = 0;
 
-  // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
+  // fn(p, μ_p, σ_p) for this thread's pages pa + tid, pa + tid + 512, … in
+  // order, read four at a time with unconditional loads (a page past pb
+  // reads page pa and is skipped): loads behind per-page branches or loop
+  // exits are issued one after another
   const size_t base = static_cast<size_t>(row) * max_pages;
+  auto for_pages = [&](auto fn) {
+    constexpr int kB = 4;
+    for (int p0 = pa + tid; p0 < pb; p0 += kB * kTauThreads) {
+      float mu[kB], sg[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int p = p0 + k * kTauThreads;
+        const size_t at = base + (p < pb ? p : pa);
+        mu[k] = ws.mu[at];
+        sg[k] = ws.sig[at];
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k)
+        if (p0 + k * kTauThreads < pb) fn(p0 + k * kTauThreads, mu[k], sg[k]);
+    }
+  };
+  // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
   const float inv_beta = 1.0f / static_cast<float>(beta);
   float lo = -INFINITY;
-  for (int p = pa + tid; p < pb; p += kTauThreads) {
-    const float mu = ws.mu[base + p];
+  for_pages([&](int p, float mu, float) {
     if (mu > -INFINITY) lo = fmaxf(lo, mu - powf(static_cast<float>(min(S, L - p * S)), -inv_beta));
-  }
+  });
   lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
   if (tid < C) cluster.map_shared_rank(&tx, tid)->lo[rank] = lo;
   cluster.sync();
@@ -142,25 +161,25 @@ __global__ void __launch_bounds__(kTauThreads)
   // thread (coalesced loads; a fixed order, so the sums are deterministic);
   // while too many pages are left for shared memory, the steps read every
   // page of the share from global memory.
-  auto live = [&](int p, double t) {
-    const float mu = ws.mu[base + p], sg = ws.sig[base + p];
+  auto live = [&](float mu, float sg, double t) {
     return mu > -INFINITY && static_cast<double>(mu) + kPruneC * static_cast<double>(sg) > t;
   };
   int nc = 0;
   bool cached = false;
   auto gather = [&](double t) {  // every thread calls it
     int mine = 0;
-    for (int p = pa + tid; p < pb; p += kTauThreads) mine += live(p, t) ? 1 : 0;
+    for_pages([&](int, float mu, float sg) { mine += live(mu, sg, t) ? 1 : 0; });
     int pos = block_exclusive_scan(mine, i_scratch, &nc);
     cached = nc <= kGaussCand;
     if (cached)
-      for (int p = pa + tid; p < pb; p += kTauThreads)
-        if (live(p, t)) {
-          c_mu[pos] = ws.mu[base + p];
-          c_sg[pos] = ws.sig[base + p];
+      for_pages([&](int p, float mu, float sg) {
+        if (live(mu, sg, t)) {
+          c_mu[pos] = mu;
+          c_sg[pos] = sg;
           c_n[pos] = static_cast<float>(min(S, L - p * S));
           ++pos;
         }
+      });
     __syncthreads();
   };
   // cuts the cached list to the pages still above t, in place, order kept:
@@ -304,17 +323,32 @@ struct FilterCtx {
   int best_i[32];
 };
 
-__device__ __forceinline__ double page_margin(const GaussWs& ws, const FilterCtx& fc, int unit, int G, int max_pages,
-                                              int p) {
-  double mg = -INFINITY;
-  for (int g = 0; g < G; ++g)
-    mg = fmax(mg, static_cast<double>(ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + p]) - fc.thr[g]);
-  return mg;
-}
 
 // The chunk's pages [c0, c1): warp w takes [c0 + w·kPer, …), its lanes
 // consecutive pages (coalesced loads).
 constexpr int kFilterPerWarp = kFilterChunk / (kGaussThreads / 32);
+constexpr int kFilterSteps = kFilterPerWarp / 32;  // pages per lane
+
+// Margins of the lane's pages p0 + 32·i + lane (i < kFilterSteps) of the
+// warp's run [p0, p1), p0 < p1, every head's ŝ read with unconditional loads
+// first (a page past p1 reads page p0; its margin is not used): loads behind
+// per-page branches are issued one after another.
+__device__ __forceinline__ void lane_margins(const GaussWs& ws, const FilterCtx& fc, int unit, int G,
+                                             int max_pages, int p0, int p1, double (&mg)[kFilterSteps]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < kFilterSteps; ++i) mg[i] = -INFINITY;
+  for (int g = 0; g < G; ++g) {
+    float hv[kFilterSteps];
+#pragma unroll
+    for (int i = 0; i < kFilterSteps; ++i) {
+      const int p = p0 + 32 * i + lane;
+      hv[i] = ws.hat[(static_cast<size_t>(unit) * G + g) * max_pages + (p < p1 ? p : p0)];
+    }
+#pragma unroll
+    for (int i = 0; i < kFilterSteps; ++i) mg[i] = fmax(mg[i], static_cast<double>(hv[i]) - fc.thr[g]);
+  }
+}
 
 __global__ void __launch_bounds__(kGaussThreads)
     gauss_count_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages, int Hkv, int G,
@@ -327,21 +361,25 @@ __global__ void __launch_bounds__(kGaussThreads)
   __shared__ FilterCtx fc;
   if (tid < G) fc.thr[tid] = ws.tau_hat[static_cast<size_t>(unit) * G + tid] - delta;
   __syncthreads();
+  auto margins = [&](int a0, int a1, double (&mg)[kFilterSteps]) {
+    lane_margins(ws, fc, unit, G, max_pages, a0, a1, mg);
+  };
   const int p0 = chunk * kFilterChunk + warp * kFilterPerWarp, p1 = min(P, p0 + kFilterPerWarp);
   double my_best = -INFINITY;
   int my_idx = 0x7fffffff, cnt = 0;
-  for (int q0 = p0; q0 < p1; q0 += 32) {
-    const int p = q0 + lane;
-    bool keep = false;
-    if (p < p1) {
-      const double mg = page_margin(ws, fc, unit, G, max_pages, p);
-      keep = mg > 0.0;
-      if (mg > my_best) {
-        my_best = mg;
+  if (p0 < p1) {
+    double mg[kFilterSteps];
+    margins(p0, p1, mg);
+#pragma unroll
+    for (int i = 0; i < kFilterSteps; ++i) {
+      const int p = p0 + 32 * i + lane;
+      const bool keep = p < p1 && mg[i] > 0.0;
+      if (p < p1 && mg[i] > my_best) {
+        my_best = mg[i];
         my_idx = p;
       }
+      cnt += __popc(__ballot_sync(0xffffffffu, keep));
     }
-    cnt += __popc(__ballot_sync(0xffffffffu, keep));
   }
   for (int o = 16; o > 0; o >>= 1) {
     const double om = __shfl_xor_sync(0xffffffffu, my_best, o);
@@ -429,20 +467,27 @@ __global__ void __launch_bounds__(kGaussThreads)
     n_sel[unit] = min(total, cap);
     if (total > cap) raise_flag(EKV_EFLAG_SEL_OVERFLOW);
   }
+  auto margins = [&](int a0, int a1, double (&mg)[kFilterSteps]) {
+    lane_margins(ws, fc, unit, G, max_pages, a0, a1, mg);
+  };
   const int p0 = chunk * kFilterChunk + warp * kFilterPerWarp, p1 = min(P, p0 + kFilterPerWarp);
   int cnt = 0;
-  for (int q0 = p0; q0 < p1; q0 += 32) {
-    const int p = q0 + lane;
-    cnt += __popc(__ballot_sync(0xffffffffu, p < p1 && page_margin(ws, fc, unit, G, max_pages, p) > 0.0));
+  double mg[kFilterSteps];
+  if (p0 < p1) {
+    margins(p0, p1, mg);
+#pragma unroll
+    for (int i = 0; i < kFilterSteps; ++i)
+      cnt += __popc(__ballot_sync(0xffffffffu, p0 + 32 * i + lane < p1 && mg[i] > 0.0));
   }
   if (lane == 0) fc.scan[warp] = cnt;
   __syncthreads();
   int pos = s_before;
   for (int w = 0; w < warp; ++w) pos += fc.scan[w];
   if (cnt == 0) return;
-  for (int q0 = p0; q0 < p1; q0 += 32) {
-    const int p = q0 + lane;
-    const bool keep = p < p1 && page_margin(ws, fc, unit, G, max_pages, p) > 0.0;
+#pragma unroll
+  for (int i = 0; i < kFilterSteps; ++i) {
+    const int p = p0 + 32 * i + lane;
+    const bool keep = p < p1 && mg[i] > 0.0;
     const unsigned int bal = __ballot_sync(0xffffffffu, keep);
     const int at = pos + __popc(bal & ((1u << lane) - 1u));
     if (keep && at < cap) out[at] = p;
