@@ -240,7 +240,8 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
 #pragma unroll
     for (int k = 0; k < (kReg ? VPT : NK); ++k) {
       const int i = k * THREADS + tid;
-      uv[k] = i < n ? am1 * z[i] : -INFINITY;
+      const float zi = z[i < n ? i : 0];  // unconditional load (see the V rows below)
+      uv[k] = i < n ? am1 * zi : -INFINITY;
     }
   }
   // fn(k, u) for every value of this thread in order of k; read from the
@@ -687,7 +688,8 @@ __global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(Decod
 #pragma unroll
   for (int k = 0; k < VPL; ++k) {
     const int i = k * 32 + lane;
-    u[k] = i < n ? am1 * __ldcg(z + i) : -INFINITY;
+    const float zi = __ldcg(z + (i < n ? i : 0));  // unconditional load, dropped past n
+    u[k] = i < n ? am1 * zi : -INFINITY;
     m = fmaxf(m, u[k]);
   }
   m = warp_max(m);
