@@ -48,7 +48,7 @@ kHostLead = 100_000  # device cycles (~50 µs) of delay before each staged stage
 SCORE_FILES = ("score.cu", "common.cuh")
 DECODE_FILES = ("decode_fused.cu", "decode.cuh", "common.cuh")
 SCORE_TRAFFIC = {"2ac4280b73b40cfc": 135471616}
-DECODE_TRAFFIC = {"7cd4a1d5c3195fd2": 35236096}
+DECODE_TRAFFIC = {"546c3d7b8f786b33": 35236864}
 
 
 def kernel_hash(files=SCORE_FILES):
