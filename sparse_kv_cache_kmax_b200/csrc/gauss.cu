@@ -12,9 +12,12 @@
 // (integration by parts with xφ = −φ').  F^(1/β) is convex and decreasing
 // (an L^β norm of (u − τ)_+), so Newton's method on it, started left of the
 // root (Jensen's bound τ_lo = max_p μ_p − n_p^(−1/β), where F ≥ 1), climbs
-// monotonically to the root and never overshoots.  Pages with c > kPruneC at τ_lo contribute below
-// n·σ^β·J_β(kPruneC) and stay negligible for every later τ (c only grows), so
-// only the survivors are iterated, from shared memory.  The recurrence
+// monotonically to the root and never overshoots; far from the root a
+// flatter transform takes larger steps (see the solve below).  Pages with
+// c > kPruneC at τ_lo contribute below
+// n·σ^β·J_β(kPruneC) and stay negligible at every τ the lists are later cut
+// at (points left of the root, which only rise: c only grows), so only the
+// survivors are iterated, from shared memory.  The recurrence
 // amplifies the rounding of Q and φ by about c^(2β)/β! for c > 0, so the fp32
 // iterations only approach the root (they stop once a step is below 1e-5);
 // the final Newton steps evaluate every term in float64.
@@ -266,39 +269,50 @@ __global__ void __launch_bounds__(kTauThreads)
     }
     par ^= 1;  // the next step writes the other half: a slow CTA may still read this one
   };
-  // fp32 terms: a monotone approach from the left while the steps are large
-  // (the lists cut every few steps); the float64 steps below converge
-  // quadratically from there
-  // Newton's method on h(τ) = F(τ)^(1/β), the L^β norm of (u − τ)_+ under the
-  // pages' mixture: convex and decreasing like F, so the steps from the left
-  // never pass the root, and close to linear far from it (Newton on F itself
-  // only closes a fraction 1/β of the gap per step there).  The step
-  // (h − 1)/(−h') is β·(F − F^(1−1/β))/(−F') = β·F^(1−1/β)·(F^(1/β) − 1)/(−F'),
-  // evaluated from F − 1 without cancellation near the root.
-  const double omb = 1.0 - 1.0 / beta;
-  auto newton_step = [&](double F, double dF) {
+  // fp32 terms while the steps are large (the lists cut every few steps);
+  // the float64 steps below converge quadratically from there.
+  // Newton's method on h_p(τ) = F(τ)^(1/p).  For p = β, h_β is the L^β norm
+  // of (u − τ)_+ under the pages' mixture: convex and decreasing like F, so
+  // its steps from the left never pass the root, and from the right they
+  // land left of it.  Where F falls off faster than a power (Gaussian tails
+  // far above most pages' means) a step on h_β closes only part of the gap,
+  // so while F > kFarF the steps use the flatter h_kFarP, which may pass the
+  // root; the first time one does (F < 1), the far steps stop and h_β takes
+  // over from the right.  The step (h_p − 1)/(−h_p') is
+  // p·F^(1−1/p)·(F^(1/p) − 1)/(−F'), evaluated from F − 1 without
+  // cancellation near the root.  Lists are cut at tau_safe, the largest τ
+  // evaluated with F ≥ 1 (left of the root), never at a τ that passed it.
+  constexpr double kFarF = 4.0, kFarP = 8.0;
+  auto newton_step = [&](double F, double dF, double p) {
     const double l = log1p(F - 1.0);
-    return beta * exp(omb * l) * expm1(l / beta) / dF;
+    return p * exp((1.0 - 1.0 / p) * l) * expm1(l / p) / dF;
   };
-  double tau = static_cast<double>(lo);
+  double tau = static_cast<double>(lo), tau_safe = tau;
+  bool far = true;
   for (int it = 0; it < 40; ++it) {
     double F, dF;
     evaluate(tau, false, F, dF);
-    const double step = newton_step(F, dF);
-    if (!(step > 0.0)) break;
+    if (F >= 1.0) tau_safe = fmax(tau_safe, tau);
+    else far = false;
+    if (!(F > 0.0) || !(dF > 0.0)) {  // past every page's mass: back off towards the last safe τ
+      if (!(tau > tau_safe)) break;
+      tau = 0.5 * (tau + tau_safe);
+      continue;
+    }
+    const double step = newton_step(F, dF, far && F > kFarF ? kFarP : static_cast<double>(beta));
     tau += step;
-    if (step <= 1e-5 * fmax(1.0, fabs(tau))) break;
+    if (fabs(step) <= 1e-5 * fmax(1.0, fabs(tau))) break;
     if ((it & 3) == 3) {
-      if (cached) recut(tau);
-      else gather(tau);
+      if (cached) recut(tau_safe);
+      else gather(tau_safe);
     }
   }
-  if (!cached) gather(tau);
+  if (!cached) gather(fmin(tau, tau_safe));
   for (int it = 0; it < 3; ++it) {  // float64 terms: quadratic convergence (either side)
     double F, dF;
     evaluate(tau, true, F, dF);
     if (!(dF > 0.0) || !(F > 0.0)) break;
-    const double step = newton_step(F, dF);
+    const double step = newton_step(F, dF, static_cast<double>(beta));
     tau += step;
     // the error left after a step of size e is of order e², so a step below
     // 1e-7 leaves τ̂ within ~1e-14: no further evaluation is needed
