@@ -19,7 +19,7 @@
 // at (points left of the root, which only rise: c only grows), so only the
 // survivors are iterated, from shared memory.  The recurrence
 // amplifies the rounding of Q and φ by about c^(2β)/β! for c > 0, so the fp32
-// iterations only approach the root (they stop once a step is below 1e-5);
+// iterations only approach the root (they stop once a step is below 1e-4);
 // the final Newton steps evaluate every term in float64.
 #include <cooperative_groups.h>
 
@@ -97,8 +97,11 @@ struct TauExchange {
 // One cluster of C CTAs per query head; CTA r owns the r-th contiguous
 // share of the head's pages.  Every sum is a fixed tree inside a CTA, then
 // the C partials in rank order, so all CTAs hold the same value and take the
-// same steps.
-__global__ void __launch_bounds__(kTauThreads)
+// same steps.  MIN_BLOCKS = 2 caps the registers so that two CTAs share an
+// SM, for launches with more CTAs than SMs (all clusters resident at once,
+// one wave); 1 leaves the compiler its registers.
+template <int MIN_BLOCKS>
+__global__ void __launch_bounds__(kTauThreads, MIN_BLOCKS)
     gauss_tau_kernel(GaussWs ws, const int32_t* __restrict__ seq_lens, int S, int max_pages, int Hkv, int G,
                      int Hq, int beta, float* __restrict__ tau_out) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -120,12 +123,12 @@ __global__ void __launch_bounds__(kTauThreads)
   int par = 0;
 
   // fn(p, μ_p, σ_p) for this thread's pages pa + tid, pa + tid + 512, … in
-  // order, read four at a time with unconditional loads (a page past pb
+  // order, read eight at a time with unconditional loads (a page past pb
   // reads page pa and is skipped): loads behind per-page branches or loop
   // exits are issued one after another
   const size_t base = static_cast<size_t>(row) * max_pages;
   auto for_pages = [&](auto fn) {
-    constexpr int kB = 4;
+    constexpr int kB = 8;
     for (int p0 = pa + tid; p0 < pb; p0 += kB * kTauThreads) {
       float mu[kB], sg[kB];
 #pragma unroll
@@ -142,9 +145,11 @@ __global__ void __launch_bounds__(kTauThreads)
   };
   // Jensen's lower bracket: F(τ_lo) ≥ 1 at τ_lo = max_p μ_p − n_p^(−1/β)
   const float inv_beta = 1.0f / static_cast<float>(beta);
+  const float full_pow = powf(static_cast<float>(S), -inv_beta);  // every page but the last holds S tokens
   float lo = -INFINITY;
   for_pages([&](int p, float mu, float) {
-    if (mu > -INFINITY) lo = fmaxf(lo, mu - powf(static_cast<float>(min(S, L - p * S)), -inv_beta));
+    const int n = L - p * S;
+    if (mu > -INFINITY) lo = fmaxf(lo, mu - (n >= S ? full_pow : powf(static_cast<float>(n), -inv_beta)));
   });
   lo = block_reduce(lo, f_scratch, [](float x, float y) { return fmaxf(x, y); });
   if (tid < C) cluster.map_shared_rank(&tx, tid)->lo[rank] = lo;
@@ -301,7 +306,9 @@ __global__ void __launch_bounds__(kTauThreads)
     }
     const double step = newton_step(F, dF, far && F > kFarF ? kFarP : static_cast<double>(beta));
     tau += step;
-    if (fabs(step) <= 1e-5 * fmax(1.0, fabs(tau))) break;
+    // the fp32 terms are good to ~1e-5 near the root: smaller steps are the
+    // float64 steps' work, and they check their own convergence
+    if (fabs(step) <= 1e-4 * fmax(1.0, fabs(tau))) break;
     if ((it & 3) == 3) {
       if (cached) recut(tau_safe);
       else gather(tau_safe);
@@ -519,11 +526,14 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
   // CTAs per head: one up to 8192 pages (a cluster's barrier per step costs
   // more than it saves there), else enough to give the B200's SMs two CTAs
   // each, at most kTauMaxCluster
+  constexpr int kSms = 148;
   const int rows = U * G;
   int C = 1;
-  while (C < kTauMaxCluster && s.max_pages > 8192 && rows * C * 2 <= 2 * 148) C *= 2;
+  while (C < kTauMaxCluster && s.max_pages > 8192 && rows * C * 2 <= 2 * kSms) C *= 2;
+  const bool two_per_sm = rows * C > kSms;
+  auto* kernel = two_per_sm ? gauss_tau_kernel<2> : gauss_tau_kernel<1>;
   const size_t smem = 3 * kGaussCand * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(gauss_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   {
     cudaLaunchConfig_t cfg = {};
@@ -540,7 +550,7 @@ cudaError_t launch_gauss_select(const ekv_cache& c, const ekv_seqs& s, int Hq, f
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, gauss_tau_kernel, ws, s.seq_lens, c.page_size, s.max_pages, Hkv, G, Hq, beta,
+    e = cudaLaunchKernelEx(&cfg, kernel, ws, s.seq_lens, c.page_size, s.max_pages, Hkv, G, Hq, beta,
                            tau_hat);
     if (e != cudaSuccess) return e;
   }
