@@ -443,11 +443,21 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) meta_stream_kernel
 constexpr int kDirectWarps = 4;
 constexpr int kTile = 16;
 
-// CTAs per SM: 4 (16 warps) while the B fragments are one 8-column tile; the
-// Gaussian statistics need 2 or 3 tiles of B and run 2 CTAs per SM.
+// 8-column tiles of B per k-step in the direct kernel.  The score takes the
+// G heads' q⁺ over the kmax half of a row and q⁻ over the kmin half, in the
+// same columns.  The Gaussian statistics take q over the mean half (G
+// columns) and q² hi, lo over the variance half (2G columns): each k-step
+// lies in one half, so it multiplies only that half's columns.
+template <int G, bool GAUSS>
+struct DirectTiles {
+  static constexpr int value = ((GAUSS ? 2 * G : G) + 7) / 8;
+};
+
+// CTAs per SM: 4 (16 warps) while the B fragments are one 8-column tile, 2
+// with more (G = 8 Gaussian statistics).
 template <int D, int G, bool GAUSS>
 struct DirectOcc {
-  static constexpr int value = Cols<G, GAUSS>::tiles > 1 ? 2 : 4;
+  static constexpr int value = DirectTiles<G, GAUSS>::value > 1 ? 2 : 4;
 };
 
 template <int D, int G, bool GAUSS>
@@ -462,8 +472,8 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
     grid_dep_enter();
   }
   bool waited = a.defer_wait == 0;
-  constexpr int KP = 2 * D / 32;              // 32-element chunks per row
-  constexpr int NT = Cols<G, GAUSS>::tiles;   // 8-column tiles of the B operand
+  constexpr int KP = 2 * D / 32;                 // 32-element chunks per row
+  constexpr int NT = DirectTiles<G, GAUSS>::value; // 8-column tiles of B per k-step
   constexpr int ROW = 2 * D * 2;              // bytes per metadata row
   extern __shared__ __align__(16) int dyn[];
   float* ctile = reinterpret_cast<float*>(dyn);                // [kDirectWarps][16][24]
@@ -573,13 +583,12 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
           const float v = __bfloat162float(qb[col * D + j]);
           return lo_half ? fmaxf(v, 0.f) : fminf(v, 0.f);
         } else {
-          if (col < G) return lo_half ? __bfloat162float(qb[col * D + j]) : 0.f;
-          if (col >= 3 * G || lo_half) return 0.f;
-          const int hh = (col - G) >> 1;
-          const float v = __bfloat162float(qb[hh * D + j]);
+          if (lo_half) return col < G ? __bfloat162float(qb[col * D + j]) : 0.f;
+          if (col >= 2 * G) return 0.f;
+          const float v = __bfloat162float(qb[(col >> 1) * D + j]);
           float hi, lo;
           split_bf16(v * v, hi, lo);
-          return ((col - G) & 1) ? lo : hi;
+          return (col & 1) ? lo : hi;
         }
       };
 #pragma unroll
@@ -592,17 +601,26 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
           bfrag[ks][nt][1] = pack_bf16_exact(coef(col, k0 + 2), coef(col, k0 + 3));
         }
     }
-    float acc[NT][4];
+    // acc: the score, or the Gaussian means; acv: the Gaussian variances
+    float acc[NT][4], acv[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = acv[nt][e] = 0.f;
 #pragma unroll
     for (int c = 0; c < KP; ++c) {
       const uint32_t f0[4] = {va[c].x, vb[c].x, va[c].y, vb[c].y};
       const uint32_t f1[4] = {va[c].z, vb[c].z, va[c].w, vb[c].w};
+      const bool var_half = GAUSS && c >= KP / 2;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        mma_bf16(acc[nt], f0, bfrag[2 * c][nt][0], bfrag[2 * c][nt][1]);
-        mma_bf16(acc[nt], f1, bfrag[2 * c + 1][nt][0], bfrag[2 * c + 1][nt][1]);
+        if (var_half) {
+          mma_bf16(acv[nt], f0, bfrag[2 * c][nt][0], bfrag[2 * c][nt][1]);
+          mma_bf16(acv[nt], f1, bfrag[2 * c + 1][nt][0], bfrag[2 * c + 1][nt][1]);
+        } else if (!GAUSS || nt * 8 < G) {  // a Gaussian mean tile holds G ≤ 8 columns
+          mma_bf16(acc[nt], f0, bfrag[2 * c][nt][0], bfrag[2 * c][nt][1]);
+          mma_bf16(acc[nt], f1, bfrag[2 * c + 1][nt][0], bfrag[2 * c + 1][nt][1]);
+        }
       }
     }
     if constexpr (!GAUSS) {
@@ -623,14 +641,22 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
         if (g + 8 < n) urow[g + 8] = ok_hi ? a.scale * m_hi : -INFINITY;
       }
     } else {
-      constexpr int TW = 24;
+      // per row: 8 mean columns (G ≤ 8 used), then 16 variance columns
+      constexpr int TW = 24, VOFF = 8;
+      static_assert(G <= 8 && VOFF + 8 * NT <= TW, "tile columns");
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int c0 = nt * 8 + 2 * t;
-        my_tile[g * TW + c0] = acc[nt][0];
-        my_tile[g * TW + c0 + 1] = acc[nt][1];
-        my_tile[(g + 8) * TW + c0] = acc[nt][2];
-        my_tile[(g + 8) * TW + c0 + 1] = acc[nt][3];
+        if (nt == 0) {
+          my_tile[g * TW + c0] = acc[0][0];
+          my_tile[g * TW + c0 + 1] = acc[0][1];
+          my_tile[(g + 8) * TW + c0] = acc[0][2];
+          my_tile[(g + 8) * TW + c0 + 1] = acc[0][3];
+        }
+        my_tile[g * TW + VOFF + c0] = acv[nt][0];
+        my_tile[g * TW + VOFF + c0 + 1] = acv[nt][1];
+        my_tile[(g + 8) * TW + VOFF + c0] = acv[nt][2];
+        my_tile[(g + 8) * TW + VOFF + c0 + 1] = acv[nt][3];
       }
       __syncwarp();
       for (int pr = lane; pr < 16 * G; pr += 32) {
@@ -638,7 +664,7 @@ __global__ void __launch_bounds__(32 * kDirectWarps, DirectOcc<D, G, GAUSS>::val
         if (r < n) {
           const int p = p0 + r;
           const float m = a.scale * my_tile[r * TW + hh];
-          const float s2 = my_tile[r * TW + G + 2 * hh] + my_tile[r * TW + G + 2 * hh + 1];
+          const float s2 = my_tile[r * TW + VOFF + 2 * hh] + my_tile[r * TW + VOFF + 2 * hh + 1];
           const float sd = a.scale * sqrtf(fmaxf(s2, 0.f));
           const float nv = static_cast<float>(min(a.S, L - p * a.S));
           float mu = a.am1 * m, sg = a.am1 * sd, hat = a.am1 * (m + sd * sqrtf(2.f * logf(nv)));
