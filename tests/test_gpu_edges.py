@@ -12,7 +12,7 @@ from sparse_kv_cache_kmax_b200 import binding as B
 from sparse_kv_cache_kmax_b200.engine import DecodeEngine
 from sparse_kv_cache_kmax_b200.workloads import scaled_down
 
-from gpu_helpers import OUT_TOL, Gpu, gen, np64, oracle_unit, row_rel_err
+from gpu_helpers import OUT_TOL, REL_TIE, Gpu, gen, np64, oracle_unit, row_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -103,6 +103,48 @@ def test_gauss_selection_overflow_is_flagged_and_truncated():
     assert B.ekv_get_error() & B.EKV_EFLAG_SEL_OVERFLOW
     assert torch.all(n == 4)
     assert torch.equal(sel[0, :, :4].cpu(), torch.arange(4, dtype=torch.int32).expand(wl.num_kv_heads, 4))
+
+
+@pytest.mark.parametrize("alpha", [2.0, 1.5, 1.25])
+def test_gauss_point_mass_pages(alpha):
+    """Every other page holds one key in all its tokens (zero spread), aligned
+    with the group's mean query so that those pages carry the top scores.
+    From Jensen's bound the expected mass is then their count (32), the
+    solve's far steps pass every page's mean, where no mass is left, and it
+    must back off and come back from the right: τ̂ and the kept set still
+    match the oracle's bisection.  The other pages drop out of the solve
+    (their spread puts them six σ below τ̂)."""
+    wl = scaled_down("clustered_128k", batch=2, context=1024)
+    inp = gen(wl, 23)
+    G, S = wl.group, wl.page_size
+    kp = inp["k_pool"]
+    for b in range(wl.batch):
+        P = -(-int(inp["seq_lens"][b]) // S)
+        ids = inp["page_table"][b, :P].long()
+        for h in range(wl.num_kv_heads):
+            qbar = inp["q"][b, h * G:(h + 1) * G].float().mean(0)
+            key = 3.0 * wl.head_dim ** 0.5 * qbar / qbar.norm()
+            kp[ids[::2], h] = key.to(kp.dtype)
+    gpu = Gpu(inp)
+    gpu.build_meta()
+    B.ekv_get_error()  # clear what earlier tests left
+    delta = 0.5
+    sel, n, tau_hat = gpu.gauss(alpha, delta)
+    torch.cuda.synchronize()
+    assert B.ekv_get_error() == 0
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            gs = oracle_unit(inp, b, h, policy="gauss", delta=delta, alpha=alpha)["gauss"]
+            t = np64(tau_hat[b, h * G:(h + 1) * G])
+            assert np.allclose(t, gs["tau_hat"], rtol=1e-5, atol=1e-5), (b, h, t, gs["tau_hat"])
+            margin = gs["margin"]
+            band = REL_TIE * np.maximum(1.0, np.abs(gs["tau_hat"] - delta))[:, None]
+            certain_in = np.any(margin > band, axis=0)
+            certain_out = np.all(margin < -band, axis=0)
+            assert certain_in[::2].all()  # the point-mass pages pass by a wide margin
+            got = set(sel[b, h, : int(n[b, h])].cpu().numpy().tolist())
+            assert set(np.nonzero(certain_in)[0].tolist()) <= got, (b, h)
+            assert not (got & set(np.nonzero(certain_out)[0].tolist())), (b, h)
 
 
 def test_fp32_cache_full_size_tiny_config():
