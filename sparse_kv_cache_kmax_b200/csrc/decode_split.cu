@@ -10,7 +10,8 @@
 //     selected slot to an L2-resident scratch.
 //  2. head_warp_kernel, one warp per query head, when the selection holds at
 //     most 512 tokens (below); otherwise head_decode_kernel, one CTA of 256
-//     threads per query head (1024 when streaming): the head's
+//     threads per query head (1024 when streaming; a streaming CTA whose
+//     unit selected at most 128 tokens runs the one-warp path): the head's
 //     scores u = (α−1)·z sit in registers (VPT per thread; above 16384
 //     selected tokens they are read again from L2 at each pass); a 256-bin
 //     histogram of u over (max u − 1, max u] brackets τ from the left (c
@@ -210,6 +211,14 @@ __device__ __forceinline__ V hd_pow_bm1(V w, V beta, int ipow) {
   }
 }
 
+template <int D, int VPL>
+__device__ __forceinline__ void warp_head(const DecodeArgs& a, int G, int row, float* s_p, int* s_i);
+
+// A streamed head whose selection holds at most 32·kHdSmallVpl tokens (a cap
+// far above the selection: the Gaussian policy's cap is a bound, its
+// selections can be a few pages) is done by one warp, with no block barrier.
+constexpr int kHdSmallVpl = 4;
+
 template <int D, int VPT, int THREADS>
 __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int G) {
   constexpr int kHdWarps = THREADS / 32;
@@ -233,6 +242,12 @@ __global__ void __launch_bounds__(THREADS) head_decode_kernel(DecodeArgs a, int 
   // four consecutive tokens per 16-byte load: token 4·((k/4)·THREADS + tid) +
   // k mod 4 (tok(k) gives it)
   constexpr bool kReg = VPT > 0;
+  if constexpr (!kReg) {
+    if (n <= 32 * kHdSmallVpl) {  // uniform over the CTA: the others leave before any barrier
+      if (warp == 0) warp_head<D, kHdSmallVpl>(a, G, row, sh.cu, sh.ci);
+      return;
+    }
+  }
   const int NK = kReg ? VPT : 4 * ((n + 4 * THREADS - 1) / (4 * THREADS));
   auto tok = [&](int k) { return kReg ? k * THREADS + tid : 4 * ((k >> 2) * THREADS + tid) + (k & 3); };
   float uv[kReg ? VPT : 1];
@@ -664,16 +679,12 @@ constexpr int head_warps() {
   return 8;
 }
 
+// Query head `row` by the calling warp alone; s_p, s_i: 32·VPL entries of
+// shared memory that only this warp uses.
 template <int D, int VPL>
-__global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(DecodeArgs a, int G, int rows) {
-  constexpr int kWarps = head_warps<VPL>();
+__device__ __forceinline__ void warp_head(const DecodeArgs& a, int G, int row, float* s_p, int* s_i) {
   constexpr int DPL = D / 32;
-  __shared__ float s_p[kWarps][32 * VPL];
-  __shared__ int s_i[kWarps][32 * VPL];
-  grid_dep_enter();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row = blockIdx.x * kWarps + warp;
-  if (row >= rows) return;  // warp-uniform, and no block barrier follows
+  const int lane = threadIdx.x & 31;
   const int unit = row / G, hg = row - unit * G, b = unit / a.Hkv, kvh = unit % a.Hkv;
   const int S = a.S;
   int L;
@@ -765,8 +776,8 @@ __global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(Decod
     if (a.bits_out && lane == 0 && k < a.words) a.bits_out[orow * a.words + k] = bal;
     if (in) {
       const int at = ns + __popc(bal & ((1u << lane) - 1u));
-      s_p[warp][at] = pow_beta_fast(u[k] - tau, beta, ipow);
-      s_i[warp][at] = i;
+      s_p[at] = pow_beta_fast(u[k] - tau, beta, ipow);
+      s_i[at] = i;
     }
     ns += __popc(bal);
   }
@@ -793,10 +804,10 @@ __global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(Decod
       // exists; an invalid page reads page 0) zeroed after: loads behind
       // per-row branches are issued one after another
       const bool in_list = e < ns;
-      const int tok = s_i[warp][in_list ? e : e0];
+      const int tok = s_i[in_list ? e : e0];
       const int ph = a.ws.sphys[static_cast<size_t>(unit) * a.cap + tok / S];
       const bool in = in_list && ph >= 0;
-      p[r] = in ? s_p[warp][in_list ? e : e0] : 0.f;
+      p[r] = in ? s_p[in_list ? e : e0] : 0.f;
       const bf16* src = static_cast<const bf16*>(a.v_pool) +
                         ((static_cast<size_t>(ph >= 0 ? ph : 0) * a.Hkv + kvh) * S + (tok % S)) * D + lane * DPL;
       if constexpr (DPL == 4) {
@@ -818,6 +829,18 @@ __global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(Decod
   }
 #pragma unroll
   for (int x = 0; x < DPL; ++x) a.out[orow * D + lane * DPL + x] = acc[x];
+}
+
+template <int D, int VPL>
+__global__ void __launch_bounds__(32 * head_warps<VPL>()) head_warp_kernel(DecodeArgs a, int G, int rows) {
+  constexpr int kWarps = head_warps<VPL>();
+  __shared__ float s_p[kWarps][32 * VPL];
+  __shared__ int s_i[kWarps][32 * VPL];
+  grid_dep_enter();
+  const int warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * kWarps + warp;
+  if (row >= rows) return;  // warp-uniform, and no block barrier follows
+  warp_head<D, VPL>(a, G, row, s_p[warp], s_i[warp]);
 }
 
 template <int D>
